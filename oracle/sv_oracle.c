@@ -1,0 +1,568 @@
+/*
+ * sv_oracle.c -- CPU oracle for batched speculative-sampling verification.
+ *
+ * TEST INFRASTRUCTURE ONLY (see sv_oracle.h).  Plain single-threaded C, no
+ * blocking, no fusion, no reordering beyond the definitions it restates.  The
+ * page citations are given per function; readings that the pages leave open
+ * are marked "reading:".
+ *
+ * Parity status of each function:
+ *   svo_philox4x32_10 ...... pinned: published known-answer vectors.
+ *   svo_row_logprobs ....... pinned: scipy log_softmax of the fp32-scaled row.
+ *   svo_row_argmax ......... pinned: numpy argmax.
+ *   svo_residual_logw ...... pinned: exact enumeration (output law == target).
+ *   svo_gumbel_argmax ...... pinned: Monte-Carlo chi-square against softmax.
+ *   svo_verify ............. pinned: exact enumeration, chi-square over 10^6
+ *                            seeded trials, KS gate, acceptance identity,
+ *                            geometric accept-length law, T = 0 argmax law.
+ *   svo_verify_multidraft .. pinned: exact enumeration (K <= 3, L <= 2),
+ *                            chi-square, K = L = 1 equals svo_verify's law,
+ *                            T = 0 longest-argmax-prefix law.
+ */
+#include "sv_oracle.h"
+
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define BERNOULLI_TIE_BAND 1e-6
+#define GUMBEL_TIE_BAND 1e-4
+#define MAX_STEPS 64
+
+/* ------------------------------------------------------------------------
+ * Philox4x32-10 (Salmon et al., SC'11, section 3.3): a 4-word counter is
+ * pushed through 10 rounds; each round multiplies words 0 and 2 by fixed
+ * odd constants, splits the 64-bit products into hi/lo halves, and xors the
+ * hi halves with the other two counter words and the round key.  The key is
+ * bumped by the Weyl constants (golden ratio, sqrt(3)-1) between rounds.
+ * ---------------------------------------------------------------------- */
+static void philox_round(uint32_t c[4], const uint32_t k[2]) {
+  const uint64_t prod0 = (uint64_t)0xD2511F53u * (uint64_t)c[0];
+  const uint64_t prod1 = (uint64_t)0xCD9E8D57u * (uint64_t)c[2];
+  const uint32_t hi0 = (uint32_t)(prod0 >> 32), lo0 = (uint32_t)prod0;
+  const uint32_t hi1 = (uint32_t)(prod1 >> 32), lo1 = (uint32_t)prod1;
+  const uint32_t n0 = hi1 ^ c[1] ^ k[0];
+  const uint32_t n2 = hi0 ^ c[3] ^ k[1];
+  c[0] = n0;
+  c[1] = lo1;
+  c[2] = n2;
+  c[3] = lo0;
+}
+
+void svo_philox4x32_10(const uint32_t ctr[4], const uint32_t key[2], uint32_t out[4]) {
+  uint32_t c[4] = {ctr[0], ctr[1], ctr[2], ctr[3]};
+  uint32_t k[2] = {key[0], key[1]};
+  for (int r = 0; r < 10; ++r) {
+    if (r > 0) {
+      k[0] += 0x9E3779B9u;
+      k[1] += 0xBB67AE85u;
+    }
+    philox_round(c, k);
+  }
+  memcpy(out, c, sizeof c);
+}
+
+/* Keyed stream, reading of "keyed by (seed, step, row, position)": key is the
+ * 64-bit seed, counter words are (c0, b, lo32(step), tag|k|pos). */
+uint32_t svo_stream_word(uint64_t seed, uint64_t step, uint32_t tag, uint32_t b,
+                         uint32_t k, uint32_t pos, uint32_t c0, uint32_t w) {
+  const uint32_t key[2] = {(uint32_t)seed, (uint32_t)(seed >> 32)};
+  const uint32_t ctr[4] = {c0, b, (uint32_t)step, (tag << 24) | (k << 12) | pos};
+  uint32_t out[4];
+  svo_philox4x32_10(ctr, key, out);
+  return out[w & 3u];
+}
+
+double svo_u01_accept(uint32_t x) { return (double)(x >> 8) * 0x1p-24; }
+
+double svo_u01_gumbel(uint32_t x) { return (double)(2u * (x >> 9) + 1u) * 0x1p-24; }
+
+/* ------------------------------------------------------------------------
+ * Row arithmetic.  [FS] Methodology s.1: the temperature is applied to the
+ * logits before the log-softmax, and the arithmetic stays in log space.
+ * ---------------------------------------------------------------------- */
+float svo_bf16_to_f32(uint16_t bits) {
+  const uint32_t w = (uint32_t)bits << 16; /* bf16 is the top half of fp32 */
+  float f;
+  memcpy(&f, &w, sizeof f);
+  return f;
+}
+
+static size_t elem_size(int dtype) { return dtype == SVO_BF16 ? 2u : 4u; }
+
+static float logit_at(const void* row, int64_t v, int dtype) {
+  if (dtype == SVO_BF16) return svo_bf16_to_f32(((const uint16_t*)row)[v]);
+  return ((const float*)row)[v];
+}
+
+typedef struct {
+  float m;     /* max_v fl32(z_v / T)                      */
+  double lnS;  /* ln sum_v exp(fl32(fl32(z_v / T) - m))    */
+} row_stat;
+
+/* s_v = fl32(z_v / T); m = max s_v; S = sum exp(fl32(s_v - m)) in fp64. */
+static int row_stats(const void* row, int64_t V, int dtype, float T, row_stat* st) {
+  float m = -INFINITY;
+  for (int64_t v = 0; v < V; ++v) {
+    const float s = logit_at(row, v, dtype) / T;
+    if (isnan(s)) return -1;
+    if (s > m) m = s;
+  }
+  if (!isfinite(m)) return -1;
+  double S = 0.0;
+  for (int64_t v = 0; v < V; ++v) {
+    const float d = logit_at(row, v, dtype) / T - m;
+    S += exp((double)d);
+  }
+  st->m = m;
+  st->lnS = log(S);
+  return 0;
+}
+
+/* lp_x = fl32(s_x - m) - lnS */
+static double logprob_at(const void* row, int64_t x, int dtype, float T, const row_stat* st) {
+  const float d = logit_at(row, x, dtype) / T - st->m;
+  return (double)d - st->lnS;
+}
+
+int svo_row_logprobs(const void* row, int64_t V, int dtype, float T, double* lp) {
+  row_stat st;
+  if (row_stats(row, V, dtype, T, &st) != 0) return -1;
+  for (int64_t v = 0; v < V; ++v) lp[v] = logprob_at(row, v, dtype, T, &st);
+  return 0;
+}
+
+/* Reading (greedy rows): at T = 0 the target is the point mass on the first
+ * index of the largest raw logit. */
+int64_t svo_row_argmax(const void* row, int64_t V, int dtype) {
+  float best = -INFINITY;
+  int64_t arg = -1;
+  for (int64_t v = 0; v < V; ++v) {
+    const float z = logit_at(row, v, dtype);
+    if (isnan(z)) return -1;
+    if (z > best) {
+      best = z;
+      arg = v;
+    }
+  }
+  if (!isfinite(best)) return -1;
+  return arg;
+}
+
+/* [SSD] s.2 "Saguaro sampling": the correction token is drawn from
+ * r(.) proportional to max(p_target - p_draft, 0); in log space
+ * log r_v = lp_v + log1p(-exp(lq_v - lp_v)) where lp_v > lq_v. */
+int64_t svo_residual_logw(const double* lp, const double* lq, int64_t V, double* out) {
+  int64_t n = 0;
+  for (int64_t v = 0; v < V; ++v) {
+    if (lp[v] > lq[v]) {
+      out[v] = lp[v] + log1p(-exp(lq[v] - lp[v]));
+      ++n;
+    } else {
+      out[v] = -INFINITY;
+    }
+  }
+  return n;
+}
+
+/* Gumbel-max: y = argmax_v (logw_v + G_v), G_v = -ln(-ln U_v), U_v the
+ * keyed Philox uniform for vocabulary entry v (counter word 0 = v >> 2, word
+ * v & 3).  -ln U is evaluated as -log1p(-(1 - U)); 1 - U is exact.  Ties go
+ * to the lowest v.  gap = best - second best score. */
+int64_t svo_gumbel_argmax(const double* logw, int64_t V, uint64_t seed, uint64_t step,
+                          uint32_t tag, uint32_t b, uint32_t pos, double* gap) {
+  double best = -INFINITY, second = -INFINITY;
+  int64_t arg = -1;
+  for (int64_t v = 0; v < V; ++v) {
+    if (logw[v] == -INFINITY) continue;
+    const uint32_t x =
+        svo_stream_word(seed, step, tag, b, 0, pos, (uint32_t)(v >> 2), (uint32_t)(v & 3));
+    const double U = svo_u01_gumbel(x);
+    const double E = -log1p(-(1.0 - U));
+    const double score = logw[v] - log(E);
+    if (arg < 0 || score > best) {
+      second = best;
+      best = score;
+      arg = v;
+    } else if (score > second) {
+      second = score;
+    }
+  }
+  if (gap) *gap = (arg >= 0 && second > -INFINITY) ? best - second : INFINITY;
+  return arg;
+}
+
+/* ------------------------------------------------------------------------
+ * Default randomness: Philox uniforms.
+ * ---------------------------------------------------------------------- */
+typedef struct {
+  uint64_t seed, step;
+} philox_ctx;
+
+static int philox_coin(void* ctx, double h, uint32_t tag, uint32_t b, uint32_t k,
+                       uint32_t pos, double* gap) {
+  const philox_ctx* c = (const philox_ctx*)ctx;
+  const double u = svo_u01_accept(svo_stream_word(c->seed, c->step, tag, b, k, pos, pos, 0));
+  if (gap) *gap = fabs(u - h);
+  return u < h;
+}
+
+static int64_t philox_categorical(void* ctx, const double* logw, int64_t V, uint32_t tag,
+                                  uint32_t b, uint32_t pos, double* gap) {
+  const philox_ctx* c = (const philox_ctx*)ctx;
+  return svo_gumbel_argmax(logw, V, c->seed, c->step, tag, b, pos, gap);
+}
+
+/* ------------------------------------------------------------------------
+ * Single-draft verification.
+ * ---------------------------------------------------------------------- */
+
+/* [FS] s.1: a draft token is accepted when u < min(1, p/q), p/q evaluated
+ * as exp(lp - lq).  Reading for q = 0: p/q = +inf if p > 0 (accept), and
+ * 0/0 rejects. */
+static double accept_prob(double lp, double lq) {
+  if (lq == -INFINITY) return lp == -INFINITY ? 0.0 : 1.0;
+  const double r = exp(lp - lq);
+  return r < 1.0 ? r : 1.0;
+}
+
+static void seq_single(const char* target, const char* draft, const int32_t* tokens,
+                       const float* temps, int gamma, int64_t V, int dtype, int64_t b,
+                       const svo_rng* rng, int32_t* out_accept_len, int32_t* out_tokens,
+                       double* out_lp, double* out_lq, uint8_t* out_tie) {
+  const size_t es = elem_size(dtype);
+  const size_t rowb = (size_t)V * es;
+  const char* trow0 = target + (size_t)b * (size_t)(gamma + 1) * rowb;
+  const char* drow0 = draft + (size_t)b * (size_t)gamma * rowb;
+  const int32_t* x = tokens + (size_t)b * (size_t)gamma;
+  int32_t* tok = out_tokens + (size_t)b * (size_t)(gamma + 1);
+  uint8_t tie = 0;
+
+  for (int i = 0; i <= gamma; ++i) tok[i] = -1;
+  out_accept_len[b] = -1;
+  if (out_lp)
+    for (int i = 0; i < gamma; ++i) out_lp[(size_t)b * gamma + i] = NAN;
+  if (out_lq)
+    for (int i = 0; i < gamma; ++i) out_lq[(size_t)b * gamma + i] = NAN;
+  if (out_tie) out_tie[b] = 0;
+
+  const float T = temps[b];
+  if (!(T >= 0.0f) || isinf(T)) return; /* invalid temperature */
+  for (int i = 0; i < gamma; ++i)
+    if (x[i] < 0 || (int64_t)x[i] >= V) return; /* token outside the vocabulary */
+
+  if (T == 0.0f) {
+    /* Greedy: accept while the draft token equals the target argmax; the
+     * correction (or bonus) token is the target argmax at the stop. */
+    int64_t g[MAX_STEPS + 1];
+    for (int i = 0; i <= gamma; ++i) {
+      g[i] = svo_row_argmax(trow0 + (size_t)i * rowb, V, dtype);
+      if (g[i] < 0) return;
+    }
+    int j = gamma;
+    for (int i = 0; i < gamma; ++i)
+      if ((int64_t)x[i] != g[i]) {
+        j = i;
+        break;
+      }
+    for (int i = 0; i < j; ++i) tok[i] = x[i];
+    tok[j] = (int32_t)g[j];
+    out_accept_len[b] = j;
+    return;
+  }
+
+  row_stat sp[MAX_STEPS + 1], sq[MAX_STEPS];
+  for (int i = 0; i <= gamma; ++i)
+    if (row_stats(trow0 + (size_t)i * rowb, V, dtype, T, &sp[i]) != 0) return;
+  for (int i = 0; i < gamma; ++i)
+    if (row_stats(drow0 + (size_t)i * rowb, V, dtype, T, &sq[i]) != 0) return;
+
+  double lp[MAX_STEPS], lq[MAX_STEPS];
+  for (int i = 0; i < gamma; ++i) {
+    lp[i] = logprob_at(trow0 + (size_t)i * rowb, x[i], dtype, T, &sp[i]);
+    lq[i] = logprob_at(drow0 + (size_t)i * rowb, x[i], dtype, T, &sq[i]);
+  }
+
+  /* Accept/reject in order; [FD] problem definition: the correction token is
+   * drawn at the first rejection point.  Uniforms after it are never used. */
+  int j = gamma;
+  for (int i = 0; i < gamma; ++i) {
+    double gap = INFINITY;
+    const int acc = rng->coin(rng->ctx, accept_prob(lp[i], lq[i]), SVO_TAG_ACCEPT,
+                              (uint32_t)b, 0, (uint32_t)i, &gap);
+    if (gap < BERNOULLI_TIE_BAND) tie |= SVO_TIE_BERNOULLI;
+    if (!acc) {
+      j = i;
+      break;
+    }
+  }
+
+  double* lw = (double*)malloc((size_t)V * sizeof(double));
+  double* lpr = (double*)malloc((size_t)V * sizeof(double));
+  double* lqr = (double*)malloc((size_t)V * sizeof(double));
+  if (!lw || !lpr || !lqr) {
+    free(lw);
+    free(lpr);
+    free(lqr);
+    return;
+  }
+  svo_row_logprobs(trow0 + (size_t)j * rowb, V, dtype, T, lpr);
+  if (j < gamma) {
+    /* Residual max(p_j - q_j, 0).  Reading: if it is identically zero (p_j
+     * == q_j to rounding), draw from p_j. */
+    svo_row_logprobs(drow0 + (size_t)j * rowb, V, dtype, T, lqr);
+    if (svo_residual_logw(lpr, lqr, V, lw) == 0) memcpy(lw, lpr, (size_t)V * sizeof(double));
+  } else {
+    /* Every draft token accepted: bonus token from the target row gamma. */
+    memcpy(lw, lpr, (size_t)V * sizeof(double));
+  }
+  double gap = INFINITY;
+  const int64_t y = rng->categorical(rng->ctx, lw, V, SVO_TAG_GUMBEL, (uint32_t)b, (uint32_t)j, &gap);
+  if (gap < GUMBEL_TIE_BAND) tie |= SVO_TIE_GUMBEL;
+  free(lw);
+  free(lpr);
+  free(lqr);
+
+  for (int i = 0; i < j; ++i) tok[i] = x[i];
+  tok[j] = (int32_t)y;
+  out_accept_len[b] = j;
+  if (out_lp)
+    for (int i = 0; i < gamma; ++i) out_lp[(size_t)b * gamma + i] = lp[i];
+  if (out_lq)
+    for (int i = 0; i < gamma; ++i) out_lq[(size_t)b * gamma + i] = lq[i];
+  if (out_tie) out_tie[b] = tie;
+}
+
+int svo_verify(const void* target, const void* draft, const int32_t* tokens,
+               const float* temps, int64_t B, int gamma, int64_t V, int dtype,
+               uint64_t seed, uint64_t step, int64_t b_begin, int64_t b_end,
+               int32_t* out_accept_len, int32_t* out_tokens, double* out_lp,
+               double* out_lq, uint8_t* out_tie, const svo_rng* rng) {
+  if (!target || !draft || !tokens || !temps || !out_accept_len || !out_tokens) return -1;
+  if (B < 0 || gamma < 1 || gamma > MAX_STEPS || V < 1 || V > ((int64_t)1 << 31)) return -1;
+  if (dtype != SVO_F32 && dtype != SVO_BF16) return -1;
+  if (step >> 32) return -1;
+  if (b_begin < 0 || b_end > B || b_begin > b_end) return -1;
+  philox_ctx pc = {seed, step};
+  svo_rng def = {&pc, philox_coin, philox_categorical};
+  if (!rng) rng = &def;
+  for (int64_t b = b_begin; b < b_end; ++b)
+    seq_single((const char*)target, (const char*)draft, tokens, temps, gamma, V, dtype, b, rng,
+               out_accept_len, out_tokens, out_lp, out_lq, out_tie);
+  return 0;
+}
+
+/* ------------------------------------------------------------------------
+ * Multi-draft verification, [GBV] Algorithm 1.
+ *
+ * Reading (equations 2 and 4 and Algorithm 2 are not printed on the page):
+ *  - Drafts are visited in index order k = 0..K-1.  A draft is considered only
+ *    if its first tau tokens equal the accepted prefix.
+ *  - Sub-block acceptance uses the greedy block-verification weights:
+ *      w_tau = min(1, R(x_tau) / Q~(x_tau)),  w_i = min(1, w_{i-1} P_i(x_i) / Q_i(x_i)),
+ *      h_i = A_i / (A_i + 1 - w_i),  A_i = sum_v max(w_i P_{i+1}(v) - Q_{i+1}(v), 0)
+ *            (h_i = 1 when the denominator is 0; h_{L-1} = w_{L-1}),
+ *    and the longest accepted sub-block wins (tau <- last i+1 with eta_i < h_i).
+ *  - R is the current target law at position tau (P_tau at first).  On an
+ *    advance, R <- norm(max(w P_tau - Q_tau, 0)) (P_L when tau reaches L) and
+ *    H is cleared.  On a rejection the draft's token x_tau joins H and
+ *    R <- norm(max(R - Q~, 0)).
+ *  - Q~ is the draft law at position tau conditioned on not being in H
+ *    (Q_tau restricted to the complement of H, renormalised).  Skipping drafts
+ *    whose token is in H is only distribution-preserving with this
+ *    conditioning; with the unconditioned Q_tau the output law drifts.
+ *  - Finish: the correction token is drawn from R at position tau (the
+ *    target row L when tau == L).
+ * ---------------------------------------------------------------------- */
+static double step_weight(double w, double num, double den) {
+  if (den > 0.0) {
+    const double t = w * (num / den);
+    return t < 1.0 ? t : 1.0;
+  }
+  return (w > 0.0 && num > 0.0) ? 1.0 : 0.0;
+}
+
+static void seq_multi(const char* target, const char* draft, const int32_t* tokens,
+                      const float* temps, int K, int L, int64_t V, int dtype, int64_t b,
+                      const svo_rng* rng, int32_t* out_accept_len, int32_t* out_tokens,
+                      int32_t* out_draft_index, uint8_t* out_tie) {
+  const size_t es = elem_size(dtype);
+  const size_t rowb = (size_t)V * es;
+  const char* trow0 = target + (size_t)b * (size_t)(L + 1) * rowb;
+  const char* drow0 = draft + (size_t)b * (size_t)L * rowb;
+  const int32_t* xs = tokens + (size_t)b * (size_t)K * (size_t)L;
+  int32_t* tok = out_tokens + (size_t)b * (size_t)(L + 1);
+  uint8_t tie = 0;
+
+  for (int i = 0; i <= L; ++i) tok[i] = -1;
+  out_accept_len[b] = -1;
+  if (out_draft_index) out_draft_index[b] = -1;
+  if (out_tie) out_tie[b] = 0;
+
+  const float T = temps[b];
+  if (!(T >= 0.0f) || isinf(T)) return;
+  for (int64_t n = 0; n < (int64_t)K * L; ++n)
+    if (xs[n] < 0 || (int64_t)xs[n] >= V) return;
+
+  if (T == 0.0f) {
+    /* Reading (greedy): the target is the argmax at every position; the
+     * accepted block is the longest draft prefix that matches it (first
+     * draft on ties), and the correction is the argmax at tau. */
+    int64_t g[MAX_STEPS + 1];
+    for (int i = 0; i <= L; ++i) {
+      g[i] = svo_row_argmax(trow0 + (size_t)i * rowb, V, dtype);
+      if (g[i] < 0) return;
+    }
+    int tau = 0, a = -1;
+    for (int k = 0; k < K; ++k) {
+      int n = 0;
+      while (n < L && (int64_t)xs[(size_t)k * L + n] == g[n]) ++n;
+      if (n > tau) {
+        tau = n;
+        a = k;
+      }
+    }
+    for (int i = 0; i < tau; ++i) tok[i] = xs[(size_t)a * L + i];
+    tok[tau] = (int32_t)g[tau];
+    out_accept_len[b] = tau;
+    if (out_draft_index) out_draft_index[b] = a;
+    return;
+  }
+
+  /* Probability vectors P_0..P_L (target) and Q_0..Q_{L-1} (draft). */
+  double* P = (double*)malloc((size_t)(L + 1) * (size_t)V * sizeof(double));
+  double* Q = (double*)malloc((size_t)L * (size_t)V * sizeof(double));
+  double* R = (double*)malloc((size_t)V * sizeof(double));
+  double* lw = (double*)malloc((size_t)V * sizeof(double));
+  unsigned char* inH = (unsigned char*)calloc((size_t)V, 1);
+  int ok = P && Q && R && lw && inH;
+  for (int i = 0; ok && i <= L; ++i)
+    ok = svo_row_logprobs(trow0 + (size_t)i * rowb, V, dtype, T, P + (size_t)i * V) == 0;
+  for (int i = 0; ok && i < L; ++i)
+    ok = svo_row_logprobs(drow0 + (size_t)i * rowb, V, dtype, T, Q + (size_t)i * V) == 0;
+  if (!ok) goto done;
+  for (size_t n = 0; n < (size_t)(L + 1) * (size_t)V; ++n) P[n] = exp(P[n]);
+  for (size_t n = 0; n < (size_t)L * (size_t)V; ++n) Q[n] = exp(Q[n]);
+#define PROW(i) (P + (size_t)(i) * (size_t)V)
+#define QROW(i) (Q + (size_t)(i) * (size_t)V)
+
+  int tau = 0, a = -1;
+  double qH = 0.0; /* Q_tau mass of H */
+  memcpy(R, PROW(0), (size_t)V * sizeof(double));
+
+  for (int k = 0; k < K; ++k) {
+    if (tau == L) break;
+    const int32_t* x = xs + (size_t)k * L;
+    if (tau > 0 && memcmp(x, xs + (size_t)a * L, (size_t)tau * sizeof(int32_t)) != 0) continue;
+    if (inH[x[tau]]) continue; /* rejected sub-block seen before */
+
+    const double keep = 1.0 - qH;
+    const double qfirst = keep > 0.0 ? QROW(tau)[x[tau]] / keep : 0.0;
+    double w = 1.0, wbest = 1.0;
+    int best = tau;
+    for (int i = tau; i < L; ++i) {
+      if (i == tau)
+        w = step_weight(w, R[x[i]], qfirst);
+      else
+        w = step_weight(w, PROW(i)[x[i]], QROW(i)[x[i]]);
+      double h;
+      if (i < L - 1) {
+        double A = 0.0;
+        const double* pn = PROW(i + 1);
+        const double* qn = QROW(i + 1);
+        for (int64_t v = 0; v < V; ++v) {
+          const double t = w * pn[v] - qn[v];
+          if (t > 0.0) A += t;
+        }
+        const double den = A + 1.0 - w;
+        h = den == 0.0 ? 1.0 : A / den;
+      } else {
+        h = w;
+      }
+      double gap = INFINITY;
+      if (rng->coin(rng->ctx, h, SVO_TAG_MD_ETA, (uint32_t)b, (uint32_t)k, (uint32_t)i, &gap)) {
+        best = i + 1;
+        wbest = w;
+      }
+      if (gap < BERNOULLI_TIE_BAND) tie |= SVO_TIE_BERNOULLI;
+    }
+
+    if (best > tau) {
+      tau = best;
+      a = k;
+      memset(inH, 0, (size_t)V);
+      qH = 0.0;
+      if (tau < L) {
+        double Z = 0.0;
+        for (int64_t v = 0; v < V; ++v) {
+          const double t = wbest * PROW(tau)[v] - QROW(tau)[v];
+          R[v] = t > 0.0 ? t : 0.0;
+          Z += R[v];
+        }
+        if (Z > 0.0)
+          for (int64_t v = 0; v < V; ++v) R[v] /= Z;
+        else
+          memcpy(R, PROW(tau), (size_t)V * sizeof(double));
+      }
+    } else {
+      double Z = 0.0;
+      for (int64_t v = 0; v < V; ++v) {
+        const double qt = (inH[v] || keep <= 0.0) ? 0.0 : QROW(tau)[v] / keep;
+        const double t = R[v] - qt;
+        lw[v] = t > 0.0 ? t : 0.0;
+        Z += lw[v];
+      }
+      if (Z > 0.0)
+        for (int64_t v = 0; v < V; ++v) R[v] = lw[v] / Z;
+      inH[x[tau]] = 1;
+      qH += QROW(tau)[x[tau]];
+    }
+  }
+
+  /* [GBV] termination: whole block accepted -> correction from the target
+   * (row L); otherwise from the residual law R at tau. */
+  if (tau == L) {
+    for (int64_t v = 0; v < V; ++v) lw[v] = log(PROW(L)[v]);
+  } else {
+    for (int64_t v = 0; v < V; ++v) lw[v] = R[v] > 0.0 ? log(R[v]) : -INFINITY;
+  }
+  {
+    double gap = INFINITY;
+    const int64_t y =
+        rng->categorical(rng->ctx, lw, V, SVO_TAG_MD_GUMBEL, (uint32_t)b, (uint32_t)tau, &gap);
+    if (gap < GUMBEL_TIE_BAND) tie |= SVO_TIE_GUMBEL;
+    for (int i = 0; i < tau; ++i) tok[i] = xs[(size_t)a * L + i];
+    tok[tau] = (int32_t)y;
+    out_accept_len[b] = tau;
+    if (out_draft_index) out_draft_index[b] = a;
+    if (out_tie) out_tie[b] = tie;
+  }
+#undef PROW
+#undef QROW
+done:
+  free(P);
+  free(Q);
+  free(R);
+  free(lw);
+  free(inH);
+}
+
+int svo_verify_multidraft(const void* target, const void* draft, const int32_t* tokens,
+                          const float* temps, int64_t B, int K, int L, int64_t V,
+                          int dtype, uint64_t seed, uint64_t step, int64_t b_begin,
+                          int64_t b_end, int32_t* out_accept_len, int32_t* out_tokens,
+                          int32_t* out_draft_index, uint8_t* out_tie, const svo_rng* rng) {
+  if (!target || !draft || !tokens || !temps || !out_accept_len || !out_tokens) return -1;
+  if (B < 0 || K < 1 || K > 32 || L < 1 || L > MAX_STEPS || V < 1 || V > ((int64_t)1 << 31))
+    return -1;
+  if (dtype != SVO_F32 && dtype != SVO_BF16) return -1;
+  if (step >> 32) return -1;
+  if (b_begin < 0 || b_end > B || b_begin > b_end) return -1;
+  philox_ctx pc = {seed, step};
+  svo_rng def = {&pc, philox_coin, philox_categorical};
+  if (!rng) rng = &def;
+  for (int64_t b = b_begin; b < b_end; ++b)
+    seq_multi((const char*)target, (const char*)draft, tokens, temps, K, L, V, dtype, b, rng,
+              out_accept_len, out_tokens, out_draft_index, out_tie);
+  return 0;
+}

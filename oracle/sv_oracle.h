@@ -1,0 +1,124 @@
+/*
+ * sv_oracle.h -- CPU oracle for batched speculative-sampling verification.
+ *
+ * TEST INFRASTRUCTURE ONLY.  This is a plain, slow, single-threaded C
+ * restatement of what the verification path computes, used by the tests, by
+ * the package's smoke check and by the benchmark's CPU-baseline leg.  It
+ * shares no code, header, table or constant with the CUDA library; the product
+ * path never links, loads or calls it.
+ *
+ * Sources (page title, section):
+ *   [FS]  "FlashSpec: Adaptive Speculative Decoding with Online Bandit Draft
+ *         Selection and Triton-Optimised Verification", Methodology s.1
+ *         (on-device verification: temperature before log-softmax, log-space
+ *         arithmetic, two log-prob scalars per candidate, on-device
+ *         accept/reject) and s.3 (KS distribution gate).
+ *   [FD]  "FlexDraft", Problem definition (bonus token sampled at the first
+ *         rejection point).
+ *   [SSD] "Speculative Speculative Decoding", Technical summary s.2 "Saguaro
+ *         sampling" (residual r(.) proportional to max(p_target - p_draft, 0)).
+ *   [GBV] "SpecTr-GBV: Multi-Draft Block Verification Accelerating Speculative
+ *         Decoding", Methodology, Algorithm 1 (tau, rejected-sub-block set H,
+ *         per-draft sub-block verification, target/residual correction).
+ *   Philox4x32-10: Salmon, Moraes, Dror, Shaw, "Parallel Random Numbers: As
+ *         Easy as 1, 2, 3", SC'11.
+ *
+ * Floating point: inputs are fp32 or bf16 (bf16 is widened exactly).  The
+ * temperature division and the shift by the row maximum are fp32 operations
+ * (that is how a logit tensor is scaled); every sum, log, exp and ratio after
+ * that is fp64.
+ */
+#ifndef SV_ORACLE_H
+#define SV_ORACLE_H
+
+#include <stdint.h>
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum { SVO_F32 = 0, SVO_BF16 = 1 };
+
+/* Philox counter tags: the 4th counter word is (tag << 24) | (k << 12) | pos. */
+enum {
+  SVO_TAG_ACCEPT = 1,      /* single-draft acceptance uniform             */
+  SVO_TAG_GUMBEL = 2,      /* single-draft residual / bonus Gumbel noise   */
+  SVO_TAG_MD_ETA = 3,      /* multi-draft sub-block acceptance uniform     */
+  SVO_TAG_MD_GUMBEL = 4    /* multi-draft correction Gumbel noise          */
+};
+
+/* Per-sequence tie flags written to out_tie[b]. */
+enum {
+  SVO_TIE_BERNOULLI = 1,   /* some accept decision had |u - h| < 1e-6      */
+  SVO_TIE_GUMBEL = 2       /* the sampled token's top-2 score gap < 1e-4   */
+};
+
+/* ---- Philox4x32-10 and the uniform conversions ------------------------ */
+void svo_philox4x32_10(const uint32_t ctr[4], const uint32_t key[2], uint32_t out[4]);
+/* U[0,1) = (x >> 8) * 2^-24 (accept / eta uniforms). */
+double svo_u01_accept(uint32_t x);
+/* U(0,1) = (2*(x >> 9) + 1) * 2^-24 (Gumbel uniforms; odd multiples of 2^-24). */
+double svo_u01_gumbel(uint32_t x);
+/* Raw 32-bit word of the keyed stream: key = (lo32(seed), hi32(seed)),
+ * counter = (c0, b, lo32(step), (tag<<24)|(k<<12)|pos), word index w in 0..3. */
+uint32_t svo_stream_word(uint64_t seed, uint64_t step, uint32_t tag, uint32_t b,
+                         uint32_t k, uint32_t pos, uint32_t c0, uint32_t w);
+
+/* ---- randomness interface ---------------------------------------------
+ * The verification algorithm draws randomness in exactly two ways: a
+ * Bernoulli(h) event and a draw from a categorical distribution given by
+ * unnormalised log-weights.  The default source (rng == NULL) implements them
+ * with Philox uniforms: u < h, and Gumbel-max.  Tests may substitute another
+ * source (e.g. an exact enumerator).  `gap` receives the tie distance that
+ * the default source measures (|u - h|, or the top-2 score gap); other
+ * sources may leave it untouched. */
+typedef struct svo_rng {
+  void* ctx;
+  int (*coin)(void* ctx, double h, uint32_t tag, uint32_t b, uint32_t k,
+              uint32_t pos, double* gap);
+  int64_t (*categorical)(void* ctx, const double* logw, int64_t V, uint32_t tag,
+                         uint32_t b, uint32_t pos, double* gap);
+} svo_rng;
+
+/* ---- building blocks ------------------------------------------------- */
+float svo_bf16_to_f32(uint16_t bits);
+/* lp[v] = log_softmax(z / T)[v] per the row definition above.  Returns 0, or
+ * -1 when the row maximum is not finite (NaN, +inf, or all -inf). */
+int svo_row_logprobs(const void* row, int64_t V, int dtype, float T, double* lp);
+/* First index of the maximum raw logit (T = 0 rows).  -1 if max not finite. */
+int64_t svo_row_argmax(const void* row, int64_t V, int dtype);
+/* log max(p - q, 0) for each v (unnormalised residual log-weight); -inf where
+ * p <= q.  Returns the number of v with p > q. */
+int64_t svo_residual_logw(const double* lp, const double* lq, int64_t V, double* out);
+/* Default Gumbel-max draw over logw with the keyed Philox stream. */
+int64_t svo_gumbel_argmax(const double* logw, int64_t V, uint64_t seed, uint64_t step,
+                          uint32_t tag, uint32_t b, uint32_t pos, double* gap);
+
+/* ---- single-draft verification ---------------------------------------
+ * target [B, gamma+1, V], draft [B, gamma, V] (dtype), tokens [B, gamma],
+ * temps [B].  Processes sequences b in [b_begin, b_end).  Outputs (indexed
+ * by absolute b): accept_len [B] (-1 for an invalid sequence), tokens
+ * [B, gamma+1] (-1 padded), lp/lq [B, gamma] fp64 (may be NULL; NaN at T = 0
+ * and for invalid sequences), tie [B] flags (may be NULL).  Returns 0, or -1
+ * on a bad argument. */
+int svo_verify(const void* target, const void* draft, const int32_t* tokens,
+               const float* temps, int64_t B, int gamma, int64_t V, int dtype,
+               uint64_t seed, uint64_t step, int64_t b_begin, int64_t b_end,
+               int32_t* out_accept_len, int32_t* out_tokens, double* out_lp,
+               double* out_lq, uint8_t* out_tie, const svo_rng* rng);
+
+/* ---- multi-draft (SpecTr-GBV style) verification ---------------------
+ * target [B, L+1, V], draft [B, L, V] shared by the K drafts, tokens
+ * [B, K, L], temps [B].  Outputs: accept_len [B] (tau, -1 invalid), tokens
+ * [B, L+1], draft_index [B] (-1 when tau == 0; may be NULL), tie [B]. */
+int svo_verify_multidraft(const void* target, const void* draft, const int32_t* tokens,
+                          const float* temps, int64_t B, int K, int L, int64_t V,
+                          int dtype, uint64_t seed, uint64_t step, int64_t b_begin,
+                          int64_t b_end, int32_t* out_accept_len, int32_t* out_tokens,
+                          int32_t* out_draft_index, uint8_t* out_tie, const svo_rng* rng);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SV_ORACLE_H */
