@@ -1,0 +1,442 @@
+#!/usr/bin/env python
+"""Benchmark of batched speculative-sampling verification on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl ours|reference]
+
+One step = one spec_verify (or spec_verify_multidraft) call over one batch
+of a workload: every row statistic, the acceptance decisions and the
+correction/bonus draw.  Metric: verified draft rows per second (B*gamma per
+step; B*K*L for the multi-draft workload), whole job over all ranks.
+
+Timing: inputs are resident in HBM before the timed region; each step reads
+its own input set from a ring of distinct sets whose total size is several
+times the L2 cache, so no step finds its logits in L2.  The K timed steps are
+captured once in a CUDA graph and replayed; CUDA events on the launching
+stream bracket the replay, with a barrier and a synchronize on both sides; the
+max over ranks is reported.  Under torchrun each rank verifies its own batch
+(batch-sharded replicas, no collective on the data path: weak scaling).
+
+e2e: the same metric through the host-buffer entry point of the C ABI: every
+step copies its inputs from pinned host memory to the device, verifies, and
+copies the results back.
+
+--impl reference times the CPU oracle (the reference arm of this build) on the
+host cores, on a bounded sample of each step.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import workloads  # noqa: E402
+
+METRIC = ("verified draft rows/s and achieved HBM GB/s vs B200 peak "
+          "(spec_verify, 1 GPU)")
+UNIT = "rows/s"
+DEFAULT_CONFIG = "c1_b16_g5_v32000_bf16"
+L2_BYTES = 126 * 2**20
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+def _source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "speculative_decoding_verification_85_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode())
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def step_bytes(cfg: workloads.Config, temps: torch.Tensor) -> dict:
+    """Bytes of logits one step must read.
+
+    formula: B (2 gamma + 1) V sizeof + B V sizeof (every row once, plus one
+    residual row per sequence).  algorithmic: the rows the method needs --
+    greedy (T = 0) sequences need only their gamma + 1 target rows and no
+    draw; sampled sequences need all 2 gamma + 1 rows plus one row for the
+    draw.  The algorithmic figure is the one used for the roofline."""
+    es = 2 if cfg.dtype == "bf16" else 4
+    B, g, V = cfg.B, cfg.gamma, cfg.V
+    formula = B * (2 * g + 1) * V * es + B * V * es
+    t = temps.cpu().numpy()
+    greedy = int(np.sum(t == 0.0))
+    sampled = B - greedy
+    algo = (greedy * (g + 1) + sampled * (2 * g + 2)) * V * es
+    return {"formula": formula, "algorithmic": algo}
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap,"
+              "utilization.gpu")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except FileNotFoundError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            time.sleep(0.3)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self) -> dict:
+        rows = []
+        if self.path and os.path.exists(self.path):
+            with open(self.path) as f:
+                for line in f:
+                    p = [x.strip() for x in line.split(",")]
+                    if len(p) >= 10:
+                        rows.append(p)
+            os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return float("nan")
+
+        load = [r for r in rows if num(r[9]) > 0] or rows
+        sm = [num(r[1]) for r in load]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in load for i in range(4)
+                          if r[5 + i].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(num(r[2]) for r in rows),
+                "reasons": reasons, "samples": len(load),
+                "power_w_max": max(num(r[3]) for r in rows)}
+
+
+def _dist_init():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def _barrier(world, local):
+    if world > 1:
+        import torch.distributed as dist
+        if torch.cuda.is_available():
+            dist.barrier(device_ids=[local])
+        else:
+            dist.barrier()
+
+
+def _max_over_ranks(x: float, world: int, device) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def _sum_over_ranks(x: float, world: int, device) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def ring_size(cfg: workloads.Config, total_steps: int) -> int:
+    es = 2 if cfg.dtype == "bf16" else 4
+    per = cfg.B * (2 * cfg.gamma + 1) * cfg.V * es
+    need = max(8, -(-4 * L2_BYTES // per))  # at least 8 sets and 4x the L2 size
+    cap = max(2, int(24e9 // per))          # at most ~24 GB of inputs
+    return int(max(2, min(total_steps, need, cap)))
+
+
+# ------------------------------------------------------------------- oracle
+def time_oracle(cfg, sample_steps: int, threads: int, budget_s: float, rank: int = 0):
+    """Run the oracle on up to `sample_steps` steps (stopping after
+    `budget_s`); return (rows/s, steps done, seconds)."""
+    import oracle
+    done, t_total, rows = 0, 0.0, 0
+    for s in range(sample_steps):
+        st = workloads.make_step(cfg, s + 100000 * rank, device="cpu")
+        tg, dr, tok, tm = workloads.host_inputs(st)
+        t0 = time.perf_counter()
+        if cfg.multidraft:
+            oracle.verify_multidraft(tg, dr, tok, tm, seed=rank, step=s, threads=threads)
+        else:
+            oracle.verify(tg, dr, tok, tm, seed=rank, step=s, threads=threads)
+        t_total += time.perf_counter() - t0
+        rows += cfg.rows_per_step
+        done += 1
+        if t_total >= budget_s:
+            break
+    return rows / t_total, done, t_total
+
+
+def run_reference(args, cfg):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    try:
+        cores = len(os.sched_getaffinity(0))
+    except AttributeError:
+        cores = os.cpu_count() or 1
+    threads = max(1, min(cores, cfg.B))
+    # warm-up steps are untimed
+    time_oracle(cfg, max(0, min(args.warmup, 1)), threads, 1e9)
+    value, done, secs = time_oracle(cfg, args.steps, threads, args.ref_budget)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": done, "warmup": args.warmup, "ms_per_step": 1e3 * secs / done,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": cfg.name, "B": cfg.B, "gamma": cfg.gamma,
+                                        "V": cfg.V, "K": cfg.K or None, "logits": cfg.dtype},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": f"{done} full steps of {cfg.name} (requested {args.steps}), "
+                                   f"sequences split over {threads} host threads"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ GPU arm
+def run_ours(args, cfg):
+    import speculative_decoding_verification_85_b200 as sv
+
+    world, rank, local = _dist_init()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    K, W = args.steps, args.warmup
+    R = ring_size(cfg, K + W)
+    sets = [workloads.make_step(cfg, s + 100000 * rank, device=dev) for s in range(R)]
+    bytes_info = step_bytes(cfg, sets[0].temps)
+    dt = sv.BF16 if cfg.dtype == "bf16" else sv.F32
+    B, g, V = cfg.B, cfg.gamma, cfg.V
+    if cfg.multidraft:
+        ws_bytes = sv.multidraft_workspace_size(B, cfg.K, g, V, dt)
+    else:
+        ws_bytes = sv.workspace_size(B, g, V, dt)
+    ws = torch.zeros(ws_bytes, dtype=torch.uint8, device=dev)
+    outs = [(torch.empty(B, dtype=torch.int32, device=dev),
+             torch.empty((B, g + 1), dtype=torch.int32, device=dev),
+             torch.empty(B, dtype=torch.int32, device=dev)) for _ in range(R)]
+    stream = torch.cuda.Stream(device=dev)
+    seed = rank
+
+    def one(i: int):
+        st = sets[i % R]
+        acc, tok, extra = outs[i % R]
+        if cfg.multidraft:
+            sv.spec_verify_multidraft(st.target, st.draft, st.tokens, st.temps, seed=seed, step=i,
+                                      workspace=ws, out_accept_len=acc, out_tokens=tok,
+                                      out_draft_index=extra, stream=stream)
+        else:
+            sv.spec_verify(st.target, st.draft, st.tokens, st.temps, seed=seed, step=i,
+                           workspace=ws, out_accept_len=acc, out_tokens=tok, stream=stream)
+
+    # warm-up (eager), then capture the K timed steps once
+    with torch.cuda.stream(stream):
+        for i in range(W):
+            one(i)
+    stream.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        for i in range(W, W + K):
+            one(i)
+    launches_per_replay = K * (2 if not cfg.multidraft else 2)
+    with torch.cuda.stream(stream):
+        graph.replay()  # warm the graph itself
+    stream.synchronize()
+
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev.index) as clk:
+        # soak so the clocks sampled below reflect this load
+        t_end = time.time() + args.soak
+        while time.time() < t_end:
+            with torch.cuda.stream(stream):
+                graph.replay()
+            stream.synchronize()
+        _barrier(world, local)
+        torch.cuda.synchronize(dev)
+        with torch.cuda.stream(stream):
+            ev0.record(stream)
+            graph.replay()
+            ev1.record(stream)
+        torch.cuda.synchronize(dev)
+        _barrier(world, local)
+    ms = ev0.elapsed_time(ev1)
+    ms_max = _max_over_ranks(ms, world, dev)
+    clocks = clk.summary()
+
+    # outcome statistics of the timed steps (acceptance rate alpha)
+    acc_all = torch.cat([o[0] for o in outs]).float()
+    valid = acc_all >= 0
+    mean_len = float(acc_all[valid].mean()) if valid.any() else float("nan")
+
+    rows_total = _sum_over_ranks(cfg.rows_per_step * K, world, dev)
+    value = rows_total / (ms_max / 1e3)
+    peak, peak_kind = _peaks()
+    algo_gbs = bytes_info["algorithmic"] / (ms / K / 1e3) / 1e9
+    traffic = None
+    tp = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(tp):
+        try:
+            with open(tp) as f:
+                tj = json.load(f)
+            if tj.get("source_hash") == _source_hash() and tj.get("workload") == cfg.name:
+                traffic = tj.get("bytes_per_launch")
+        except Exception:
+            traffic = None
+
+    # ---- e2e through the host-buffer entry point (single-draft workloads)
+    e2e = None
+    if not cfg.multidraft:
+        staging = torch.zeros(sv.staging_size(B, g, V, dt), dtype=torch.uint8, device=dev)
+        nh = 2
+        host = []
+        for s in range(nh):
+            st = sets[s]
+            host.append([x.cpu().pin_memory() for x in (st.target, st.draft, st.tokens,
+                                                        st.temps)])
+        acc_h = torch.empty(B, dtype=torch.int32, pin_memory=True)
+        tok_h = torch.empty((B, g + 1), dtype=torch.int32, pin_memory=True)
+        for i in range(min(W, 3) + 1):
+            sv.spec_verify_host(*host[i % nh], staging=staging, seed=seed, step=i,
+                                out_accept_len=acc_h, out_tokens=tok_h, stream=stream)
+        ke = K
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        _barrier(world, local)
+        torch.cuda.synchronize(dev)
+        e0.record(stream)
+        for i in range(ke):
+            sv.spec_verify_host(*host[i % nh], staging=staging, seed=seed, step=i,
+                                out_accept_len=acc_h, out_tokens=tok_h, stream=stream)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        _barrier(world, local)
+        ems = _max_over_ranks(e0.elapsed_time(e1), world, dev)
+        es = 2 if cfg.dtype == "bf16" else 4
+        h2d = B * (2 * g + 1) * V * es + B * g * 4 + B * 4
+        d2h = B * 4 + B * (g + 1) * 4
+        e2e = {"value": _sum_over_ranks(cfg.rows_per_step * ke, world, dev) / (ems / 1e3),
+               "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "ms_per_step": ems / ke, "path": "spec_verify_host (pinned host buffers)"}
+
+    # ---- CPU baseline: the oracle on a bounded sample (rank 0, N = 1 only)
+    cpu = None
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        v, done, secs = time_oracle(cfg, args.cpu_steps, 1, args.cpu_budget)
+        cpu = {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle",
+               "sample": f"{done} full steps of {cfg.name}, single-threaded, {secs:.1f} s"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+            "warmup": W, "ms_per_step": ms_max / K, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": cfg.name, "B": cfg.B, "gamma": cfg.gamma, "V": cfg.V,
+                       "K": cfg.K or None, "logits": cfg.dtype,
+                       "inputs": f"ring of {R} distinct resident input sets "
+                                 f"({R * bytes_info['formula'] / 1e9:.2f} GB > L2); "
+                                 "no L2 flush needed",
+                       "launch": "K steps captured in one CUDA graph, replayed",
+                       "parallelism": f"batch-sharded replicas x{world}"},
+            "roofline": {"bound": "hbm", "kernel": "spec_verify step (row pass + draw pass)",
+                         "achieved": algo_gbs, "peak": peak, "unit": "GB/s",
+                         "frac": algo_gbs / peak, "traffic": traffic,
+                         "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)",
+                         "algorithmic_bytes_per_launch": bytes_info["algorithmic"],
+                         "formula_bytes_per_step": bytes_info["formula"],
+                         "formula_gbs": bytes_info["formula"] / (ms / K / 1e3) / 1e9},
+            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches_per_replay,
+            "clocks": clocks,
+            "accept": {"mean_accept_len": mean_len,
+                       "alpha": mean_len / (cfg.gamma if not cfg.multidraft else cfg.gamma)},
+        }
+        print(json.dumps(line), flush=True)
+    del graph
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=None)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default=DEFAULT_CONFIG)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--soak", type=float, default=1.5, help="seconds of untimed load before timing")
+    ap.add_argument("--cpu-steps", type=int, default=200)
+    ap.add_argument("--cpu-budget", type=float, default=10.0)
+    ap.add_argument("--ref-budget", type=float, default=60.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    cfg = workloads.get(args.config)
+    if args.steps is None:
+        args.steps = 1000 if cfg.index in (1, 3) else (200 if cfg.index == 2 else
+                                                         (100 if cfg.index == 4 else 1000))
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args, cfg)
+    else:
+        run_ours(args, cfg)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,18 @@
+"""B200 (sm_100a) batched speculative-sampling verification.
+
+The hot path is the C-ABI library ``libspecverify.so`` (hand-written CUDA
+kernels, ``include/spec_verify.h``); this package is a thin ctypes binding
+that marshals torch tensors (device memory, the current stream) into that ABI.
+It performs no computation of its own and has no CPU fallback: importing it
+without the built library, or calling it on tensors that are not on a CUDA
+device, raises.
+"""
+from ._binding import (  # noqa: F401
+    BF16, F32, SpecVerifyError, Verifier, lib, library_path, multidraft_workspace_size,
+    spec_verify, spec_verify_host, spec_verify_multidraft, staging_size, workspace_size,
+)
+
+__all__ = [
+    "spec_verify", "spec_verify_multidraft", "spec_verify_host", "Verifier", "workspace_size",
+    "multidraft_workspace_size", "staging_size", "SpecVerifyError", "lib", "library_path",
+]

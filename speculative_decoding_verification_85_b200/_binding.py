@@ -1,0 +1,222 @@
+"""ctypes binding of include/spec_verify.h (argument marshalling only)."""
+from __future__ import annotations
+
+import ctypes as C
+import os
+import threading
+
+import torch
+
+F32, BF16 = 0, 1
+_STATUS = {0: "SV_OK", 1: "SV_ERR_INVALID_ARG", 2: "SV_ERR_UNSUPPORTED", 3: "SV_ERR_CUDA",
+           4: "SV_ERR_WORKSPACE"}
+_HERE = os.path.dirname(os.path.abspath(__file__))
+library_path = os.path.join(_HERE, "libspecverify.so")
+
+_lock = threading.Lock()
+_lib = None
+
+
+class SpecVerifyError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{_STATUS.get(status, status)}: {message}")
+        self.status = status
+
+
+def lib() -> C.CDLL:
+    """Load the CUDA library; raise if it has not been built."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(library_path):
+                raise ImportError(
+                    f"{library_path} is missing: build it with "
+                    "`python -m speculative_decoding_verification_85_b200.build`")
+            L = C.CDLL(library_path)
+            vp, i32, u64, sz = C.c_void_p, C.c_int, C.c_uint64, C.c_size_t
+            L.spec_verify_version.restype = i32
+            L.spec_verify_last_error.restype = C.c_char_p
+            L.spec_verify_workspace_size.argtypes = [i32, i32, i32, i32]
+            L.spec_verify_workspace_size.restype = sz
+            L.spec_verify_multidraft_workspace_size.argtypes = [i32, i32, i32, i32, i32]
+            L.spec_verify_multidraft_workspace_size.restype = sz
+            L.spec_verify_workspace_init.argtypes = [vp, sz, vp]
+            L.spec_verify_workspace_init.restype = i32
+            L.spec_verify.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, u64, u64, vp, vp, vp, vp,
+                                      vp, sz, vp]
+            L.spec_verify.restype = i32
+            L.spec_verify_multidraft.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, u64, u64,
+                                                 vp, vp, vp, vp, sz, vp]
+            L.spec_verify_multidraft.restype = i32
+            L.spec_verify_host_staging_size.argtypes = [i32, i32, i32, i32]
+            L.spec_verify_host_staging_size.restype = sz
+            L.spec_verify_host.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, u64, u64, vp, vp,
+                                           vp, vp, vp, sz, vp]
+            L.spec_verify_host.restype = i32
+            _lib = L
+    return _lib
+
+
+def _check(rc: int):
+    if rc != 0:
+        raise SpecVerifyError(rc, lib().spec_verify_last_error().decode())
+
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return BF16
+    if t.dtype == torch.float32:
+        return F32
+    raise TypeError(f"logits must be bfloat16 or float32, got {t.dtype}")
+
+
+def _ptr(t):
+    return None if t is None else C.c_void_p(t.data_ptr())
+
+
+def _dev(t: torch.Tensor, name: str):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (no CPU path)")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _stream(device, stream):
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return C.c_void_p(stream.cuda_stream)
+
+
+def workspace_size(B: int, gamma: int, V: int, dtype: int) -> int:
+    return int(lib().spec_verify_workspace_size(B, gamma, V, dtype))
+
+
+def multidraft_workspace_size(B: int, K: int, L: int, V: int, dtype: int) -> int:
+    return int(lib().spec_verify_multidraft_workspace_size(B, K, L, V, dtype))
+
+
+def staging_size(B: int, gamma: int, V: int, dtype: int) -> int:
+    return int(lib().spec_verify_host_staging_size(B, gamma, V, dtype))
+
+
+def _zeroed(nbytes: int, device) -> torch.Tensor:
+    # 256-byte alignment is guaranteed by the caching allocator for fresh blocks
+    return torch.zeros(max(nbytes, 1), dtype=torch.uint8, device=device)
+
+
+def spec_verify(target, draft, tokens, temps, *, seed: int = 0, step: int = 0, workspace=None,
+                out_accept_len=None, out_tokens=None, out_target_logp=None, out_draft_logp=None,
+                with_logprobs: bool = False, stream=None):
+    """Verify a batch: target [B, g+1, V], draft [B, g, V] (bf16/fp32), tokens
+    [B, g] int32, temps [B] fp32, all on one CUDA device.  Returns
+    (accept_len [B], tokens [B, g+1], target_logp, draft_logp)."""
+    for t, n in ((target, "target"), (draft, "draft"), (tokens, "tokens"), (temps, "temps")):
+        _dev(t, n)
+    B, g1, V = target.shape
+    g = g1 - 1
+    dt = _dt(target)
+    if draft.dtype != target.dtype or tuple(draft.shape) != (B, g, V):
+        raise ValueError("draft must match target's dtype and be [B, gamma, V]")
+    if tokens.dtype != torch.int32 or tuple(tokens.shape) != (B, g):
+        raise ValueError("tokens must be int32 [B, gamma]")
+    if temps.dtype != torch.float32 or tuple(temps.shape) != (B,):
+        raise ValueError("temps must be float32 [B]")
+    dev = target.device
+    if out_accept_len is None:
+        out_accept_len = torch.empty(B, dtype=torch.int32, device=dev)
+    if out_tokens is None:
+        out_tokens = torch.empty((B, g + 1), dtype=torch.int32, device=dev)
+    if with_logprobs and out_target_logp is None:
+        out_target_logp = torch.empty((B, g), dtype=torch.float32, device=dev)
+    if with_logprobs and out_draft_logp is None:
+        out_draft_logp = torch.empty((B, g), dtype=torch.float32, device=dev)
+    if workspace is None:
+        workspace = _zeroed(workspace_size(B, g, V, dt), dev)
+    _check(lib().spec_verify(_ptr(target), _ptr(draft), _ptr(tokens), _ptr(temps), B, g, V, dt,
+                             seed, step, _ptr(out_accept_len), _ptr(out_tokens),
+                             _ptr(out_target_logp), _ptr(out_draft_logp), _ptr(workspace),
+                             workspace.numel() * workspace.element_size(), _stream(dev, stream)))
+    return out_accept_len, out_tokens, out_target_logp, out_draft_logp
+
+
+def spec_verify_multidraft(target, draft, tokens, temps, *, seed: int = 0, step: int = 0,
+                           workspace=None, out_accept_len=None, out_tokens=None,
+                           out_draft_index=None, stream=None):
+    """Multi-draft verification: target [B, L+1, V], draft [B, L, V], tokens
+    [B, K, L] int32, temps [B].  Returns (accept_len, tokens [B, L+1], draft_index)."""
+    for t, n in ((target, "target"), (draft, "draft"), (tokens, "tokens"), (temps, "temps")):
+        _dev(t, n)
+    B, l1, V = target.shape
+    L = l1 - 1
+    K = tokens.shape[1]
+    dt = _dt(target)
+    if draft.dtype != target.dtype or tuple(draft.shape) != (B, L, V):
+        raise ValueError("draft must match target's dtype and be [B, L, V]")
+    if tokens.dtype != torch.int32 or tuple(tokens.shape) != (B, K, L):
+        raise ValueError("tokens must be int32 [B, K, L]")
+    if temps.dtype != torch.float32 or tuple(temps.shape) != (B,):
+        raise ValueError("temps must be float32 [B]")
+    dev = target.device
+    if out_accept_len is None:
+        out_accept_len = torch.empty(B, dtype=torch.int32, device=dev)
+    if out_tokens is None:
+        out_tokens = torch.empty((B, L + 1), dtype=torch.int32, device=dev)
+    if out_draft_index is None:
+        out_draft_index = torch.empty(B, dtype=torch.int32, device=dev)
+    if workspace is None:
+        workspace = _zeroed(multidraft_workspace_size(B, K, L, V, dt), dev)
+    _check(lib().spec_verify_multidraft(_ptr(target), _ptr(draft), _ptr(tokens), _ptr(temps), B,
+                                        K, L, V, dt, seed, step, _ptr(out_accept_len),
+                                        _ptr(out_tokens), _ptr(out_draft_index), _ptr(workspace),
+                                        workspace.numel() * workspace.element_size(),
+                                        _stream(dev, stream)))
+    return out_accept_len, out_tokens, out_draft_index
+
+
+def spec_verify_host(target, draft, tokens, temps, *, staging, seed: int = 0, step: int = 0,
+                     out_accept_len=None, out_tokens=None, stream=None, with_logprobs=False):
+    """spec_verify on host (preferably pinned) CPU tensors through the C ABI's
+    host-buffer entry point; `staging` is a zero-initialised CUDA uint8 tensor
+    of at least staging_size(...) bytes.  Synchronous."""
+    B, g1, V = target.shape
+    g = g1 - 1
+    dt = _dt(target)
+    for t, n in ((target, "target"), (draft, "draft"), (tokens, "tokens"), (temps, "temps")):
+        if t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{n} must be a contiguous host tensor")
+    if out_accept_len is None:
+        out_accept_len = torch.empty(B, dtype=torch.int32, pin_memory=True)
+    if out_tokens is None:
+        out_tokens = torch.empty((B, g + 1), dtype=torch.int32, pin_memory=True)
+    lp = torch.empty((B, g), dtype=torch.float32, pin_memory=True) if with_logprobs else None
+    lq = torch.empty((B, g), dtype=torch.float32, pin_memory=True) if with_logprobs else None
+    _check(lib().spec_verify_host(_ptr(target), _ptr(draft), _ptr(tokens), _ptr(temps), B, g, V,
+                                  dt, seed, step, _ptr(out_accept_len), _ptr(out_tokens),
+                                  _ptr(lp), _ptr(lq), _ptr(staging),
+                                  staging.numel() * staging.element_size(),
+                                  _stream(staging.device, stream)))
+    return out_accept_len, out_tokens, lp, lq
+
+
+class Verifier:
+    """Owns a zero-initialised workspace sized for the largest shape seen."""
+
+    def __init__(self, device=None):
+        self.device = torch.device(device or "cuda")
+        self._ws = None
+
+    def _workspace(self, nbytes):
+        if self._ws is None or self._ws.numel() < nbytes:
+            self._ws = _zeroed(nbytes, self.device)
+        return self._ws
+
+    def verify(self, target, draft, tokens, temps, **kw):
+        B, g1, V = target.shape
+        ws = self._workspace(workspace_size(B, g1 - 1, V, _dt(target)))
+        return spec_verify(target, draft, tokens, temps, workspace=ws, **kw)
+
+    def verify_multidraft(self, target, draft, tokens, temps, **kw):
+        B, l1, V = target.shape
+        ws = self._workspace(multidraft_workspace_size(B, tokens.shape[1], l1 - 1, V,
+                                                       _dt(target)))
+        return spec_verify_multidraft(target, draft, tokens, temps, workspace=ws, **kw)

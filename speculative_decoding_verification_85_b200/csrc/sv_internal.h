@@ -1,0 +1,128 @@
+// sv_internal.h -- shared host/device declarations of the verifier library.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "spec_verify.h"
+
+namespace sv {
+
+constexpr int kP1Threads = 256;   // pass-1 CTA size
+constexpr int kP2Threads = 256;   // pass-2 CTA size
+constexpr int kMdThreads = 1024;  // multi-draft sequential kernel CTA size
+constexpr int kMaxRowsPerSeq = 2 * SV_MAX_GAMMA + 1;
+
+// Pass-1 partial of one (row, chunk): raw max, sum of 2^{(z - max) c}, first
+// argmax index (greedy rows), NaN seen.  16 bytes, stored as one vector.
+struct alignas(16) RowPartial {
+  float m;
+  float s;
+  int arg;
+  int bad;
+};
+
+// Per-sequence hand-off from the decision to pass 2.
+struct alignas(16) SeqInfo {
+  int mode;     // kModeNone / kModeResidual / kModeBonus
+  int j;        // position of the draw
+  float zmp;    // raw max of target row j
+  float zmq;    // raw max of draft row j (residual)
+  float c;      // log2(e) / T
+  float isp;    // 1 / (target row's scaled sum): p_v = 2^{(z_v - zmp) c} isp
+  float isq;    // 1 / (draft row's scaled sum)
+  float pad;
+};
+
+// Pass-2 partial: best exponential-race candidate of one chunk.
+struct alignas(16) RacePartial {
+  float w;
+  float e;
+  int idx;
+  int pad;
+};
+
+struct Pass1Params {
+  const void* target;
+  const void* draft;
+  const int32_t* tokens;
+  const float* temps;
+  int B, gamma, V, nc, rps;  // gamma = L for multi-draft; rps = 2 gamma + 1
+  uint64_t seed;
+  uint32_t step;
+  RowPartial* part;     // [B * rps * nc]
+  unsigned* ticket;     // [B]
+  RowPartial* rowstat;  // [B * rps] combined rows (multi-draft)
+  SeqInfo* info;        // [B] (single-draft)
+  unsigned* flag;       // [B] decision published (fused path), or NULL
+  int32_t* accept_len;
+  int32_t* out_tokens;
+  float* out_lp;
+  float* out_lq;
+};
+
+struct Pass2Params {
+  const void* target;
+  const void* draft;
+  int B, gamma, V, nc2, blocks_per_chunk;
+  uint64_t seed;
+  uint32_t step;
+  const SeqInfo* info;
+  RacePartial* part;  // [B * nc2]
+  unsigned* ticket;   // [B]
+  int32_t* out_tokens;
+};
+
+struct MdParams {
+  const void* target;
+  const void* draft;
+  const int32_t* tokens;
+  const float* temps;
+  int B, K, L, V;
+  uint64_t seed;
+  uint32_t step;
+  const RowPartial* rowstat;  // [B * (2L + 1)]
+  float* R;                   // [B * V] residual law workspace
+  int32_t* accept_len;
+  int32_t* out_tokens;
+  int32_t* out_draft_index;
+};
+
+// Workspace layout of one call.  The arrival counters live in a header of
+// fixed size at offset 0 (one slot per sequence, up to SV_MAX_BATCH), so their
+// position does not depend on the shape: every call leaves them at zero and a
+// later call of any shape finds zeroed counters.
+// Header: [queue head, exited CTAs, error word, pad] then three per-sequence
+// counter arrays (pass-1 arrivals, pass-2 arrivals, decision flags).
+constexpr size_t kHeaderCtl = 256;
+constexpr size_t kHeaderBytes = kHeaderCtl + 3 * static_cast<size_t>(SV_MAX_BATCH) * sizeof(unsigned);
+enum HeaderWord { kHead = 0, kExited = 1, kError = 2 };
+// Error bits recorded in the header's error word.
+constexpr unsigned kErrWaitTimeout = 1u;
+
+struct Layout {
+  size_t ctl, part1, ticket1, info, rowstat, part2, ticket2, flag, resid, total;
+  int nc, nc2;
+};
+
+Layout layout_single(int B, int gamma, int V, int dtype);
+Layout layout_multi(int B, int K, int L, int V, int dtype);
+
+// Host helpers (sv_api.cu).
+int set_error(int status, const char* fmt, ...);
+int check_device();
+int check_launch(const char* what);
+
+// Kernel launchers (sv_single.cu / sv_multi.cu).
+int launch_single(const void* target, const void* draft, const int32_t* tokens,
+                  const float* temps, int B, int gamma, int V, int dtype, uint64_t seed,
+                  uint64_t step, int32_t* out_accept_len, int32_t* out_tokens, float* out_lp,
+                  float* out_lq, void* workspace, const Layout& lay, cudaStream_t stream);
+int launch_multi(const void* target, const void* draft, const int32_t* tokens,
+                 const float* temps, int B, int K, int L, int V, int dtype, uint64_t seed,
+                 uint64_t step, int32_t* out_accept_len, int32_t* out_tokens,
+                 int32_t* out_draft_index, void* workspace, const Layout& lay,
+                 cudaStream_t stream);
+
+}  // namespace sv

@@ -1,0 +1,78 @@
+"""Comparison rules between the CUDA path and the oracle.
+
+- accept_len and every emitted token id must be identical;
+- a sequence whose oracle run logged a Bernoulli tie (|u - h| < 1e-6) is
+  excluded when its accept_len differs (logged, not a mismatch);
+- a sequence whose oracle draw logged a Gumbel near-tie (top-2 gap < 1e-4)
+  is excluded when only the drawn token differs;
+- gathered log-probabilities agree within 1e-5 absolute.
+"""
+from __future__ import annotations
+
+import os
+
+import numpy as np
+
+import oracle
+import workloads
+
+LOGP_ATOL = 1e-5
+
+
+def host_threads() -> int:
+    try:
+        return max(1, len(os.sched_getaffinity(0)))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def run_oracle(st: workloads.Step, seed: int, step: int, threads: int | None = None):
+    tg, dr, tok, tm = workloads.host_inputs(st)
+    th = threads or host_threads()
+    if tok.ndim == 3:
+        return oracle.verify_multidraft(tg, dr, tok, tm, seed=seed, step=step, threads=th)
+    return oracle.verify(tg, dr, tok, tm, seed=seed, step=step, threads=th)
+
+
+def compare(gpu: dict, ora: dict, check_logprobs: bool = True) -> dict:
+    """Return counts; raise AssertionError with details on a real mismatch."""
+    acc_g, tok_g = gpu["accept_len"], gpu["tokens"]
+    acc_o, tok_o, tie = ora["accept_len"], ora["tokens"], ora["tie"]
+    B = acc_o.shape[0]
+    stats = {"rows": B, "bernoulli_ties": 0, "gumbel_ties": 0, "excluded": 0}
+    bad = []
+    for b in range(B):
+        bt = bool(tie[b] & oracle.TIE_BERNOULLI)
+        gt = bool(tie[b] & oracle.TIE_GUMBEL)
+        stats["bernoulli_ties"] += bt
+        stats["gumbel_ties"] += gt
+        if acc_g[b] != acc_o[b]:
+            if bt:
+                stats["excluded"] += 1
+                continue
+            bad.append((b, "accept_len", int(acc_g[b]), int(acc_o[b])))
+            continue
+        if np.array_equal(tok_g[b], tok_o[b]):
+            if "draft_index" in ora and gpu.get("draft_index") is not None:
+                if gpu["draft_index"][b] != ora["draft_index"][b]:
+                    bad.append((b, "draft_index", int(gpu["draft_index"][b]),
+                                int(ora["draft_index"][b])))
+            continue
+        j = int(acc_o[b])
+        same_prefix = j < 0 or np.array_equal(tok_g[b, :j], tok_o[b, :j])
+        only_draw = same_prefix and j >= 0 and np.array_equal(tok_g[b, j + 1:], tok_o[b, j + 1:])
+        if only_draw and gt:
+            stats["excluded"] += 1
+            continue
+        bad.append((b, "tokens", tok_g[b].tolist(), tok_o[b].tolist(), int(tie[b])))
+    if check_logprobs and gpu.get("lp") is not None and ora.get("lp") is not None:
+        for key in ("lp", "lq"):
+            g, o = gpu[key].astype(np.float64), ora[key]
+            fin = np.isfinite(o)
+            assert np.array_equal(fin, np.isfinite(g)), f"{key}: finite pattern differs"
+            if fin.any():
+                err = np.max(np.abs(g[fin] - o[fin]))
+                stats[f"{key}_max_abs_err"] = float(err)
+                assert err <= LOGP_ATOL, f"{key}: max |gpu - oracle| = {err:.3g} > {LOGP_ATOL}"
+    assert not bad, f"{len(bad)} mismatching sequences, first: {bad[:5]}"
+    return stats

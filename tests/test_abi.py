@@ -1,0 +1,63 @@
+"""CPU checks of the C-ABI library: it loads without a GPU and exports every
+function that include/spec_verify.h declares; size queries work; calls fail
+loudly (no CPU fallback) when there is no device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import speculative_decoding_verification_85_b200 as sv
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = []
+    for h in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if h.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", h)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names += re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(\w+)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+def test_library_exports_every_declared_symbol():
+    names = _declared()
+    assert "spec_verify" in names and "spec_verify_multidraft" in names
+    lib = ctypes.CDLL(sv.library_path)
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in include/ but not exported"
+
+
+def test_size_queries():
+    assert sv.lib().spec_verify_version() >> 16 == 1
+    assert sv.workspace_size(256, 4, 151936, sv.BF16) > 0
+    assert sv.workspace_size(1, 0, 10, sv.BF16) == 0      # gamma out of range
+    assert sv.workspace_size(1, 65, 10, sv.BF16) == 0
+    assert sv.workspace_size(1, 4, 10, 7) == 0            # unknown dtype
+    assert sv.multidraft_workspace_size(8, 4, 5, 32000, sv.BF16) > 0
+    assert sv.multidraft_workspace_size(8, 33, 5, 32000, sv.BF16) == 0
+    assert sv.staging_size(16, 5, 32000, sv.BF16) > 16 * 11 * 32000 * 2
+
+
+def test_host_side_argument_errors():
+    L = sv.lib()
+    # B = 0 is a no-op; bad sizes are rejected before any CUDA call
+    assert L.spec_verify(None, None, None, None, 0, 4, 10, 1, 0, 0, None, None, None, None,
+                         None, 0, None) == 0
+    assert L.spec_verify(None, None, None, None, 1, 0, 10, 1, 0, 0, None, None, None, None,
+                         None, 0, None) == 1
+    assert b"draft length" in L.spec_verify_last_error()
+    assert L.spec_verify(None, None, None, None, 1, 4, 10, 1, 0, 2**32, None, None, None,
+                         None, None, 0, None) == 1
+    assert L.spec_verify_multidraft(None, None, None, None, 1, 0, 4, 10, 1, 0, 0, None, None,
+                                    None, None, 0, None) == 1
+
+
+def test_cpu_tensors_rejected():
+    import torch
+    t = torch.zeros(1, 3, 8)
+    with pytest.raises(ValueError, match="CUDA"):
+        sv.spec_verify(t, torch.zeros(1, 2, 8), torch.zeros(1, 2, dtype=torch.int32),
+                       torch.ones(1))
