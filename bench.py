@@ -296,7 +296,9 @@ def run_ours(args, cfg):
     with torch.cuda.graph(graph, stream=stream):
         for i in range(W, W + K):
             one(i)
-    launches_per_replay = K * (2 if not cfg.multidraft else 2)
+    # kernels of this library per step: one fused launch (single draft), or the
+    # row pass plus the sequential verification kernel (multi-draft)
+    launches_per_replay = K * (2 if cfg.multidraft else 1)
     with torch.cuda.stream(stream):
         graph.replay()  # warm the graph itself
     stream.synchronize()
@@ -394,7 +396,9 @@ def run_ours(args, cfg):
                                  "no L2 flush needed",
                        "launch": "K steps captured in one CUDA graph, replayed",
                        "parallelism": f"batch-sharded replicas x{world}"},
-            "roofline": {"bound": "hbm", "kernel": "spec_verify step (row pass + draw pass)",
+            "roofline": {"bound": "hbm",
+                         "kernel": ("pass1_multi_kernel + md_gbv_kernel (whole step)"
+                                    if cfg.multidraft else "fused_single_kernel (one launch per step)"),
                          "achieved": algo_gbs, "peak": peak, "unit": "GB/s",
                          "frac": algo_gbs / peak, "traffic": traffic,
                          "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)",

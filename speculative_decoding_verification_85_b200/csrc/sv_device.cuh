@@ -140,6 +140,14 @@ __device__ __forceinline__ void argmax_merge(float& m, int& a, float m2, int a2)
   }
 }
 
+// Barrier among the first kThreads threads of the block (named barrier 1).
+// Kernels whose CTA has extra warps (a producer warp) use it for the threads
+// that do the reductions; with kThreads == blockDim.x it is a block barrier.
+template <int kThreads>
+__device__ __forceinline__ void block_sync() {
+  asm volatile("bar.sync 1, %0;" ::"n"(kThreads) : "memory");
+}
+
 // Exponential-race candidate (w, E, index): w / E larger wins, ties go to
 // the lower index; w == 0 means "no candidate".
 __device__ __forceinline__ bool race_better(float w, float e, int idx, float bw, float be,
@@ -154,8 +162,9 @@ __device__ __forceinline__ bool race_better(float w, float e, int idx, float bw,
 
 namespace sv {
 
-// Block-wide reduction of exponential-race candidates to thread 0.
-// `scratch` holds kThreads / 32 float4 slots.  Ends with __syncthreads().
+// Block-wide reduction of exponential-race candidates.  The winner is
+// returned to EVERY thread of the block (so a branch on it is uniform and may
+// contain barriers).  `scratch` holds kThreads / 32 float4 slots.
 template <int kThreads>
 __device__ __forceinline__ void race_reduce(float& bw, float& be, int& bi, float4* scratch) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -171,7 +180,7 @@ __device__ __forceinline__ void race_reduce(float& bw, float& be, int& bi, float
     }
   }
   if (lane == 0) scratch[warp] = make_float4(bw, be, __int_as_float(bi), 0.0f);
-  __syncthreads();
+  block_sync<kThreads>();
   if (warp == 0) {
     constexpr int kWarps = kThreads / 32;
     const float4 q = lane < kWarps ? scratch[lane] : make_float4(0.0f, 1.0f, __int_as_float(0x7fffffff), 0.0f);
@@ -189,8 +198,14 @@ __device__ __forceinline__ void race_reduce(float& bw, float& be, int& bi, float
         bi = i2;
       }
     }
+    if (lane == 0) scratch[0] = make_float4(bw, be, __int_as_float(bi), 0.0f);
   }
-  __syncthreads();
+  block_sync<kThreads>();
+  const float4 r = scratch[0];
+  bw = r.x;
+  be = r.y;
+  bi = __float_as_int(r.z);
+  block_sync<kThreads>();  // scratch may be reused right after
 }
 
 // Block-wide fp64 sum, result returned to every thread.  `red` holds 33
@@ -201,7 +216,7 @@ __device__ __forceinline__ double block_sum(double v, double* red) {
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) v += __shfl_down_sync(0xffffffffu, v, off);
   if (lane == 0) red[warp] = v;
-  __syncthreads();
+  block_sync<kThreads>();
   if (warp == 0) {
     constexpr int kWarps = kThreads / 32;
     v = lane < kWarps ? red[lane] : 0.0;
@@ -209,7 +224,7 @@ __device__ __forceinline__ double block_sum(double v, double* red) {
     for (int off = 16; off > 0; off >>= 1) v += __shfl_down_sync(0xffffffffu, v, off);
     if (lane == 0) red[32] = v;
   }
-  __syncthreads();
+  block_sync<kThreads>();
   return red[32];
 }
 
@@ -245,6 +260,11 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "r"(smem_addr(bar)), "r"(parity)
       : "memory");
   return ok != 0;
+}
+// Order this thread's (and, after a barrier, the block's) earlier generic
+// shared-memory accesses before later async-proxy (bulk copy) accesses.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 // Bulk global->shared copy of `bytes` (multiple of 16, both addresses 16-byte
 // aligned) completing on `bar`.  No cluster multicast.

@@ -93,10 +93,13 @@ struct MdParams {
 // fixed size at offset 0 (one slot per sequence, up to SV_MAX_BATCH), so their
 // position does not depend on the shape: every call leaves them at zero and a
 // later call of any shape finds zeroed counters.
-// Header: [queue head, exited CTAs, error word, pad] then three per-sequence
-// counter arrays (pass-1 arrivals, pass-2 arrivals, decision flags).
+// Header: [queue head, exited CTAs, error word, pad] then the per-sequence
+// pass-1 and pass-2 arrival counters and the decision flags; a flag occupies
+// its own 128-byte line (stride kFlagStride words) because CTAs poll it.
 constexpr size_t kHeaderCtl = 256;
-constexpr size_t kHeaderBytes = kHeaderCtl + 3 * static_cast<size_t>(SV_MAX_BATCH) * sizeof(unsigned);
+constexpr int kFlagStride = 32;
+constexpr size_t kHeaderBytes = kHeaderCtl + 2 * static_cast<size_t>(SV_MAX_BATCH) * sizeof(unsigned) +
+                                static_cast<size_t>(SV_MAX_BATCH) * kFlagStride * sizeof(unsigned);
 enum HeaderWord { kHead = 0, kExited = 1, kError = 2 };
 // Error bits recorded in the header's error word.
 constexpr unsigned kErrWaitTimeout = 1u;

@@ -32,7 +32,7 @@ __global__ void __launch_bounds__(kP1Threads) pass1_multi_kernel(Pass1Params p) 
   const int b = rowg / p.rps;
   const int r = rowg - b * p.rps;
   if (!pass1_chunk<kBf16>(p, b, r, chunk)) return;
-  combine_rows(p, b, rows);
+  combine_rows<kP1Threads>(p, b, rows);
   for (int q = threadIdx.x; q < p.rps; q += kP1Threads)
     store_partial(p.rowstat + static_cast<size_t>(b) * p.rps + q, rows[q]);
 }

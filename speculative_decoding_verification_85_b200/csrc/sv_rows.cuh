@@ -177,7 +177,7 @@ __device__ __forceinline__ RowAcc block_reduce_acc(RowAcc a, float c, RowAcc* sc
     acc_merge<kMode>(a, o, c);
   }
   if (lane == 0) scratch[warp] = a;
-  __syncthreads();
+  block_sync<kThreads>();
   if (warp == 0) {
     constexpr int kWarps = kThreads / 32;
     a = lane < kWarps ? scratch[lane] : RowAcc{-INFINITY, 0.0f, 0x7fffffff, 0};
@@ -218,6 +218,7 @@ __device__ __forceinline__ const char* row_ptr(const Pass1Params& p, int b, int 
 
 // Publish a chunk partial and take the sequence's arrival ticket.  Returns
 // true in every thread of the CTA that arrived last for sequence b.
+template <int kThreads>
 __device__ __forceinline__ bool publish_partial(const Pass1Params& p, int b, int r, int chunk,
                                                 const RowAcc& a) {
   __shared__ int last;
@@ -228,7 +229,7 @@ __device__ __forceinline__ bool publish_partial(const Pass1Params& p, int b, int
     last = (t == static_cast<unsigned>(p.rps * p.nc - 1));
     if (last) p.ticket[b] = 0;  // leave the counter at zero for the next call
   }
-  __syncthreads();
+  block_sync<kThreads>();
   if (last) __threadfence();
   return last;
 }
@@ -250,7 +251,7 @@ __device__ __forceinline__ bool pass1_chunk(const Pass1Params& p, int b, int r, 
     scan_chunk<kBf16, kRowArgmax, kP1Threads>(a, rp, p.V, chunk, p.nc, 0.0f);
     a = block_reduce_acc<kRowArgmax, kP1Threads>(a, 0.0f, scratch);
   }
-  return publish_partial(p, b, r, chunk, a);
+  return publish_partial<kP1Threads>(p, b, r, chunk, a);
 }
 
 // The 16-byte-aligned body of chunk `chunk` of a row: vectors [k0, k1)
@@ -300,9 +301,10 @@ __device__ __forceinline__ void scan_staged(RowAcc& a, const char* rp, int V, in
 
 // Combine the nc chunk partials of every row of sequence b into rows[].
 // Called by all threads of the last-arriving CTA.
+template <int kThreads>
 __device__ __forceinline__ void combine_rows(const Pass1Params& p, int b, RowAcc* rows) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  constexpr int kWarps = kP1Threads / 32;
+  constexpr int kWarps = kThreads / 32;
   const float T = __ldg(p.temps + b);
   for (int r = warp; r < p.rps; r += kWarps) {
     const int mode = row_mode(T, r <= p.gamma);
@@ -330,7 +332,7 @@ __device__ __forceinline__ void combine_rows(const Pass1Params& p, int b, RowAcc
     }
     if (lane == 0) rows[r] = a;
   }
-  __syncthreads();
+  block_sync<kThreads>();
 }
 
 }  // namespace sv

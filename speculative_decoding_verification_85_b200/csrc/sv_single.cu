@@ -71,7 +71,7 @@ __device__ __noinline__ void decide_single(const Pass1Params& p, int b, const Ro
       p.info[b].mode = kModeNone;
       if (p.flag) {
         __threadfence();
-        store_release(p.flag + b, 2u);
+        store_release(p.flag + static_cast<size_t>(b) * kFlagStride, 2u);
       }
     }
     return;
@@ -144,7 +144,7 @@ __device__ __noinline__ void decide_single(const Pass1Params& p, int b, const Ro
     p.info[b] = si;
     if (p.flag) {
       __threadfence();
-      store_release(p.flag + b, si.mode == kModeNone ? 2u : 1u);
+      store_release(p.flag + static_cast<size_t>(b) * kFlagStride, si.mode == kModeNone ? 2u : 1u);
     }
   }
 }
@@ -253,15 +253,27 @@ __device__ __forceinline__ void race_block(const Pass2Params& p, const SeqInfo& 
 }
 
 // ------------------------------------------------------- fused single pass
-// One launch per call.  Work items are handed out in queue order through a
-// global counter: all pass-1 chunks of a sequence come before its pass-2
-// chunks (by `lag` sequences), so a CTA that waits for a sequence's decision
-// waits only for items that running CTAs have already taken and that never
-// wait themselves; progress does not depend on how many CTAs are resident.
-// Every wait is bounded in time; on expiry the kernel records an error bit in
-// the workspace header and moves on.
+// One launch per call, warp-specialised.  Work items are handed out in queue
+// order through a global counter: all pass-1 chunks of a sequence come before
+// its pass-2 chunks (by `lag` sequences), so a CTA that waits for a
+// sequence's decision waits only for items that running CTAs have already
+// taken and that never wait themselves; progress does not depend on how many
+// CTAs are resident.
+//
+// In each CTA one producer warp takes items from the queue and, for pass-1
+// chunks, starts a 1-D bulk copy (TMA engine) of the chunk into a ring of
+// kStages shared-memory stages (full/empty mbarriers); eight consumer warps
+// reduce the staged chunk, publish it, make a sequence's decision when they
+// complete it, and run the pass-2 draws.  The producer runs up to kStages items
+// ahead, so the copies of later chunks overlap the consumers' work and their
+// waits.  Every wait is bounded in time; on expiry the kernel records an
+// error bit in the workspace header and stops taking work.
+constexpr int kConsumers = kP1Threads;         // 8 consumer warps
+constexpr int kFusedThreads = kConsumers + 32;  // + 1 producer warp
+constexpr int kStages = 4;
+constexpr uint32_t kStageBytes = 16384;  // one pass-1 chunk body (1024 x 16 B)
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
-static_assert(kP1Threads == kP2Threads, "pass-2 items run in pass-1 sized CTAs");
+static_assert(kP1Threads == kP2Threads, "pass-2 items run on the consumer warps");
 
 struct FusedParams {
   Pass1Params p1;
@@ -309,134 +321,8 @@ __device__ __forceinline__ void map_item(const FusedParams& f, long long q, int&
   x = static_cast<int>(q % c2);
 }
 
-template <bool kBf16>
-__device__ void pass2_item(const FusedParams& f, int b, int chunk, float4* scratch,
-                          unsigned* s_flag, int* s_last) {
-  const Pass2Params& p = f.p2;
-  if (threadIdx.x == 0) {
-    unsigned v = load_acquire(f.p1.flag + b);
-    if (v == 0) {
-      const uint64_t t0 = global_ns();
-      while ((v = load_acquire(f.p1.flag + b)) == 0) {
-        if (global_ns() - t0 > kWaitLimitNs) {
-          atomicOr(f.error, kErrWaitTimeout);
-          v = 3;
-          break;
-        }
-        __nanosleep(100);
-      }
-    }
-    *s_flag = v;
-  }
-  __syncthreads();
-  const unsigned v = *s_flag;
-  float bw = 0.0f, be = 1.0f;
-  int bi = INT_MAX;
-  SeqInfo si{};
-  bool draw = false;
-  const int nblocks = (p.V + 3) / 4;
-  if (v == 1) {
-    const float4* ip = reinterpret_cast<const float4*>(f.p1.info + b);
-    const float4 w0 = __ldcg(ip), w1 = __ldcg(ip + 1);
-    si.mode = __float_as_int(w0.x);
-    si.j = __float_as_int(w0.y);
-    si.zmp = w0.z;
-    si.zmq = w0.w;
-    si.c = w1.x;
-    si.isp = w1.y;
-    si.isq = w1.z;
-    draw = (si.mode == kModeResidual || si.mode == kModeBonus) && si.j >= 0 && si.j <= p.gamma &&
-           !(si.mode == kModeResidual && si.j == p.gamma);
-    if (draw) {
-      const int g0 = chunk * p.blocks_per_chunk;
-      const int g1 = min(nblocks, g0 + p.blocks_per_chunk);
-      race_block<kBf16>(p, si, b, g0, g1, bw, be, bi);
-    }
-  }
-  race_reduce<kP1Threads>(bw, be, bi, scratch);
-  if (threadIdx.x == 0) {
-    RacePartial* pp = p.part + static_cast<size_t>(b) * p.nc2 + chunk;
-    *reinterpret_cast<float4*>(pp) = make_float4(bw, be, __int_as_float(bi), 0.0f);
-    __threadfence();
-    const unsigned t = atomicAdd(p.ticket + b, 1u);
-    *s_last = (t == static_cast<unsigned>(p.nc2 - 1));
-    if (*s_last) p.ticket[b] = 0;
-  }
-  __syncthreads();
-  if (!*s_last) return;
-  __threadfence();
-  if (draw) {
-    bw = 0.0f;
-    be = 1.0f;
-    bi = INT_MAX;
-    for (int q = threadIdx.x; q < p.nc2; q += kP1Threads) {
-      const float4 g = __ldcg(reinterpret_cast<const float4*>(p.part + static_cast<size_t>(b) * p.nc2 + q));
-      if (race_better(g.x, g.y, __float_as_int(g.z), bw, be, bi)) {
-        bw = g.x;
-        be = g.y;
-        bi = __float_as_int(g.z);
-      }
-    }
-    race_reduce<kP1Threads>(bw, be, bi, scratch);
-    if (!(bw > 0.0f)) {
-      si.mode = kModeBonus;  // residual vanished: draw from p_j
-      bw = 0.0f;
-      be = 1.0f;
-      bi = INT_MAX;
-      race_block<kBf16>(p, si, b, 0, nblocks, bw, be, bi);
-      race_reduce<kP1Threads>(bw, be, bi, scratch);
-    }
-    if (threadIdx.x == 0) p.out_tokens[static_cast<size_t>(b) * (p.gamma + 1) + si.j] = bi;
-  }
-  if (threadIdx.x == 0) f.p1.flag[b] = 0u;  // every pass-2 CTA of b has read it
-}
-
-constexpr uint32_t kStageBytes = 16384;  // one pass-1 chunk body (1024 x 16 B)
-
-// Pass-1 items that read logits get their chunk body staged into shared
-// memory by one bulk copy (TMA engine), issued one item ahead.
-struct StagePlan {
-  bool load;       // the item is a pass-1 chunk whose row must be read
-  int b, r, chunk, mode;
-};
-
-template <bool kBf16>
-__device__ __forceinline__ StagePlan plan_item(const FusedParams& f, long long q) {
-  StagePlan s{false, 0, 0, 0, kRowSkip};
-  int kind, b, x;
-  map_item(f, q, kind, b, x);
-  s.b = b;
-  if (kind != 1) {
-    s.r = -1;
-    return s;
-  }
-  s.r = x / f.p1.nc;
-  s.chunk = x - s.r * f.p1.nc;
-  s.mode = row_mode(__ldg(f.p1.temps + b), s.r <= f.p1.gamma);
-  s.load = s.mode != kRowSkip;
-  return s;
-}
-
-// Thread 0: start the copy of item q's chunk body into `buf`.
-template <bool kBf16>
-__device__ __forceinline__ void issue_stage(const FusedParams& f, long long q, uint4* buf,
-                                            uint64_t* bar) {
-  const StagePlan s = plan_item<kBf16>(f, q);
-  if (!s.load) return;
-  bool is_target;
-  const char* rp = row_ptr<kBf16>(f.p1, s.b, s.r, is_target);
-  const ChunkSpan<kBf16> sp(rp, f.p1.V, s.chunk, f.p1.nc);
-  const uint32_t bytes = sp.bytes();
-  if (bytes) {
-    mbar_expect_tx(bar, bytes);
-    bulk_load(buf, sp.body(rp), bytes, bar);
-  } else {
-    mbar_arrive(bar);
-  }
-}
-
 // Wait for phase `parity` of `bar`, at most kWaitLimitNs.
-__device__ __forceinline__ bool wait_stage(uint64_t* bar, uint32_t parity, unsigned* error) {
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned* error) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_ns();
   while (!mbar_try_wait(bar, parity)) {
@@ -446,6 +332,140 @@ __device__ __forceinline__ bool wait_stage(uint64_t* bar, uint32_t parity, unsig
     }
   }
   return true;
+}
+
+template <bool kBf16>
+__device__ void pass2_item(const FusedParams& f, int b, int chunk, float4* scratch,
+                          unsigned* s_flag, int* s_last) {
+  __shared__ SeqInfo s_si;
+  const Pass2Params& p = f.p2;
+  unsigned* flag = f.p1.flag + static_cast<size_t>(b) * kFlagStride;
+  if (threadIdx.x == 0) {
+    unsigned v = load_acquire(flag);
+    if (v == 0) {
+      const uint64_t t0 = global_ns();
+      unsigned nap = 32;
+      while ((v = load_acquire(flag)) == 0) {
+        if (global_ns() - t0 > kWaitLimitNs) {
+          atomicOr(f.error, kErrWaitTimeout);
+          v = 3;
+          break;
+        }
+        __nanosleep(nap);
+        if (nap < 1024) nap *= 2;
+      }
+    }
+    SeqInfo si{};
+    if (v == 1) {
+      const float4* ip = reinterpret_cast<const float4*>(f.p1.info + b);
+      const float4 w0 = __ldcg(ip), w1 = __ldcg(ip + 1);
+      si.mode = __float_as_int(w0.x);
+      si.j = __float_as_int(w0.y);
+      si.zmp = w0.z;
+      si.zmq = w0.w;
+      si.c = w1.x;
+      si.isp = w1.y;
+      si.isq = w1.z;
+      const bool ok = (si.mode == kModeResidual || si.mode == kModeBonus) && si.j >= 0 &&
+                      si.j <= p.gamma && !(si.mode == kModeResidual && si.j == p.gamma);
+      if (!ok) v = 3;
+    }
+    s_si = si;
+    *s_flag = v;
+  }
+  block_sync<kConsumers>();
+  // v and si come from shared memory: every consumer takes the same branches.
+  const unsigned v = *s_flag;
+  SeqInfo si = s_si;
+  const bool draw = (v == 1);
+  float bw = 0.0f, be = 1.0f;
+  int bi = INT_MAX;
+  const int nblocks = (p.V + 3) / 4;
+  if (draw) {
+    const int g0 = chunk * p.blocks_per_chunk;
+    const int g1 = min(nblocks, g0 + p.blocks_per_chunk);
+    race_block<kBf16>(p, si, b, g0, g1, bw, be, bi);
+  }
+  race_reduce<kConsumers>(bw, be, bi, scratch);
+  if (threadIdx.x == 0) {
+    RacePartial* pp = p.part + static_cast<size_t>(b) * p.nc2 + chunk;
+    *reinterpret_cast<float4*>(pp) = make_float4(bw, be, __int_as_float(bi), 0.0f);
+    __threadfence();
+    const unsigned t = atomicAdd(p.ticket + b, 1u);
+    *s_last = (t == static_cast<unsigned>(p.nc2 - 1));
+    if (*s_last) p.ticket[b] = 0;
+  }
+  block_sync<kConsumers>();
+  if (!*s_last) return;
+  __threadfence();
+  if (draw) {
+    bw = 0.0f;
+    be = 1.0f;
+    bi = INT_MAX;
+    for (int q = threadIdx.x; q < p.nc2; q += kConsumers) {
+      const float4 g = __ldcg(reinterpret_cast<const float4*>(p.part + static_cast<size_t>(b) * p.nc2 + q));
+      if (race_better(g.x, g.y, __float_as_int(g.z), bw, be, bi)) {
+        bw = g.x;
+        be = g.y;
+        bi = __float_as_int(g.z);
+      }
+    }
+    race_reduce<kConsumers>(bw, be, bi, scratch);
+    if (!(bw > 0.0f)) {
+      si.mode = kModeBonus;  // residual vanished: draw from p_j
+      bw = 0.0f;
+      be = 1.0f;
+      bi = INT_MAX;
+      race_block<kBf16>(p, si, b, 0, nblocks, bw, be, bi);
+      race_reduce<kConsumers>(bw, be, bi, scratch);
+    }
+    if (threadIdx.x == 0) p.out_tokens[static_cast<size_t>(b) * (p.gamma + 1) + si.j] = bi;
+  }
+  if (threadIdx.x == 0) *flag = 0u;  // every pass-2 CTA of b has read it
+}
+
+struct StagePlan {
+  bool load;  // a pass-1 chunk whose row must be read
+  int b, r, chunk, mode;
+};
+
+template <bool kBf16>
+__device__ __forceinline__ StagePlan plan_item(const FusedParams& f, long long q) {
+  StagePlan s{false, 0, -1, 0, kRowSkip};
+  int kind, b, x;
+  map_item(f, q, kind, b, x);
+  s.b = b;
+  if (kind != 1) {
+    s.chunk = x;
+    return s;
+  }
+  s.r = x / f.p1.nc;
+  s.chunk = x - s.r * f.p1.nc;
+  s.mode = row_mode(__ldg(f.p1.temps + b), s.r <= f.p1.gamma);
+  s.load = s.mode != kRowSkip;
+  return s;
+}
+
+// Producer: publish item q in a stage and start its copy (or just arrive).
+template <bool kBf16>
+__device__ __forceinline__ void produce(const FusedParams& f, long long q, long long total,
+                                        uint4* stage, uint64_t* full) {
+  if (q < total) {
+    const StagePlan s = plan_item<kBf16>(f, q);
+    if (s.load) {
+      bool is_target;
+      const char* rp = row_ptr<kBf16>(f.p1, s.b, s.r, is_target);
+      const ChunkSpan<kBf16> sp(rp, f.p1.V, s.chunk, f.p1.nc);
+      const uint32_t bytes = sp.bytes();
+      if (bytes) {
+        fence_proxy_async_smem();  // the stage was last read through the generic proxy
+        mbar_expect_tx(full, bytes);
+        bulk_load(stage, sp.body(rp), bytes, full);
+        return;
+      }
+    }
+  }
+  mbar_arrive(full);
 }
 
 template <bool kBf16>
@@ -459,83 +479,87 @@ __device__ __forceinline__ bool pass1_staged(const FusedParams& f, const StagePl
     const ChunkSpan<kBf16> sp(rp, p.V, s.chunk, p.nc);
     if (s.mode == kRowLse) {
       const float c = __fdiv_rn(kLog2e, __ldg(p.temps + s.b));
-      scan_staged<kBf16, kRowLse, kP1Threads>(a, rp, p.V, s.chunk, p.nc, sp, sm, c);
-      a = block_reduce_acc<kRowLse, kP1Threads>(a, c, scratch);
+      scan_staged<kBf16, kRowLse, kConsumers>(a, rp, p.V, s.chunk, p.nc, sp, sm, c);
+      a = block_reduce_acc<kRowLse, kConsumers>(a, c, scratch);
     } else {
-      scan_staged<kBf16, kRowArgmax, kP1Threads>(a, rp, p.V, s.chunk, p.nc, sp, sm, 0.0f);
-      a = block_reduce_acc<kRowArgmax, kP1Threads>(a, 0.0f, scratch);
+      scan_staged<kBf16, kRowArgmax, kConsumers>(a, rp, p.V, s.chunk, p.nc, sp, sm, 0.0f);
+      a = block_reduce_acc<kRowArgmax, kConsumers>(a, 0.0f, scratch);
     }
   }
-  return publish_partial(p, s.b, s.r, s.chunk, a);
+  return publish_partial<kConsumers>(p, s.b, s.r, s.chunk, a);
 }
 
 template <bool kBf16>
-__global__ void __launch_bounds__(kP1Threads, 3) fused_single_kernel(FusedParams f) {
-  extern __shared__ __align__(128) uint4 stage[];  // 2 x kStageBytes
-  __shared__ __align__(8) uint64_t bars[2];
+__global__ void __launch_bounds__(kFusedThreads, 2) fused_single_kernel(FusedParams f) {
+  extern __shared__ __align__(128) uint4 stage[];  // kStages x kStageBytes
+  __shared__ __align__(8) uint64_t full[kStages], empty[kStages];
+  __shared__ long long slot[kStages];
   __shared__ RowAcc rows[kMaxRowsPerSeq];
-  __shared__ RowAcc scratch[kP1Threads / 32];
-  __shared__ float4 race_scratch[kP1Threads / 32];
-  __shared__ long long s_item[2];
+  __shared__ RowAcc scratch[kConsumers / 32];
+  __shared__ float4 race_scratch[kConsumers / 32];
   __shared__ unsigned s_flag;
-  __shared__ int s_last, s_abort;
-  uint4* buf[2] = {stage, stage + kStageBytes / 16};
+  __shared__ int s_last;
+  __shared__ volatile int s_abort;
   // Wait for the previous grid in the stream (programmatic dependent launch),
   // then let the next one start launching its CTAs.
   asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;");
   const long long total = f.n1 + f.n2;
-  if (threadIdx.x == 0) {
-    mbar_init(&bars[0], 1);
-    mbar_init(&bars[1], 1);
+  const int tid = threadIdx.x;
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
     mbar_fence_init();
     s_abort = 0;
-    const long long q = static_cast<long long>(atomicAdd(f.head, 1ull));
-    s_item[0] = q;
-    if (q < total) issue_stage<kBf16>(f, q, buf[0], &bars[0]);
   }
   __syncthreads();
-  uint32_t parity[2] = {0u, 0u};
-  int cb = 0;
-  long long cur = s_item[0];
-  while (cur < total) {
-    if (threadIdx.x == 0) {
-      const long long nx = static_cast<long long>(atomicAdd(f.head, 1ull));
-      s_item[cb ^ 1] = nx;
-      if (nx < total) issue_stage<kBf16>(f, nx, buf[cb ^ 1], &bars[cb ^ 1]);
-    }
-    const StagePlan s = plan_item<kBf16>(f, cur);
-    if (s.r >= 0) {
-      if (s.load) {
-        if (threadIdx.x == 0 && !wait_stage(&bars[cb], parity[cb], f.error)) s_abort = 1;
-        __syncthreads();
-        if (s_abort) break;
-        mbar_try_wait(&bars[cb], parity[cb]);  // acquire the staged bytes in every thread
-        parity[cb] ^= 1u;
+
+  if (tid >= kConsumers) {
+    // ---- producer warp (one lane) ----
+    if (tid == kConsumers) {
+      uint32_t emask = (1u << kStages) - 1;  // a fresh barrier's "previous" phase is complete
+      for (int s = 0;; s = (s + 1) % kStages) {
+        if (s_abort || !mbar_wait(&empty[s], (emask >> s) & 1u, f.error)) {
+          s_abort = 1;
+          slot[s] = total;  // let the consumers stop
+          mbar_arrive(&full[s]);
+          break;
+        }
+        emask ^= 1u << s;
+        const long long q = static_cast<long long>(atomicAdd(f.head, 1ull));
+        slot[s] = q;
+        produce<kBf16>(f, q, total, stage + static_cast<size_t>(s) * (kStageBytes / 16), &full[s]);
+        if (q >= total) break;
       }
-      if (pass1_staged<kBf16>(f, s, buf[cb], scratch)) {
-        combine_rows(f.p1, s.b, rows);
-        if (threadIdx.x < 32) decide_single<kBf16>(f.p1, s.b, rows);
+    }
+    return;
+  }
+
+  // ---- consumer warps ----
+  uint32_t fmask = 0u;
+  for (int s = 0;; s = (s + 1) % kStages) {
+    if (tid == 0 && !mbar_wait(&full[s], (fmask >> s) & 1u, f.error)) s_abort = 1;
+    block_sync<kConsumers>();
+    if (s_abort) break;
+    mbar_try_wait(&full[s], (fmask >> s) & 1u);  // acquire the stage in every consumer
+    fmask ^= 1u << s;
+    const long long q = slot[s];
+    if (q >= total) break;
+    const StagePlan pl = plan_item<kBf16>(f, q);
+    if (pl.r >= 0) {
+      if (pass1_staged<kBf16>(f, pl, stage + static_cast<size_t>(s) * (kStageBytes / 16), scratch)) {
+        combine_rows<kConsumers>(f.p1, pl.b, rows);
+        if (tid < 32) decide_single<kBf16>(f.p1, pl.b, rows);
       }
     } else {
-      int kind, b, x;
-      map_item(f, cur, kind, b, x);
-      pass2_item<kBf16>(f, b, x, race_scratch, &s_flag, &s_last);
+      pass2_item<kBf16>(f, pl.b, pl.chunk, race_scratch, &s_flag, &s_last);
     }
-    __syncthreads();
-    cb ^= 1;
-    cur = s_item[cb];
+    block_sync<kConsumers>();  // every consumer is done with stage s
+    if (tid == 0) mbar_arrive(&empty[s]);
   }
-  if (s_abort) {
-    // A staged copy did not arrive in time: drain what is still in flight
-    // (bounded) before the CTA's shared memory is released.
-    if (threadIdx.x == 0) {
-      wait_stage(&bars[0], parity[0], f.error);
-      wait_stage(&bars[1], parity[1], f.error);
-    }
-    __syncthreads();
-  }
-  if (threadIdx.x == 0) {
+  if (tid == 0) {
     const unsigned n = atomicAdd(f.exited, 1u);
     if (n == gridDim.x - 1) {  // last CTA out leaves the queue reset
       *f.head = 0ull;
@@ -553,16 +577,20 @@ std::mutex g_occ_mu;
 
 int resident_ctas(bool bf16) {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148 * 4;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
   std::lock_guard<std::mutex> lk(g_occ_mu);
   Occupancy& o = g_occ[dev];
   if (o.sms == 0) cudaDeviceGetAttribute(&o.sms, cudaDevAttrMultiProcessorCount, dev);
   int& n = o.per_sm[bf16 ? 1 : 0];
   if (n == 0) {
-    if (bf16)
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fused_single_kernel<true>, kP1Threads, 2 * kStageBytes);
-    else
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fused_single_kernel<false>, kP1Threads, 2 * kStageBytes);
+    const int dyn = kStages * static_cast<int>(kStageBytes);
+    if (bf16) {
+      cudaFuncSetAttribute(fused_single_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn);
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fused_single_kernel<true>, kFusedThreads, dyn);
+    } else {
+      cudaFuncSetAttribute(fused_single_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn);
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fused_single_kernel<false>, kFusedThreads, dyn);
+    }
     if (n < 1) n = 1;
   }
   return o.sms * n;
@@ -618,17 +646,19 @@ int launch_single(const void* target, const void* draft, const int32_t* tokens,
   f.n2 = static_cast<long long>(B) * lay.nc2;
   const bool bf16 = dtype == SV_BF16;
   const int S = resident_ctas(bf16);
-  // Pass-2 items of a sequence are queued about one resident wave after its
-  // pass-1 items, so its decision is usually made before they are taken.
-  int lag = S / f.a + 1;
-  f.lag = lag < B ? lag : B;
   const long long items = f.n1 + f.n2;
   const unsigned grid = static_cast<unsigned>(items < S ? items : S);
+  // Pass-2 items of a sequence are queued about one resident wave of items
+  // (every CTA's stages plus the one in hand) after its pass-1 items, so its
+  // decision is usually made before they are taken.
+  const long long inflight = static_cast<long long>(grid) * (kStages + 1);
+  const long long lag = inflight / f.a + 1;
+  f.lag = static_cast<int>(lag < B ? lag : B);
 
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(kP1Threads);
-  cfg.dynamicSmemBytes = 2 * kStageBytes;
+  cfg.blockDim = dim3(kFusedThreads);
+  cfg.dynamicSmemBytes = kStages * kStageBytes;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
