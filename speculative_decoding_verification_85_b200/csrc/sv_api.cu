@@ -24,12 +24,7 @@ int chunks_per_row(int V, int dtype) {
   return nc < 1 ? 1 : nc;
 }
 
-// Pass-2 chunk: 1024 Philox blocks (4096 vocabulary entries) per CTA.
-int chunks_pass2(int V) {
-  const int blocks = (V + 3) / 4;
-  int nc = (blocks + 1023) / 1024;
-  return nc < 1 ? 1 : nc;
-}
+
 
 bool sizes_ok(int B, int g, int V, int dtype) {
   return B >= 0 && B <= SV_MAX_BATCH && g >= 1 && g <= SV_MAX_GAMMA && V >= 1 && (dtype == SV_F32 || dtype == SV_BF16);
@@ -74,23 +69,34 @@ int check_device() {
   return SV_OK;
 }
 
+// Upper bound on the vocabulary segments of a row pair (a segment is at least
+// one 8 KB stage per row; at most 32 segments).
+int max_segments(int V, int dtype) {
+  const long long bytes = static_cast<long long>(V) * (dtype == SV_BF16 ? 2 : 4);
+  long long n = (bytes / 16 + 1 + 511) / 512;
+  if (n < 1) n = 1;
+  if (n > 32) n = 32;
+  return static_cast<int>(n);
+}
+
 Layout layout_single(int B, int gamma, int V, int dtype) {
   Layout l{};
-  l.nc = chunks_per_row(V, dtype);
-  l.nc2 = chunks_pass2(V);
-  const size_t rps = static_cast<size_t>(2 * gamma + 1);
+  l.nc = max_segments(V, dtype);
+  l.nc2 = draw_chunks(V, dtype);
   l.ctl = 0;
   l.ticket1 = kHeaderCtl;
   l.ticket2 = kHeaderCtl + static_cast<size_t>(SV_MAX_BATCH) * sizeof(unsigned);
   l.flag = kHeaderCtl + 2 * static_cast<size_t>(SV_MAX_BATCH) * sizeof(unsigned);
   size_t off = kHeaderBytes;
-  l.part1 = off;
-  off += up(static_cast<size_t>(B) * rps * l.nc * sizeof(RowPartial));
+  l.part1 = off;  // row-pair partials: [B][gamma + 1][nseg] x 2 x 16 bytes
+  off += up(static_cast<size_t>(B) * (gamma + 1) * l.nc * 2 * sizeof(RowPartial));
   l.info = off;
   off += up(static_cast<size_t>(B) * sizeof(SeqInfo));
   l.part2 = off;
   off += up(static_cast<size_t>(B) * l.nc2 * sizeof(RacePartial));
-  l.rowstat = l.resid = 0;
+  l.resid = off;  // the draft tokens' gathered logits: [B][gamma][nseg][2] fp32
+  off += up(static_cast<size_t>(B) * gamma * l.nc * 2 * sizeof(float));
+  l.rowstat = 0;
   l.total = off;
   return l;
 }

@@ -94,6 +94,17 @@ __device__ __forceinline__ unsigned load_acquire(const unsigned* p) {
   asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
   return v;
 }
+// Arrival ticket with release semantics (orders this thread's earlier
+// stores before the increment), and the acquire fence a last arriver takes
+// before reading what the others published.
+__device__ __forceinline__ unsigned ticket_release(unsigned* p) {
+  unsigned old;
+  asm volatile("atom.add.release.gpu.global.u32 %0, [%1], 1;" : "=r"(old) : "l"(p) : "memory");
+  return old;
+}
+__device__ __forceinline__ void fence_acquire() {
+  asm volatile("fence.acq_rel.gpu;" ::: "memory");
+}
 __device__ __forceinline__ uint64_t global_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));

@@ -110,6 +110,7 @@ struct Layout {
 };
 
 Layout layout_single(int B, int gamma, int V, int dtype);
+int draw_chunks(int V, int dtype);  // draw items per sequence (sv_single.cu)
 Layout layout_multi(int B, int K, int L, int V, int dtype);
 
 // Host helpers (sv_api.cu).
