@@ -296,9 +296,10 @@ def run_ours(args, cfg):
     with torch.cuda.graph(graph, stream=stream):
         for i in range(W, W + K):
             one(i)
-    # kernels of this library per step: one fused launch (single draft), or the
-    # row pass plus the sequential verification kernel (multi-draft)
-    launches_per_replay = K * (2 if cfg.multidraft else 1)
+    # kernels of this library per step: the row kernel plus the draw kernel
+    # (single draft), or the row pass plus the sequential verification kernel
+    # (multi-draft)
+    launches_per_replay = K * 2
     with torch.cuda.stream(stream):
         graph.replay()  # warm the graph itself
     stream.synchronize()
@@ -398,7 +399,7 @@ def run_ours(args, cfg):
                        "parallelism": f"batch-sharded replicas x{world}"},
             "roofline": {"bound": "hbm",
                          "kernel": ("pass1_multi_kernel + md_gbv_kernel (whole step)"
-                                    if cfg.multidraft else "fused_single_kernel (one launch per step)"),
+                                    if cfg.multidraft else "rows_kernel + draw_kernel (whole step)"),
                          "achieved": algo_gbs, "peak": peak, "unit": "GB/s",
                          "frac": algo_gbs / peak, "traffic": traffic,
                          "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)",

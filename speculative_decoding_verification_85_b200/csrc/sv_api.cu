@@ -24,8 +24,6 @@ int chunks_per_row(int V, int dtype) {
   return nc < 1 ? 1 : nc;
 }
 
-
-
 bool sizes_ok(int B, int g, int V, int dtype) {
   return B >= 0 && B <= SV_MAX_BATCH && g >= 1 && g <= SV_MAX_GAMMA && V >= 1 && (dtype == SV_F32 || dtype == SV_BF16);
 }
@@ -69,24 +67,13 @@ int check_device() {
   return SV_OK;
 }
 
-// Upper bound on the vocabulary segments of a row pair (a segment is at least
-// one 8 KB stage per row; at most 32 segments).
-int max_segments(int V, int dtype) {
-  const long long bytes = static_cast<long long>(V) * (dtype == SV_BF16 ? 2 : 4);
-  long long n = (bytes / 16 + 1 + 511) / 512;
-  if (n < 1) n = 1;
-  if (n > 32) n = 32;
-  return static_cast<int>(n);
-}
-
 Layout layout_single(int B, int gamma, int V, int dtype) {
   Layout l{};
-  l.nc = max_segments(V, dtype);
+  l.nc = row_segments(V, dtype);
   l.nc2 = draw_chunks(V, dtype);
   l.ctl = 0;
   l.ticket1 = kHeaderCtl;
   l.ticket2 = kHeaderCtl + static_cast<size_t>(SV_MAX_BATCH) * sizeof(unsigned);
-  l.flag = kHeaderCtl + 2 * static_cast<size_t>(SV_MAX_BATCH) * sizeof(unsigned);
   size_t off = kHeaderBytes;
   l.part1 = off;  // row-pair partials: [B][gamma + 1][nseg] x 2 x 16 bytes
   off += up(static_cast<size_t>(B) * (gamma + 1) * l.nc * 2 * sizeof(RowPartial));
@@ -110,7 +97,6 @@ Layout layout_multi(int B, int K, int L, int V, int dtype) {
   l.ctl = 0;
   l.ticket1 = kHeaderCtl;
   l.ticket2 = kHeaderCtl + static_cast<size_t>(SV_MAX_BATCH) * sizeof(unsigned);
-  l.flag = kHeaderCtl + 2 * static_cast<size_t>(SV_MAX_BATCH) * sizeof(unsigned);
   size_t off = kHeaderBytes;
   l.part1 = off;
   off += up(static_cast<size_t>(B) * rps * l.nc * sizeof(RowPartial));

@@ -55,23 +55,10 @@ struct Pass1Params {
   unsigned* ticket;     // [B]
   RowPartial* rowstat;  // [B * rps] combined rows (multi-draft)
   SeqInfo* info;        // [B] (single-draft)
-  unsigned* flag;       // [B] decision published (fused path), or NULL
   int32_t* accept_len;
   int32_t* out_tokens;
   float* out_lp;
   float* out_lq;
-};
-
-struct Pass2Params {
-  const void* target;
-  const void* draft;
-  int B, gamma, V, nc2, blocks_per_chunk;
-  uint64_t seed;
-  uint32_t step;
-  const SeqInfo* info;
-  RacePartial* part;  // [B * nc2]
-  unsigned* ticket;   // [B]
-  int32_t* out_tokens;
 };
 
 struct MdParams {
@@ -93,24 +80,19 @@ struct MdParams {
 // fixed size at offset 0 (one slot per sequence, up to SV_MAX_BATCH), so their
 // position does not depend on the shape: every call leaves them at zero and a
 // later call of any shape finds zeroed counters.
-// Header: [queue head, exited CTAs, error word, pad] then the per-sequence
-// pass-1 and pass-2 arrival counters and the decision flags; a flag occupies
-// its own 128-byte line (stride kFlagStride words) because CTAs poll it.
+// Header: 256 reserved bytes, then the per-sequence row-kernel and
+// draw-kernel arrival counters.
 constexpr size_t kHeaderCtl = 256;
-constexpr int kFlagStride = 32;
-constexpr size_t kHeaderBytes = kHeaderCtl + 2 * static_cast<size_t>(SV_MAX_BATCH) * sizeof(unsigned) +
-                                static_cast<size_t>(SV_MAX_BATCH) * kFlagStride * sizeof(unsigned);
-enum HeaderWord { kHead = 0, kExited = 1, kError = 2 };
-// Error bits recorded in the header's error word.
-constexpr unsigned kErrWaitTimeout = 1u;
+constexpr size_t kHeaderBytes = kHeaderCtl + 2 * static_cast<size_t>(SV_MAX_BATCH) * sizeof(unsigned);
 
 struct Layout {
-  size_t ctl, part1, ticket1, info, rowstat, part2, ticket2, flag, resid, total;
+  size_t ctl, part1, ticket1, info, rowstat, part2, ticket2, resid, total;
   int nc, nc2;
 };
 
 Layout layout_single(int B, int gamma, int V, int dtype);
-int draw_chunks(int V, int dtype);  // draw items per sequence (sv_single.cu)
+int draw_chunks(int V, int dtype);   // bound on draw CTAs per sequence (sv_single.cu)
+int row_segments(int V, int dtype);  // row CTAs per row (sv_single.cu)
 Layout layout_multi(int B, int K, int L, int V, int dtype);
 
 // Host helpers (sv_api.cu).

@@ -1,28 +1,22 @@
-// sv_single.cu -- single-draft verification: one fused, warp-specialised
-// launch per call.
+// sv_single.cu -- single-draft verification: a row kernel and a draw
+// kernel per call, chained by programmatic dependent launch.
 //
-// Row statistics (FlashSpec, Methodology s.1): every target and draft row is
-// streamed once; per row the maximum and the temperature-scaled softmax sum
-// are reduced, and the draft token's two logits are picked up on the way.
-// Decision: the CTA that completes a sequence's rows gathers the two
-// log-probabilities of every draft token, draws the Philox acceptance
-// uniforms and finds the first rejection with a warp ballot (FlexDraft,
-// Problem definition).  Draw (Speculative Speculative Decoding, s.2 Saguaro
-// sampling): the correction token comes from max(p_j - q_j, 0), the bonus
-// token from p_gamma, by an exponential race with Philox noise keyed per
-// vocabulary entry, split over CTAs; the last one combines.
-//
-// Work is handed out in queue order through a global counter: all row items
-// of a sequence come before its draw items (by `lag` sequences), so whoever
-// waits for a sequence's decision waits only for items that running CTAs have
-// already taken and that never wait themselves; progress does not depend on
-// how many CTAs are resident.  In each CTA one producer warp takes items,
-// describes them and stages their logits into a ring of shared-memory stages
-// with 1-D bulk copies (TMA engine); for a draw item it first waits for the
-// sequence's decision.  Eight consumer warps reduce the staged rows, publish
-// per-item partials, make decisions and run the draws from the staged chunks.
-// Every wait is bounded in time; on expiry the kernel records an error bit in
-// the workspace header and stops taking work.
+// Row kernel (FlashSpec, Methodology s.1): one CTA per (sequence, position,
+// vocabulary segment) streams the target row and the draft row of that
+// position over the segment with 16-byte loads issued up front, reduces the
+// maximum and the temperature-scaled softmax sum of both rows, picks up the
+// draft token's two logits, and publishes one partial.  The CTA that
+// completes a sequence (arrival ticket) combines its partials and makes the
+// decision: the two log-probabilities of every draft token, the Philox
+// acceptance uniforms, the first rejection by warp ballot (FlexDraft,
+// Problem definition).
+// Draw kernel (Speculative Speculative Decoding, s.2 Saguaro sampling): once
+// the row kernel has completed (griddepcontrol.wait), one CTA per (sequence,
+// vocabulary chunk) runs the exponential race for the correction token from
+// max(p_j - q_j, 0), or the bonus token from p_gamma, with Philox noise keyed
+// per vocabulary entry; the CTA that completes a sequence combines.
+// Neither kernel waits on another CTA: all ordering is by arrival tickets and
+// by the launch dependency.
 #include <climits>
 #include <mutex>
 
@@ -84,10 +78,6 @@ __device__ __noinline__ void decide_single(const Pass1Params& p, int b, const Ro
     if (lane == 0) {
       p.accept_len[b] = -1;
       p.info[b].mode = kModeNone;
-      if (p.flag) {
-        __threadfence();
-        store_release(p.flag + static_cast<size_t>(b) * kFlagStride, 2u);
-      }
     }
     return;
   }
@@ -160,350 +150,101 @@ __device__ __noinline__ void decide_single(const Pass1Params& p, int b, const Ro
       }
     }
     p.info[b] = si;
-    if (p.flag) {
-      __threadfence();
-      store_release(p.flag + static_cast<size_t>(b) * kFlagStride, si.mode == kModeNone ? 2u : 1u);
-    }
   }
 }
 
 
 // ------------------------------------------------------------------ layout
-constexpr int kConsumers = kP1Threads;          // 8 consumer warps
-constexpr int kFusedThreads = kConsumers + 32;  // + 1 producer warp
-constexpr int kStages = 3;
-constexpr uint32_t kStageBytes = 2 * kStageVec * 16;  // target + draft piece (2 x 16 KB)
-constexpr uint64_t kWaitLimitNs = 2000000000ull;      // 2 s
-static_assert(kP1Threads == kP2Threads, "draw items run on the consumer warps");
+constexpr int kRowThreads = kTileThreads;  // 256
+constexpr int kDrawThreads = kP2Threads;   // 256
+constexpr int kDrawMaxBlocks = 8;          // Philox blocks per thread and draw CTA
+static_assert(kRowThreads == kDrawThreads, "one thread count for both kernels");
+static_assert(kRowThreads == kP1Threads, "row kernel block size");
 
-// Vocabulary entries per draw item: a multiple of 4 (whole Philox blocks)
-// that still fits a stage after rounding out to 16-byte vectors.
-__host__ __device__ constexpr int draw_chunk(bool bf16) {
-  return ((kStageVec - 2) * (bf16 ? 8 : 4)) / 4 * 4;
-}
-
-struct FusedParams {
-  Pass1Params p1;             // inputs, outputs, decision state
-  RacePartial* part2;         // [B][nc2] draw partials
-  unsigned* ticket2;          // [B] draw arrivals
-  int nc2;                    // draw items per sequence
-  unsigned long long* head;   // queue position
-  unsigned* exited;           // CTAs that left the queue
-  unsigned* error;            // error bits
-  long long n1, n2;           // row items / draw items
-  int a;                      // row items per sequence ((gamma + 1) * nseg)
-  int lag;                    // min(lag, B)
-  int nseg;                   // vocabulary segments per row pair
-  float4* pairpart;           // [B][gamma + 1][nseg] x {target, draft} partials
-  float* zx;                  // [B][gamma][nseg][2] draft token's target / draft logit
+struct SingleParams {
+  Pass1Params p1;       // inputs, outputs, decision state
+  RacePartial* part2;   // [B][nc2] draw partials
+  unsigned* ticket2;    // [B] draw arrivals
+  int nc2;              // draw CTAs per sequence
+  int chunk2;           // vocabulary entries per draw CTA (multiple of 4 * kDrawThreads)
+  int nseg;             // row segments per row (gridDim.y of the row kernel)
+  int segvec;           // 16-byte vectors per row segment (multiple of kTileVec)
+  float4* pairpart;     // [B][gamma + 1][nseg] x {target, draft} partials
+  float* zx;            // [B][gamma][nseg][2] draft token's target / draft logit
 };
 
-// Queue position -> (kind, b, x): kind 1 = row item x of sequence b, kind 2 =
-// draw item x of sequence b.  The queue is: row items of sequences [0, lag),
-// then for k = 0..B-lag-1 the row items of sequence k+lag followed by the
-// draw items of sequence k, then the draw items of the last lag sequences.
-__device__ __forceinline__ void map_item(const FusedParams& f, long long q, int& kind, int& b,
-                                         int& x) {
-  const long long a = f.a, c2 = f.nc2, B = f.p1.B, lg = f.lag;
-  if (q < lg * a) {
-    kind = 1;
-    b = static_cast<int>(q / a);
-    x = static_cast<int>(q % a);
-    return;
-  }
-  q -= lg * a;
-  const long long unit = a + c2, nunit = B - lg;
-  if (q < nunit * unit) {
-    const long long k = q / unit, off = q % unit;
-    if (off < a) {
-      kind = 1;
-      b = static_cast<int>(k + lg);
-      x = static_cast<int>(off);
-    } else {
-      kind = 2;
-      b = static_cast<int>(k);
-      x = static_cast<int>(off - a);
-    }
-    return;
-  }
-  q -= nunit * unit;
-  kind = 2;
-  b = static_cast<int>(nunit + q / c2);
-  x = static_cast<int>(q % c2);
-}
-
 template <bool kBf16>
-__device__ __forceinline__ const char* target_row(const FusedParams& f, int b, int i) {
+__device__ __forceinline__ const char* target_row(const Pass1Params& p, int b, int i) {
   constexpr size_t es = kBf16 ? 2 : 4;
-  return static_cast<const char*>(f.p1.target) +
-         (static_cast<size_t>(b) * (f.p1.gamma + 1) + i) * static_cast<size_t>(f.p1.V) * es;
+  return static_cast<const char*>(p.target) +
+         (static_cast<size_t>(b) * (p.gamma + 1) + i) * static_cast<size_t>(p.V) * es;
 }
 template <bool kBf16>
-__device__ __forceinline__ const char* draft_row(const FusedParams& f, int b, int i) {
+__device__ __forceinline__ const char* draft_row(const Pass1Params& p, int b, int i) {
   constexpr size_t es = kBf16 ? 2 : 4;
-  return static_cast<const char*>(f.p1.draft) +
-         (static_cast<size_t>(b) * f.p1.gamma + i) * static_cast<size_t>(f.p1.V) * es;
+  return static_cast<const char*>(p.draft) +
+         (static_cast<size_t>(b) * p.gamma + i) * static_cast<size_t>(p.V) * es;
 }
 
-// Wait for phase `parity` of `bar`, at most kWaitLimitNs.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned* error) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = global_ns();
-  while (!mbar_try_wait(bar, parity)) {
-    if (global_ns() - t0 > kWaitLimitNs) {
-      atomicOr(error, kErrWaitTimeout);
-      return false;
-    }
-  }
-  return true;
+__device__ __forceinline__ void pdl_wait_and_release() {
+  // Wait for the previous grid in the stream (programmatic dependent launch),
+  // then let the next one start launching its CTAs.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;");
 }
 
-// What the producer tells the consumers about one stage; computed once per
-// item, so the consumers do no index arithmetic of their own.
-struct StageDesc {
-  int kind;  // 0 = end of work, 1 = row piece, 2 = draw chunk
-  int b, x;  // sequence; row item: position i; draw item: chunk
-  int t, nst;
-  // row pieces
-  int seg, modeA, loadB, nA, nB, vA, edges, gA, gB, xg;
-  float c;  // log2(e) / T
-  // draw chunks
-  int draw, mode2, j, e0, e1, sbA, sbB, nvA, nvB;
-  float zmp, zmq, isp, isq;
-};
-
-// Producer side of a draw item: wait for the decision, then stage the
-// target (and, for a residual, draft) logits of the chunk.
-template <bool kBf16>
-__device__ __forceinline__ void describe_draw(const FusedParams& f, int b, int chunk,
-                                              StageDesc& d, const char*& rpA, const char*& rpB,
-                                              int& kA, int& kB) {
-  d.draw = 0;
-  rpA = rpB = nullptr;
-  const unsigned* flag = f.p1.flag + static_cast<size_t>(b) * kFlagStride;
-  unsigned v = load_acquire(flag);
-  if (v == 0) {
-    const uint64_t t0 = global_ns();
-    unsigned nap = 32;
-    while ((v = load_acquire(flag)) == 0) {
-      if (global_ns() - t0 > kWaitLimitNs) {
-        atomicOr(f.error, kErrWaitTimeout);
-        return;
-      }
-      __nanosleep(nap);
-      if (nap < 1024) nap *= 2;
-    }
-  }
-  if (v != 1) return;  // greedy or invalid sequence: nothing to draw
-  const float4* ip = reinterpret_cast<const float4*>(f.p1.info + b);
-  const float4 w0 = __ldcg(ip), w1 = __ldcg(ip + 1);
-  const int mode = __float_as_int(w0.x), j = __float_as_int(w0.y);
-  const int g = f.p1.gamma, V = f.p1.V;
-  if (!((mode == kModeResidual && j >= 0 && j < g) || (mode == kModeBonus && j == g))) return;
-  d.draw = 1;
-  d.mode2 = mode;
-  d.j = j;
-  d.zmp = w0.z;
-  d.zmq = w0.w;
-  d.c = w1.x;
-  d.isp = w1.y;
-  d.isq = w1.z;
-  constexpr int kN = Vec16<kBf16>::kN;
-  d.e0 = chunk * draw_chunk(kBf16);
-  d.e1 = min(V, d.e0 + draw_chunk(kBf16));
-  auto span = [&](const char* rp, int& sb, int& nv, int& k0) {
-    const RowGeom<kBf16> gm(rp, V);
-    const int lo = max(d.e0, gm.head), hi = min(d.e1, gm.tail0);
-    if (hi <= lo) {
-      sb = 0;
-      nv = 0;
-      k0 = 0;
-      return;
-    }
-    k0 = (lo - gm.head) / kN;
-    const int k1 = (hi - gm.head + kN - 1) / kN;
-    sb = gm.head + k0 * kN;
-    nv = k1 - k0;
-  };
-  rpA = target_row<kBf16>(f, b, j);
-  span(rpA, d.sbA, d.nvA, kA);
-  if (mode == kModeResidual) {
-    rpB = draft_row<kBf16>(f, b, j);
-    span(rpB, d.sbB, d.nvB, kB);
-  } else {
-    d.nvB = 0;
-  }
-}
-
-// The 4 logits of Philox block g (entries 4g..4g+3) of a draw row: from the
-// staged chunk, or from global memory for entries outside it (a row's
-// unaligned head and tail); entries at or beyond V read as -inf.
-template <bool kBf16>
-__device__ __forceinline__ void draw_block(const uint4* sm, int sb, int nv, const char* rp, int V,
-                                           int g, float (&z)[4]) {
-  constexpr int kN = Vec16<kBf16>::kN;
-  const int v0 = 4 * g;
-  const int off = v0 - sb;
-  if (off >= 0 && off + 4 <= nv * kN && (off & 3) == 0) {
-    if constexpr (kBf16) {
-      const uint2 r = reinterpret_cast<const uint2*>(sm)[off >> 2];
-      z[0] = bf16_lo(r.x);
-      z[1] = bf16_hi(r.x);
-      z[2] = bf16_lo(r.y);
-      z[3] = bf16_hi(r.y);
-    } else {
-      const float4 r = reinterpret_cast<const float4*>(sm)[off >> 2];
-      z[0] = r.x;
-      z[1] = r.y;
-      z[2] = r.z;
-      z[3] = r.w;
-    }
-    return;
-  }
-#pragma unroll
-  for (int w = 0; w < 4; ++w) {
-    const int v = v0 + w, o = v - sb;
-    if (v >= V) {
-      z[w] = -INFINITY;
-    } else if (o >= 0 && o < nv * kN) {
-      if constexpr (kBf16)
-        z[w] = __uint_as_float(static_cast<uint32_t>(reinterpret_cast<const uint16_t*>(sm)[o]) << 16);
-      else
-        z[w] = reinterpret_cast<const float*>(sm)[o];
-    } else {
-      z[w] = logit_at<kBf16>(rp, v);
-    }
-  }
-}
-
-// Exponential race over blocks [g0, g1) (w_v / E_v, E_v = -ln U_v): w =
-// max(p - q, 0) for a residual, w = 2^{(z - max) c} for a bonus.  A
-// candidate is skipped without its logarithm when even the bound
-// E_v >= 1 - U_v cannot beat the current best.
-template <bool kBf16>
-__device__ __forceinline__ void race_staged(const FusedParams& f, const StageDesc& d, int b,
-                                            const uint4* smA, const uint4* smB, int g0, int g1,
-                                            float& bw, float& be, int& bi) {
-  const bool resid = d.mode2 == kModeResidual;
-  const char* rpA = target_row<kBf16>(f, b, d.j);
-  const char* rpB = resid ? draft_row<kBf16>(f, b, d.j) : rpA;
-  const int V = f.p1.V;
-  for (int g = g0 + static_cast<int>(threadIdx.x); g < g1; g += kConsumers) {
-    float zt[4], zd[4];
-    draw_block<kBf16>(smA, d.sbA, d.nvA, rpA, V, g, zt);
-    if (resid) draw_block<kBf16>(smB, d.sbB, d.nvB, rpB, V, g, zd);
-    const uint4 rnd = keyed_block(f.p1.seed, f.p1.step, kTagGumbel, b, 0, d.j, g);
-#pragma unroll
-    for (int w = 0; w < 4; ++w) {
-      float wt = ex2_approx((zt[w] - d.zmp) * d.c);
-      if (resid) wt = wt * d.isp - ex2_approx((zd[w] - d.zmq) * d.c) * d.isq;
-      if (!(wt > 0.0f)) continue;
-      const uint32_t x = word_of(rnd, w);
-      if (bw > 0.0f && wt * be <= bw * gumbel_one_minus_u(x)) continue;
-      const float e = exponential_from_bits(x);
-      const int v = 4 * g + w;
-      if (race_better(wt, e, v, bw, be, bi)) {
-        bw = wt;
-        be = e;
-        bi = v;
-      }
-    }
-  }
-}
-
-// Fallback draw over a whole target row from global memory (the residual
-// vanished: p_j == q_j to rounding), run by the consumers of one CTA.
-template <bool kBf16>
-__device__ void race_row_global(const FusedParams& f, const StageDesc& d, int b, float& bw,
-                                float& be, int& bi) {
-  const char* rp = target_row<kBf16>(f, b, d.j);
-  const int V = f.p1.V;
-  for (int g = threadIdx.x; g < (V + 3) / 4; g += kConsumers) {
-    const uint4 rnd = keyed_block(f.p1.seed, f.p1.step, kTagGumbel, b, 0, d.j, g);
-#pragma unroll
-    for (int w = 0; w < 4; ++w) {
-      const int v = 4 * g + w;
-      if (v >= V) break;
-      const float wt = ex2_approx((logit_at<kBf16>(rp, v) - d.zmp) * d.c);
-      if (!(wt > 0.0f)) continue;
-      const float e = exponential_from_bits(word_of(rnd, w));
-      if (race_better(wt, e, v, bw, be, bi)) {
-        bw = wt;
-        be = e;
-        bi = v;
-      }
-    }
-  }
-}
-
-// Reduce the two rows' accumulators over the consumer threads (one barrier);
-// the result is valid in thread 0.
-__device__ __forceinline__ void reduce_pair(RowAcc& A, RowAcc& B, int modeA, float c,
+// Block reduction of the two rows' accumulators (one barrier); the result is
+// valid in thread 0.
+__device__ __forceinline__ void reduce_pair(RowAcc& A, RowAcc& B, bool argmaxA, float c,
                                             RowAcc* scratch) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) {
-    RowAcc oa, ob;
-    oa.m = __shfl_down_sync(0xffffffffu, A.m, off);
-    oa.s = __shfl_down_sync(0xffffffffu, A.s, off);
-    oa.arg = __shfl_down_sync(0xffffffffu, A.arg, off);
-    oa.bad = __shfl_down_sync(0xffffffffu, A.bad, off);
-    ob.m = __shfl_down_sync(0xffffffffu, B.m, off);
-    ob.s = __shfl_down_sync(0xffffffffu, B.s, off);
-    ob.bad = __shfl_down_sync(0xffffffffu, B.bad, off);
-    ob.arg = 0x7fffffff;
-    if (modeA == kRowArgmax) acc_merge<kRowArgmax>(A, oa, c); else acc_merge<kRowLse>(A, oa, c);
-    acc_merge<kRowLse>(B, ob, c);
-  }
+  warp_merge(A, argmaxA, c);
+  warp_merge(B, false, c);
   if (lane == 0) {
     scratch[2 * warp] = A;
     scratch[2 * warp + 1] = B;
   }
-  block_sync<kConsumers>();
+  block_sync<kRowThreads>();
   if (threadIdx.x == 0) {
-    for (int w = 1; w < kConsumers / 32; ++w) {
-      if (modeA == kRowArgmax) acc_merge<kRowArgmax>(A, scratch[2 * w], c);
-      else acc_merge<kRowLse>(A, scratch[2 * w], c);
-      acc_merge<kRowLse>(B, scratch[2 * w + 1], c);
+    for (int w = 1; w < kRowThreads / 32; ++w) {
+      merge_ref(A, scratch[2 * w], argmaxA, c);
+      merge_ref(B, scratch[2 * w + 1], false, c);
     }
   }
+}
+
+// The softmax sum relative to the row maximum, s = S 2^{R(m) - m c}, from a
+// sum S relative to the reference R(m) (fp64 scaling).
+__device__ __forceinline__ float sum_rel_max(const RowAcc& a, float c) {
+  if (!(a.m > -INFINITY) || isinf(a.m)) return a.s;  // invalid row: left to the decision
+  const double sh = exp2(static_cast<double>(ref_exp(a.m, c)) -
+                         static_cast<double>(a.m) * static_cast<double>(c));
+  return static_cast<float>(static_cast<double>(a.s) * sh);
 }
 
 // Combine the nseg pair partials of every position of sequence b into the
 // row table rows[] (target rows 0..gamma, then draft rows), and pick up the
 // draft tokens' logits (zsel[2i], zsel[2i+1]).
-__device__ __forceinline__ void combine_pairs(const FusedParams& f, int b, RowAcc* rows,
+__device__ __forceinline__ void combine_pairs(const SingleParams& f, int b, RowAcc* rows,
                                               float* zsel) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int g = f.p1.gamma;
   const float T = __ldg(f.p1.temps + b);
-  const int modeA = row_mode(T, true);
-  const float c = modeA == kRowLse ? __fdiv_rn(kLog2e, T) : 0.0f;
-  for (int i = warp; i <= g; i += kConsumers / 32) {
+  const bool argmaxA = row_mode(T, true) == kRowArgmax;
+  const float c = row_mode(T, true) == kRowLse ? __fdiv_rn(kLog2e, T) : 0.0f;
+  for (int i = warp; i <= g; i += kRowThreads / 32) {
     RowAcc A{-INFINITY, 0.0f, 0x7fffffff, 0}, B{-INFINITY, 0.0f, 0x7fffffff, 0};
     const float4* pp = f.pairpart + (static_cast<size_t>(b) * (g + 1) + i) * f.nseg * 2;
     for (int q = lane; q < f.nseg; q += 32) {
       const float4 a = __ldcg(pp + 2 * q), d = __ldcg(pp + 2 * q + 1);
-      const RowAcc oa{a.x, a.y, __float_as_int(a.z), __float_as_int(a.w)};
-      const RowAcc ob{d.x, d.y, __float_as_int(d.z), __float_as_int(d.w)};
-      if (modeA == kRowArgmax) acc_merge<kRowArgmax>(A, oa, c); else acc_merge<kRowLse>(A, oa, c);
-      acc_merge<kRowLse>(B, ob, c);
+      merge_ref(A, RowAcc{a.x, a.y, __float_as_int(a.z), __float_as_int(a.w)}, argmaxA, c);
+      merge_ref(B, RowAcc{d.x, d.y, __float_as_int(d.z), __float_as_int(d.w)}, false, c);
     }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-      RowAcc oa, ob;
-      oa.m = __shfl_down_sync(0xffffffffu, A.m, off);
-      oa.s = __shfl_down_sync(0xffffffffu, A.s, off);
-      oa.arg = __shfl_down_sync(0xffffffffu, A.arg, off);
-      oa.bad = __shfl_down_sync(0xffffffffu, A.bad, off);
-      ob.m = __shfl_down_sync(0xffffffffu, B.m, off);
-      ob.s = __shfl_down_sync(0xffffffffu, B.s, off);
-      ob.bad = __shfl_down_sync(0xffffffffu, B.bad, off);
-      ob.arg = 0x7fffffff;
-      if (modeA == kRowArgmax) acc_merge<kRowArgmax>(A, oa, c); else acc_merge<kRowLse>(A, oa, c);
-      acc_merge<kRowLse>(B, ob, c);
-    }
+    warp_merge(A, argmaxA, c);
+    warp_merge(B, false, c);
     if (lane == 0) {
+      if (!argmaxA) A.s = sum_rel_max(A, c);
+      B.s = sum_rel_max(B, c);
       rows[i] = A;
       if (i < g) rows[g + 1 + i] = B;
     }
@@ -529,356 +270,379 @@ __device__ __forceinline__ void combine_pairs(const FusedParams& f, int b, RowAc
       }
     }
   }
-  block_sync<kConsumers>();
+  block_sync<kRowThreads>();
 }
 
+// Head (entries before the first 16-byte boundary) and tail (after the last)
+// of a row, read as scalars by the first / last segment's CTA.
 template <bool kBf16>
-__device__ __forceinline__ void row_edges(const FusedParams& f, const char* rp, int mode, float c,
-                                          bool head, bool tail, int xg, float* zx, RunAcc& acc) {
-  const RowGeom<kBf16> g(rp, f.p1.V);
+__device__ __forceinline__ void row_edges(const char* rp, int V, const RowGeom<kBf16>& g, bool argmax,
+                                          float c, bool head, bool tail, int xg, float* zx,
+                                          RunAcc& acc) {
   const int tid = threadIdx.x;
   if (head)
-    for (int v = tid; v < g.head; v += kConsumers) {
+    for (int v = tid; v < g.head; v += kRowThreads) {
       const float z = logit_at<kBf16>(rp, v);
       if (v == xg) *zx = z;
-      if (mode == kRowLse) lse_scalar(acc, z, c); else argmax_scalar(acc, z, v);
+      if (argmax) argmax_scalar(acc, z, v); else lse_scalar(acc, z, c);
     }
   if (tail)
-    for (int v = g.tail0 + tid; v < f.p1.V; v += kConsumers) {
+    for (int v = g.tail0 + tid; v < V; v += kRowThreads) {
       const float z = logit_at<kBf16>(rp, v);
       if (v == xg) *zx = z;
-      if (mode == kRowLse) lse_scalar(acc, z, c); else argmax_scalar(acc, z, v);
+      if (argmax) argmax_scalar(acc, z, v); else lse_scalar(acc, z, c);
     }
 }
 
-// ----------------------------------------------------------------- kernel
+// The body vector that holds entry xg of a row, if this thread loads it within
+// the segment [k0, k1); -1 otherwise.
 template <bool kBf16>
-__global__ void __launch_bounds__(kFusedThreads, 2) fused_single_kernel(FusedParams f) {
-  extern __shared__ __align__(128) uint4 stage[];  // kStages x (2 x kStageVec) vectors
-  __shared__ __align__(8) uint64_t full[kStages], empty[kStages];
-  __shared__ StageDesc desc[kStages];
+__device__ __forceinline__ int owned_vector(const RowGeom<kBf16>& g, int xg, int k0, int k1) {
+  if (xg < g.head || xg >= g.tail0) return -1;
+  const int k = (xg - g.head) / Vec16<kBf16>::kN;
+  if (k < k0 || k >= k1 || (k - k0) % kRowThreads != static_cast<int>(threadIdx.x)) return -1;
+  return k;
+}
+
+template <bool kBf16>
+__device__ __forceinline__ void pick_logit(const uint4 (&r)[kTileRegs], int own, int kb, int xg,
+                                           const RowGeom<kBf16>& g, float* zx) {
+  if (own < kb || own >= kb + kTileVec) return;
+  const int j = (own - kb) / kRowThreads;
+  const int e = (xg - g.head) % Vec16<kBf16>::kN;
+#pragma unroll
+  for (int q = 0; q < kTileRegs; ++q)  // compile-time q keeps r[] in registers
+    if (q == j) *zx = Vec16<kBf16>::at(r[q], e);
+}
+
+// --------------------------------------------------------------- row kernel
+// Grid: x = b (gamma + 1) + i (row pair), y = segment.
+template <bool kBf16>
+__global__ void __launch_bounds__(kRowThreads, 3) rows_kernel(const __grid_constant__ SingleParams f) {
   __shared__ RowAcc rows[kMaxRowsPerSeq];
-  __shared__ RowAcc scratch[2 * (kConsumers / 32)];
-  __shared__ float4 race_scratch[kConsumers / 32];
+  __shared__ RowAcc scratch[2 * (kRowThreads / 32)];
+  __shared__ float s_zx[2];
+  __shared__ float s_zsel[2 * SV_MAX_GAMMA];
   __shared__ int s_last;
-  __shared__ float s_zx[2];                   // the draft token's logits in the current row item
-  __shared__ float s_zsel[2 * SV_MAX_GAMMA];  // per position, for the decision
-  __shared__ volatile int s_abort;
-  // Wait for the previous grid in the stream (programmatic dependent launch),
-  // then let the next one start launching its CTAs.
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  asm volatile("griddepcontrol.launch_dependents;");
-  const long long total = f.n1 + f.n2;
+  pdl_wait_and_release();
+  const Pass1Params& p = f.p1;
   const int tid = threadIdx.x;
-  constexpr int kN = Vec16<kBf16>::kN;
-  constexpr size_t kStride = 2 * kStageVec;  // vectors per stage
+  const int pair = blockIdx.x;
+  const int b = pair / (p.gamma + 1);
+  const int i = pair - b * (p.gamma + 1);
+  const int seg = blockIdx.y;
+  const float T = __ldg(p.temps + b);
+  const int modeA = row_mode(T, true);
+  const bool argmaxA = modeA == kRowArgmax;
+  const bool loadA = modeA != kRowSkip;
+  const bool loadB = i < p.gamma && row_mode(T, false) == kRowLse;
+  const float c = modeA == kRowLse ? __fdiv_rn(kLog2e, T) : 0.0f;
+  int xg = -1;
+  if (modeA == kRowLse && i < p.gamma) {
+    const int xt = __ldg(p.tokens + static_cast<size_t>(b) * p.gamma + i);
+    if (xt >= 0 && xt < p.V) xg = xt;
+  }
+  if (tid == 0) s_zx[0] = s_zx[1] = __int_as_float(0x7fc00000);  // NaN: "not in this segment"
+  block_sync<kRowThreads>();
+
+  RunAcc accA, accB;
+  accA.reset();
+  accB.reset();
+  const char* rpA = target_row<kBf16>(p, b, i);
+  const char* rpB = loadB ? draft_row<kBf16>(p, b, i) : rpA;
+  const RowGeom<kBf16> gA(rpA, p.V), gB(rpB, p.V);
+  const int k0 = seg * f.segvec;
+  const int a1 = min(gA.nvec, k0 + f.segvec), b1 = min(gB.nvec, k0 + f.segvec);
+  const uint4* vA = gA.body(rpA);
+  const uint4* vB = gB.body(rpB);
+  const int ownA = owned_vector<kBf16>(gA, xg, k0, a1);
+  const int ownB = owned_vector<kBf16>(gB, xg, k0, b1);
+  const int kend = max(loadA ? a1 : k0, loadB ? b1 : k0);
+  for (int kb = k0; kb < kend; kb += kTileVec) {
+    uint4 ra[kTileRegs], rb[kTileRegs];
+    if (loadA) load_tile<kBf16>(vA, kb, a1, ra);
+    if (loadB) load_tile<kBf16>(vB, kb, b1, rb);
+    if (loadA) {
+      pick_logit<kBf16>(ra, ownA, kb, xg, gA, &s_zx[0]);
+      if (argmaxA)
+        argmax_tile<kBf16>(accA, ra, gA.head + (kb + tid) * Vec16<kBf16>::kN);
+      else
+        lse_tile<kBf16>(accA, ra, c);
+    }
+    if (loadB) {
+      pick_logit<kBf16>(rb, ownB, kb, xg, gB, &s_zx[1]);
+      lse_tile<kBf16>(accB, rb, c);
+    }
+  }
+  const bool first = seg == 0, last = seg == f.nseg - 1;
+  if (loadA && (first || last))
+    row_edges<kBf16>(rpA, p.V, gA, argmaxA, c, first, last, xg, &s_zx[0], accA);
+  if (loadB && (first || last))
+    row_edges<kBf16>(rpB, p.V, gB, false, c, first, last, xg, &s_zx[1], accB);
+
+  RowAcc A = accA.row(), B = accB.row();
+  reduce_pair(A, B, argmaxA, c, scratch);
   if (tid == 0) {
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], kConsumers / 32);  // one arrival per consumer warp
+    float4* pp = f.pairpart + ((static_cast<size_t>(b) * (p.gamma + 1) + i) * f.nseg + seg) * 2;
+    pp[0] = make_float4(A.m, A.s, __int_as_float(A.arg), __int_as_float(A.bad));
+    pp[1] = make_float4(B.m, B.s, __int_as_float(B.arg), __int_as_float(B.bad));
+    if (i < p.gamma) {
+      float* z = f.zx + ((static_cast<size_t>(b) * p.gamma + i) * f.nseg + seg) * 2;
+      z[0] = s_zx[0];
+      z[1] = s_zx[1];
     }
-    mbar_fence_init();
-    s_abort = 0;
-    s_zx[0] = s_zx[1] = __int_as_float(0x7fc00000);
+    const unsigned tk = ticket_release(p.ticket + b);
+    const unsigned arrivals = static_cast<unsigned>((p.gamma + 1) * f.nseg);
+    s_last = (tk == arrivals - 1);
+    if (s_last) p.ticket[b] = 0;  // leave the counter at zero for the next call
   }
-  __syncthreads();
+  block_sync<kRowThreads>();
+  if (!s_last) return;
+  fence_acquire();
+  combine_pairs(f, b, rows, s_zsel);
+  if (tid < 32) decide_single<kBf16>(p, b, rows, s_zsel);
+}
 
-  if (tid >= kConsumers) {
-    // ---------------- producer warp (one lane) ----------------
-    if (tid != kConsumers) return;
-    uint32_t emask = (1u << kStages) - 1;  // a fresh barrier's "previous" phase is complete
-    int s = 0;
-    long long q = static_cast<long long>(atomicAdd(f.head, 1ull));
-    for (;;) {
-      // take the next position now; its latency overlaps this item's staging
-      const long long qn = q < total ? static_cast<long long>(atomicAdd(f.head, 1ull)) : total;
-      StageDesc d{};
-      const char *rpA = nullptr, *rpB = nullptr;
-      int a0 = 0, a1 = 0, b0 = 0, b1 = 0, headA = 0, headB = 0, kA = 0, kB = 0;
-      d.nst = 1;
-      if (q < total) {
-        int kind, b, x;
-        map_item(f, q, kind, b, x);
-        d.kind = kind;
-        d.b = b;
-        d.x = x;
-        if (kind == 1) {
-          const float T = __ldg(f.p1.temps + b);
-          const int i = x / f.nseg;
-          d.x = i;
-          d.seg = x - i * f.nseg;
-          d.modeA = row_mode(T, true);
-          d.loadB = i < f.p1.gamma && row_mode(T, false) == kRowLse;
-          d.c = d.modeA == kRowLse ? __fdiv_rn(kLog2e, T) : 0.0f;
-          d.xg = -1;
-          if (d.modeA == kRowLse && i < f.p1.gamma) {
-            const int xt = __ldg(f.p1.tokens + static_cast<size_t>(b) * f.p1.gamma + i);
-            if (xt >= 0 && xt < f.p1.V) d.xg = xt;
-          }
-          int n = 0;
-          if (d.modeA != kRowSkip) {
-            rpA = target_row<kBf16>(f, b, i);
-            const RowGeom<kBf16> g(rpA, f.p1.V);
-            g.segment(d.seg, f.nseg, a0, a1);
-            headA = g.head;
-            n = (a1 - a0 + kStageVec - 1) / kStageVec;
-          }
-          if (d.loadB) {
-            rpB = draft_row<kBf16>(f, b, i);
-            const RowGeom<kBf16> g(rpB, f.p1.V);
-            g.segment(d.seg, f.nseg, b0, b1);
-            headB = g.head;
-            n = max(n, (b1 - b0 + kStageVec - 1) / kStageVec);
-          }
-          d.nst = n < 1 ? 1 : n;
-        } else {
-          describe_draw<kBf16>(f, b, x, d, rpA, rpB, kA, kB);
-        }
-      }
-      for (int t = 0; t < d.nst; ++t) {
-        if (s_abort || !mbar_wait(&empty[s], (emask >> s) & 1u, f.error)) {
-          s_abort = 1;  // the consumers stop at their next stage
-          return;
-        }
-        emask ^= 1u << s;
-        StageDesc e = d;
-        e.t = t;
-        uint4* st = stage + s * kStride;
-        uint32_t bytesA = 0, bytesB = 0;
-        const void *srcA = nullptr, *srcB = nullptr;
-        if (d.kind == 1) {
-          const int ka = min(a1, a0 + t * kStageVec), kb = min(b1, b0 + t * kStageVec);
-          e.nA = rpA ? min(a1, ka + kStageVec) - ka : 0;
-          e.nB = rpB ? min(b1, kb + kStageVec) - kb : 0;
-          const int baseA = headA + ka * kN, baseB = headB + kb * kN;
-          e.vA = baseA;
-          e.gA = (d.xg >= baseA && d.xg < baseA + e.nA * kN) ? d.xg - baseA : -1;
-          e.gB = (d.xg >= baseB && d.xg < baseB + e.nB * kN) ? d.xg - baseB : -1;
-          const bool first = d.seg == 0 && t == 0, last = d.seg == f.nseg - 1 && t == d.nst - 1;
-          e.edges = (rpA && first ? 1 : 0) | (rpA && last ? 2 : 0) | (rpB && first ? 4 : 0) |
-                    (rpB && last ? 8 : 0);
-          bytesA = static_cast<uint32_t>(e.nA) * 16u;
-          bytesB = static_cast<uint32_t>(e.nB) * 16u;
-          if (bytesA) srcA = rpA + static_cast<size_t>(headA) * (kBf16 ? 2 : 4) + static_cast<size_t>(ka) * 16;
-          if (bytesB) srcB = rpB + static_cast<size_t>(headB) * (kBf16 ? 2 : 4) + static_cast<size_t>(kb) * 16;
-        } else if (d.kind == 2 && d.draw) {
-          bytesA = static_cast<uint32_t>(d.nvA) * 16u;
-          bytesB = static_cast<uint32_t>(d.nvB) * 16u;
-          if (bytesA) srcA = rpA + static_cast<size_t>(d.sbA) * (kBf16 ? 2 : 4);
-          if (bytesB) srcB = rpB + static_cast<size_t>(d.sbB) * (kBf16 ? 2 : 4);
-        }
-        desc[s] = e;
-        if (bytesA + bytesB) {
-          fence_proxy_async_smem();  // the stage was last read through the generic proxy
-          mbar_expect_tx(&full[s], bytesA + bytesB);
-          if (bytesA) bulk_load(st, srcA, bytesA, &full[s]);
-          if (bytesB) bulk_load(st + kStageVec, srcB, bytesB, &full[s]);
-        } else {
-          mbar_arrive(&full[s]);
-        }
-        s = (s + 1) % kStages;
-      }
-      if (q >= total) return;  // the end-of-work stage has been published
-      q = qn;
-    }
-  }
+// -------------------------------------------------------------- draw kernel
+// The 4 logits of Philox block g of a row, kept packed until used; entries
+// at or beyond V read as -inf.
+template <bool kBf16>
+struct Block4;
 
-  // ---------------- consumer warps ----------------
-  uint32_t fmask = 0u;
-  int s = 0;
-  // Thread 0 waits (bounded); the barrier makes the abort decision uniform;
-  // then every consumer acquires the stage.
-  auto wait_stage = [&]() -> bool {
-    if (tid == 0 && !mbar_wait(&full[s], (fmask >> s) & 1u, f.error)) s_abort = 1;
-    block_sync<kConsumers>();
-    if (s_abort) return false;
-    mbar_try_wait(&full[s], (fmask >> s) & 1u);
-    fmask ^= 1u << s;
-    return true;
-  };
-  auto release_stage = [&]() {
-    __syncwarp();
-    if ((tid & 31) == 0) mbar_arrive(&empty[s]);
-    s = (s + 1) % kStages;
-  };
-  for (;;) {
-    if (!wait_stage()) break;
-    const int kind = desc[s].kind;
-    if (kind == 0) break;
-    const int b = desc[s].b, x = desc[s].x;
-    if (kind == 1) {
-      // ---- row item: target row x and draft row x over one segment ----
-      const int seg = desc[s].seg, nst = desc[s].nst, modeA = desc[s].modeA;
-      const float c = desc[s].c;
-      RunAcc accA, accB;
-      accA.reset();
-      accB.reset();
-      for (int t = 0;;) {
-        const StageDesc& d = desc[s];
-        const uint4* sm = stage + s * kStride;
-        constexpr int kR = kStageVec / kConsumers;  // vectors per thread per row piece
-        {
-          uint4 ra[kR];
-          const int na = d.nA > tid ? (d.nA - tid + kConsumers - 1) / kConsumers : 0;
-#pragma unroll
-          for (int j = 0; j < kR; ++j)
-            if (j < na) ra[j] = sm[tid + j * kConsumers];
-#pragma unroll
-          for (int j = 0; j < kR; ++j)  // compile-time j keeps ra[] in registers
-            if (d.gA >= 0 && d.gA / kN == tid + j * kConsumers) s_zx[0] = Vec16<kBf16>::at(ra[j], d.gA % kN);
-          if (modeA == kRowLse) {
-            lse_block<kBf16, kR>(accA, ra, na, c);
-          } else if (modeA == kRowArgmax) {
-            int v0[kR];
-#pragma unroll
-            for (int j = 0; j < kR; ++j) v0[j] = d.vA + (tid + j * kConsumers) * kN;
-            argmax_block<kBf16, kR>(accA, ra, na, v0);
-          }
-        }
-        {
-          uint4 rb[kR];
-          const int nb = d.nB > tid ? (d.nB - tid + kConsumers - 1) / kConsumers : 0;
-#pragma unroll
-          for (int j = 0; j < kR; ++j)
-            if (j < nb) rb[j] = sm[kStageVec + tid + j * kConsumers];
-#pragma unroll
-          for (int j = 0; j < kR; ++j)
-            if (d.gB >= 0 && d.gB / kN == tid + j * kConsumers) s_zx[1] = Vec16<kBf16>::at(rb[j], d.gB % kN);
-          lse_block<kBf16, kR>(accB, rb, nb, c);
-        }
-        const int edges = d.edges, xg = d.xg;
-        release_stage();  // desc[] of this stage is not read past this point
-        if (edges & 3)
-          row_edges<kBf16>(f, target_row<kBf16>(f, b, x), modeA, c, edges & 1, edges & 2, xg, &s_zx[0], accA);
-        if (edges & 12)
-          row_edges<kBf16>(f, draft_row<kBf16>(f, b, x), kRowLse, c, edges & 4, edges & 8, xg, &s_zx[1], accB);
-        if (++t == nst) break;
-        if (!wait_stage()) break;
-      }
-      if (s_abort) break;
-      // ---- finalize: reduce, publish, take the sequence's ticket ----
-      RowAcc A = accA.row(), B = accB.row();
-      reduce_pair(A, B, modeA, c, scratch);
-      if (tid == 0) {
-        float4* pp = f.pairpart + ((static_cast<size_t>(b) * (f.p1.gamma + 1) + x) * f.nseg + seg) * 2;
-        pp[0] = make_float4(A.m, A.s, __int_as_float(A.arg), __int_as_float(A.bad));
-        pp[1] = make_float4(B.m, B.s, __int_as_float(B.arg), __int_as_float(B.bad));
-        if (x < f.p1.gamma) {
-          float* z = f.zx + ((static_cast<size_t>(b) * f.p1.gamma + x) * f.nseg + seg) * 2;
-          z[0] = s_zx[0];
-          z[1] = s_zx[1];
-        }
-        s_zx[0] = s_zx[1] = __int_as_float(0x7fc00000);  // NaN: "not in this segment"
-        const unsigned tk = ticket_release(f.p1.ticket + b);
-        s_last = (tk == static_cast<unsigned>(f.a - 1));
-        if (s_last) f.p1.ticket[b] = 0;  // leave the counter at zero for the next call
-      }
-      block_sync<kConsumers>();
-      if (s_last) {
-        fence_acquire();
-        combine_pairs(f, b, rows, s_zsel);
-        if (tid < 32) decide_single<kBf16>(f.p1, b, rows, s_zsel);
-        block_sync<kConsumers>();  // rows[] / s_last are reused by the next item
-      }
+template <>
+struct Block4<true> {
+  uint2 r;
+  __device__ __forceinline__ void load(const char* row, bool vec_ok, int V, int g) {
+    const int v0 = 4 * g;
+    if (vec_ok && v0 + 3 < V) {
+      r = __ldg(reinterpret_cast<const uint2*>(row) + g);
     } else {
-      // ---- draw item: race over the staged chunk ----
-      const StageDesc d = desc[s];  // copy: the stage is released before the combine
-      float bw = 0.0f, be = 1.0f;
-      int bi = INT_MAX;
-      if (d.draw) {
-        const uint4* sm = stage + s * kStride;
-        race_staged<kBf16>(f, d, b, sm, sm + kStageVec, d.e0 / 4, (d.e1 + 3) / 4, bw, be, bi);
-      }
-      release_stage();
-      race_reduce<kConsumers>(bw, be, bi, race_scratch);
-      if (tid == 0) {
-        RacePartial* pp = f.part2 + static_cast<size_t>(b) * f.nc2 + x;
-        *reinterpret_cast<float4*>(pp) = make_float4(bw, be, __int_as_float(bi), 0.0f);
-        const unsigned tk = ticket_release(f.ticket2 + b);
-        s_last = (tk == static_cast<unsigned>(f.nc2 - 1));
-        if (s_last) f.ticket2[b] = 0;
-      }
-      block_sync<kConsumers>();
-      if (s_last) {
-        fence_acquire();
-        if (d.draw) {
-          bw = 0.0f;
-          be = 1.0f;
-          bi = INT_MAX;
-          for (int q = tid; q < f.nc2; q += kConsumers) {
-            const float4 g = __ldcg(reinterpret_cast<const float4*>(f.part2 + static_cast<size_t>(b) * f.nc2 + q));
-            if (race_better(g.x, g.y, __float_as_int(g.z), bw, be, bi)) {
-              bw = g.x;
-              be = g.y;
-              bi = __float_as_int(g.z);
-            }
-          }
-          race_reduce<kConsumers>(bw, be, bi, race_scratch);
-          if (!(bw > 0.0f)) {  // uniform: race_reduce returns the winner to every thread
-            bw = 0.0f;
-            be = 1.0f;
-            bi = INT_MAX;
-            race_row_global<kBf16>(f, d, b, bw, be, bi);
-            race_reduce<kConsumers>(bw, be, bi, race_scratch);
-          }
-          if (tid == 0) f.p1.out_tokens[static_cast<size_t>(b) * (f.p1.gamma + 1) + d.j] = bi;
-        }
-        if (tid == 0) f.p1.flag[static_cast<size_t>(b) * kFlagStride] = 0u;  // all readers are done
-        block_sync<kConsumers>();  // s_last is reused by the next item
+      const uint16_t* q = reinterpret_cast<const uint16_t*>(row);
+      const uint32_t ninf = 0xFF80u;  // bf16 -inf
+      uint32_t h[4];
+#pragma unroll
+      for (int w = 0; w < 4; ++w) h[w] = v0 + w < V ? static_cast<uint32_t>(__ldg(q + v0 + w)) : ninf;
+      r = make_uint2(h[0] | (h[1] << 16), h[2] | (h[3] << 16));
+    }
+  }
+  __device__ __forceinline__ float at(int w) const {
+    const uint32_t x = w < 2 ? r.x : r.y;
+    return (w & 1) ? bf16_hi(x) : bf16_lo(x);
+  }
+};
+
+template <>
+struct Block4<false> {
+  float4 r;
+  __device__ __forceinline__ void load(const char* row, bool vec_ok, int V, int g) {
+    const int v0 = 4 * g;
+    if (vec_ok && v0 + 3 < V) {
+      r = __ldg(reinterpret_cast<const float4*>(row) + g);
+    } else {
+      const float* q = reinterpret_cast<const float*>(row);
+      r.x = v0 + 0 < V ? __ldg(q + v0 + 0) : -INFINITY;
+      r.y = v0 + 1 < V ? __ldg(q + v0 + 1) : -INFINITY;
+      r.z = v0 + 2 < V ? __ldg(q + v0 + 2) : -INFINITY;
+      r.w = v0 + 3 < V ? __ldg(q + v0 + 3) : -INFINITY;
+    }
+  }
+  __device__ __forceinline__ float at(int w) const {
+    return w == 0 ? r.x : (w == 1 ? r.y : (w == 2 ? r.z : r.w));
+  }
+};
+
+// Exponential race over Philox blocks [g0, g1) of the draw row(s): the winner
+// of w_v / E_v (E_v = -ln U_v) with w = max(p - q, 0) (residual) or
+// w = 2^{(z - max) c} (bonus).  Each thread loads all of its blocks before
+// using any of them.  A candidate is skipped without its logarithm when even
+// the bound E_v >= 1 - U_v cannot beat the current best.
+template <bool kBf16>
+__device__ __forceinline__ void race_chunk(const SingleParams& f, const SeqInfo& si, int b, int g0,
+                                           int g1, float& bw, float& be, int& bi) {
+  constexpr uintptr_t kVecAlign = kBf16 ? 8 : 16;
+  const Pass1Params& p = f.p1;
+  const char* trow = target_row<kBf16>(p, b, si.j);
+  const bool resid = si.mode == kModeResidual;
+  const char* drow = resid ? draft_row<kBf16>(p, b, si.j) : trow;
+  const bool tvec = (reinterpret_cast<uintptr_t>(trow) % kVecAlign) == 0;
+  const bool dvec = (reinterpret_cast<uintptr_t>(drow) % kVecAlign) == 0;
+  Block4<kBf16> zt[kDrawMaxBlocks], zd[kDrawMaxBlocks];
+  const int gb = g0 + static_cast<int>(threadIdx.x);
+#pragma unroll
+  for (int u = 0; u < kDrawMaxBlocks; ++u) {
+    const int g = gb + u * kDrawThreads;
+    if (g < g1) {
+      zt[u].load(trow, tvec, p.V, g);
+      if (resid) zd[u].load(drow, dvec, p.V, g);
+    }
+  }
+#pragma unroll
+  for (int u = 0; u < kDrawMaxBlocks; ++u) {
+    const int g = gb + u * kDrawThreads;
+    if (g >= g1) break;
+    const uint4 rnd = keyed_block(p.seed, p.step, kTagGumbel, b, 0, si.j, g);
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      float wt = ex2_approx((zt[u].at(w) - si.zmp) * si.c);
+      if (resid) wt = wt * si.isp - ex2_approx((zd[u].at(w) - si.zmq) * si.c) * si.isq;
+      if (!(wt > 0.0f)) continue;
+      const uint32_t x = word_of(rnd, w);
+      if (bw > 0.0f && wt * be <= bw * gumbel_one_minus_u(x)) continue;
+      const float e = exponential_from_bits(x);
+      const int v = 4 * g + w;
+      if (race_better(wt, e, v, bw, be, bi)) {
+        bw = wt;
+        be = e;
+        bi = v;
       }
     }
   }
-  block_sync<kConsumers>();
-  if (tid == 0) {
-    const unsigned n = atomicAdd(f.exited, 1u);
-    if (n == gridDim.x - 1) {  // last CTA out leaves the queue reset
-      *f.head = 0ull;
-      *f.exited = 0u;
+}
+
+// Fallback draw over a whole target row (the residual vanished: p_j == q_j
+// to rounding): bonus-style race over p_j, by one CTA.
+template <bool kBf16>
+__device__ void race_row(const SingleParams& f, SeqInfo si, int b, float& bw, float& be, int& bi) {
+  si.mode = kModeBonus;
+  const int nblocks = (f.p1.V + 3) / 4;
+  for (int g0 = 0; g0 < nblocks; g0 += kDrawMaxBlocks * kDrawThreads)
+    race_chunk<kBf16>(f, si, b, g0, min(nblocks, g0 + kDrawMaxBlocks * kDrawThreads), bw, be, bi);
+}
+
+template <bool kBf16>
+__global__ void __launch_bounds__(kDrawThreads) draw_kernel(const __grid_constant__ SingleParams f) {
+  __shared__ float4 scratch[kDrawThreads / 32];
+  __shared__ int s_last;
+  pdl_wait_and_release();  // the row kernel has completed: every decision is visible
+  const int b = blockIdx.x / f.nc2;
+  const int chunk = blockIdx.x - b * f.nc2;
+  const Pass1Params& p = f.p1;
+  const float4* ip = reinterpret_cast<const float4*>(p.info + b);
+  const float4 w0 = __ldcg(ip), w1 = __ldcg(ip + 1);
+  SeqInfo si{};
+  si.mode = __float_as_int(w0.x);
+  si.j = __float_as_int(w0.y);
+  si.zmp = w0.z;
+  si.zmq = w0.w;
+  si.c = w1.x;
+  si.isp = w1.y;
+  si.isq = w1.z;
+  const bool draw = (si.mode == kModeResidual && si.j >= 0 && si.j < p.gamma) ||
+                    (si.mode == kModeBonus && si.j == p.gamma);
+  if (!draw) return;  // uniform: greedy or invalid sequence
+  const int nblocks = (p.V + 3) / 4;
+  const int g0 = chunk * (f.chunk2 / 4);
+  const int g1 = min(nblocks, g0 + f.chunk2 / 4);
+  float bw = 0.0f, be = 1.0f;
+  int bi = INT_MAX;
+  race_chunk<kBf16>(f, si, b, g0, g1, bw, be, bi);
+  race_reduce<kDrawThreads>(bw, be, bi, scratch);
+  if (threadIdx.x == 0) {
+    RacePartial* pp = f.part2 + static_cast<size_t>(b) * f.nc2 + chunk;
+    *reinterpret_cast<float4*>(pp) = make_float4(bw, be, __int_as_float(bi), 0.0f);
+    const unsigned t = ticket_release(f.ticket2 + b);
+    s_last = (t == static_cast<unsigned>(f.nc2 - 1));
+    if (s_last) f.ticket2[b] = 0;
+  }
+  block_sync<kDrawThreads>();
+  if (!s_last) return;
+  fence_acquire();
+  bw = 0.0f;
+  be = 1.0f;
+  bi = INT_MAX;
+  for (int q = threadIdx.x; q < f.nc2; q += kDrawThreads) {
+    const float4 g = __ldcg(reinterpret_cast<const float4*>(f.part2 + static_cast<size_t>(b) * f.nc2 + q));
+    if (race_better(g.x, g.y, __float_as_int(g.z), bw, be, bi)) {
+      bw = g.x;
+      be = g.y;
+      bi = __float_as_int(g.z);
     }
   }
+  race_reduce<kDrawThreads>(bw, be, bi, scratch);
+  if (!(bw > 0.0f)) {  // uniform: race_reduce returns the winner to every thread
+    bw = 0.0f;
+    be = 1.0f;
+    bi = INT_MAX;
+    race_row<kBf16>(f, si, b, bw, be, bi);
+    race_reduce<kDrawThreads>(bw, be, bi, scratch);
+  }
+  if (threadIdx.x == 0) p.out_tokens[static_cast<size_t>(b) * (p.gamma + 1) + si.j] = bi;
 }
 
 // ------------------------------------------------------------------ launch
 namespace {
-struct Occupancy {
-  int sms = 0, per_sm[2] = {0, 0};
-};
-Occupancy g_occ[64];
-std::mutex g_occ_mu;
-
-int resident_ctas(bool bf16) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-  std::lock_guard<std::mutex> lk(g_occ_mu);
-  Occupancy& o = g_occ[dev];
-  if (o.sms == 0) cudaDeviceGetAttribute(&o.sms, cudaDevAttrMultiProcessorCount, dev);
-  int& n = o.per_sm[bf16 ? 1 : 0];
-  if (n == 0) {
-    const int dyn = kStages * static_cast<int>(kStageBytes);
-    if (bf16) {
-      cudaFuncSetAttribute(fused_single_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn);
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fused_single_kernel<true>, kFusedThreads, dyn);
-    } else {
-      cudaFuncSetAttribute(fused_single_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn);
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fused_single_kernel<false>, kFusedThreads, dyn);
-    }
-    if (n < 1) n = 1;
-  }
-  return o.sms * n;
+int body_tiles(int V, int dtype) {  // tiles of kTileVec vectors covering a row's body
+  const long long vecs = static_cast<long long>(V) * (dtype == SV_BF16 ? 2 : 4) / 16;
+  const long long t = (vecs + kTileVec - 1) / kTileVec;
+  return t < 1 ? 1 : static_cast<int>(t);
 }
 }  // namespace
 
-int draw_chunks(int V, int dtype) {
-  const int per = draw_chunk(dtype == SV_BF16);
-  return (V + per - 1) / per;
+int row_segments(int V, int dtype) { return body_tiles(V, dtype); }  // bound on segments per row
+
+int draw_chunks(int V, int dtype) {  // upper bound on draw CTAs per sequence
+  (void)dtype;
+  return (V + 4 * kDrawThreads - 1) / (4 * kDrawThreads);
 }
+
+namespace {
+int sm_count() {
+  static int cached[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (cached[dev] == 0) {
+    int n = 0;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    cached[dev] = n > 0 ? n : 148;
+  }
+  return cached[dev];
+}
+
+// Resident row-kernel CTAs per SM (occupancy query, cached per device).
+int row_ctas_per_sm(bool bf16) {
+  static int cached[64][2];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 3;
+  int& slot = cached[dev][bf16 ? 1 : 0];
+  if (slot == 0) {
+    int n = 0;
+    const cudaError_t e =
+        bf16 ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, rows_kernel<true>, kRowThreads, 0)
+             : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, rows_kernel<false>, kRowThreads, 0);
+    if (e != cudaSuccess) (void)cudaGetLastError();
+    slot = (e == cudaSuccess && n > 0) ? n : 3;
+  }
+  return slot;
+}
+
+template <typename K>
+cudaError_t launch_pdl(K kernel, dim3 grid, unsigned block, cudaStream_t stream,
+                       const SingleParams& f) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(block);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, f);
+  if (e != cudaSuccess) {
+    (void)cudaGetLastError();
+    cfg.numAttrs = 0;  // retry as an ordinary stream-ordered launch
+    e = cudaLaunchKernelEx(&cfg, kernel, f);
+  }
+  return e;
+}
+}  // namespace
 
 int launch_single(const void* target, const void* draft, const int32_t* tokens,
                   const float* temps, int B, int gamma, int V, int dtype, uint64_t seed,
                   uint64_t step, int32_t* out_accept_len, int32_t* out_tokens, float* out_lp,
                   float* out_lq, void* workspace, const Layout& lay, cudaStream_t stream) {
   char* ws = static_cast<char*>(workspace);
-  FusedParams f{};
+  SingleParams f{};
   Pass1Params& p1 = f.p1;
   p1.target = target;
   p1.draft = draft;
@@ -892,60 +656,55 @@ int launch_single(const void* target, const void* draft, const int32_t* tokens,
   p1.step = static_cast<uint32_t>(step);
   p1.ticket = reinterpret_cast<unsigned*>(ws + lay.ticket1);
   p1.info = reinterpret_cast<SeqInfo*>(ws + lay.info);
-  p1.flag = reinterpret_cast<unsigned*>(ws + lay.flag);
   p1.accept_len = out_accept_len;
   p1.out_tokens = out_tokens;
   p1.out_lp = out_lp;
   p1.out_lq = out_lq;
-  f.part2 = reinterpret_cast<RacePartial*>(ws + lay.part2);
-  f.ticket2 = reinterpret_cast<unsigned*>(ws + lay.ticket2);
-  f.nc2 = lay.nc2;
-  f.head = reinterpret_cast<unsigned long long*>(ws + lay.ctl);
-  f.exited = reinterpret_cast<unsigned*>(ws + lay.ctl + 8);
-  f.error = reinterpret_cast<unsigned*>(ws + lay.ctl + 12);
+  // Row segments: whole tiles, about kRowWaves waves of CTAs over the GPU but
+  // at most kMaxSegTiles tiles per CTA; balanced so segments differ by at
+  // most one tile.
   const bool bf16 = dtype == SV_BF16;
-  const int S = resident_ctas(bf16);
-  // Segments per row pair: about 8 row items per resident CTA (load
-  // balance), bounded by the workspace's segment capacity.
-  const long long pairs = static_cast<long long>(B) * (gamma + 1);
-  long long nseg = (8LL * S + pairs - 1) / pairs;
-  if (nseg > lay.nc) nseg = lay.nc;
-  if (nseg < 1) nseg = 1;
-  f.nseg = static_cast<int>(nseg);
+  {
+    constexpr int kRowWaves = 4, kMaxSegTiles = 8;
+    const int tiles = body_tiles(V, dtype);
+    const long long pairs = static_cast<long long>(B) * (gamma + 1);
+    const long long slots = static_cast<long long>(sm_count()) * row_ctas_per_sm(bf16);
+    long long st = pairs * tiles / (kRowWaves * slots);
+    st = st < 1 ? 1 : (st > kMaxSegTiles ? kMaxSegTiles : st);
+    int nseg = static_cast<int>((tiles + st - 1) / st);
+    if (nseg > lay.nc) nseg = lay.nc;
+    if (nseg > 65535) nseg = 65535;  // gridDim.y
+    st = (tiles + nseg - 1) / nseg;
+    f.nseg = nseg;
+    f.segvec = static_cast<int>(st) * kTileVec;
+  }
   f.pairpart = reinterpret_cast<float4*>(ws + lay.part1);
   f.zx = reinterpret_cast<float*>(ws + lay.resid);
-  f.a = (gamma + 1) * f.nseg;
-  f.n1 = static_cast<long long>(B) * f.a;
-  f.n2 = static_cast<long long>(B) * f.nc2;
-  const long long items = f.n1 + f.n2;
-  const unsigned grid = static_cast<unsigned>(items < S ? items : S);
-  // A sequence's draw items are queued about one resident wave of items
-  // after its row items: late enough that its decision is usually made, early
-  // enough that its rows are usually still in L2.
-  const long long lag = static_cast<long long>(grid) / f.a + 1;
-  f.lag = static_cast<int>(lag < B ? lag : B);
+  f.part2 = reinterpret_cast<RacePartial*>(ws + lay.part2);
+  f.ticket2 = reinterpret_cast<unsigned*>(ws + lay.ticket2);
+  // Draw chunks: enough CTAs to cover the GPU about twice when the batch is
+  // small, at most kDrawMaxBlocks Philox blocks per thread.
+  const long long want = (2LL * sm_count() + B - 1) / B;
+  const int unit = 4 * kDrawThreads;  // entries per Philox block per thread
+  const int min_chunks = (V + unit * kDrawMaxBlocks - 1) / (unit * kDrawMaxBlocks);
+  long long nc2 = want > min_chunks ? want : min_chunks;
+  if (nc2 > lay.nc2) nc2 = lay.nc2;
+  int chunk = static_cast<int>((V + nc2 - 1) / nc2);
+  chunk = (chunk + unit - 1) / unit * unit;
+  f.chunk2 = chunk;
+  f.nc2 = (V + chunk - 1) / chunk;
 
-  cudaLaunchConfig_t cfg{};
-  cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(kFusedThreads);
-  cfg.dynamicSmemBytes = kStages * kStageBytes;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  cudaError_t e = bf16 ? cudaLaunchKernelEx(&cfg, fused_single_kernel<true>, f)
-                       : cudaLaunchKernelEx(&cfg, fused_single_kernel<false>, f);
-  if (e != cudaSuccess) {
-    (void)cudaGetLastError();
-    cfg.numAttrs = 0;  // retry as an ordinary stream-ordered launch
-    e = bf16 ? cudaLaunchKernelEx(&cfg, fused_single_kernel<true>, f)
-             : cudaLaunchKernelEx(&cfg, fused_single_kernel<false>, f);
-  }
+  const dim3 grid1(static_cast<unsigned>(B * (gamma + 1)), static_cast<unsigned>(f.nseg));
+  cudaError_t e = bf16 ? launch_pdl(rows_kernel<true>, grid1, kRowThreads, stream, f)
+                       : launch_pdl(rows_kernel<false>, grid1, kRowThreads, stream, f);
   if (e != cudaSuccess)
-    return set_error(SV_ERR_CUDA, "fused verify launch failed: %s", cudaGetErrorString(e));
-  return check_launch("fused verify");
+    return set_error(SV_ERR_CUDA, "row kernel launch failed: %s", cudaGetErrorString(e));
+  const dim3 grid2(static_cast<unsigned>(static_cast<long long>(B) * f.nc2));
+  e = bf16 ? launch_pdl(draw_kernel<true>, grid2, kDrawThreads, stream, f)
+           : launch_pdl(draw_kernel<false>, grid2, kDrawThreads, stream, f);
+  if (e != cudaSuccess)
+    return set_error(SV_ERR_CUDA, "draw kernel launch failed: %s", cudaGetErrorString(e));
+  return check_launch("verify");
 }
 
 }  // namespace sv

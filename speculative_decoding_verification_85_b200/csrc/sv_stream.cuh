@@ -1,15 +1,23 @@
-// sv_stream.cuh -- row-pair streaming reduction for the fused single-draft
-// kernel.
+// sv_stream.cuh -- per-thread row reductions of the single-draft row kernel.
 //
-// A pass-1 work item is (sequence b, position i, vocabulary segment): target
+// A row-kernel CTA covers (sequence b, position i, vocabulary segment): target
 // row i and draft row i over the same segment (position gamma: the target row
-// alone).  The producer warp stages the item in pieces of up to kStageVec
-// 16-byte vectors per row; the consumer threads keep running per-row
-// accumulators in registers across the pieces and publish one partial per item.
+// alone).  The segment is walked in tiles of kTileVec 16-byte vectors; each
+// thread loads its kTileRegs vectors of a tile into registers, then folds
+// them into a running accumulator.
 //
-// Arithmetic per bf16 element: exact widening, NaN-propagating max on packed
-// bf16x2, then (z - max) * log2(e)/T with packed fp32x2 add/mul, one MUFU
-// ex2, and a packed fp32x2 running sum.
+// Softmax sums use an integer reference exponent.  With c = log2(e) / T and
+// R(m) = ceil(fl(m c)) for the running maximum m, a thread accumulates
+//     S = sum_v 2^{z_v c - R(m)}
+// where each exponent z_v c - R is one fused multiply-add (a single rounding;
+// the largest term is at most 2^1).  Two partial sums with references R1 >= R2
+// merge as S1 + S2 2^{R2 - R1}, a multiplication by an exact power of two.
+// The row's sum relative to its maximum, s = sum_v 2^{(z_v - m) c}, is
+// recovered once per row as S 2^{R(m) - m c} (in fp64).
+//
+// Per bf16 element: one bit operation to widen, half of a packed fp32x2 FMA,
+// one MUFU ex2, half of a packed fp32x2 add; the tile maximum costs one
+// packed bf16x2 max per two elements.
 #pragma once
 
 #include "sv_device.cuh"
@@ -18,7 +26,9 @@
 
 namespace sv {
 
-constexpr int kStageVec = 1024;  // 16-byte vectors per row per stage (16 KB)
+constexpr int kTileThreads = 256;                   // threads of a row-kernel CTA
+constexpr int kTileRegs = 4;                        // vectors per thread per row per tile
+constexpr int kTileVec = kTileThreads * kTileRegs;  // 16-byte vectors per row per tile (16 KB)
 
 __device__ __forceinline__ uint32_t hmax2_nan(uint32_t a, uint32_t b) {
   uint32_t d;
@@ -26,14 +36,24 @@ __device__ __forceinline__ uint32_t hmax2_nan(uint32_t a, uint32_t b) {
   return d;
 }
 
-// Per-thread running reduction of one row.
+// Exact 2^d for an integral d <= 0 (0 below the normal range).
+__device__ __forceinline__ float exp2_int(float d) {
+  return d < -126.0f ? 0.0f : __int_as_float((static_cast<int>(d) + 127) << 23);
+}
+
+// Reference exponent R(m) = ceil(fl(m c)); the same operations everywhere.
+__device__ __forceinline__ float ref_exp(float m, float c) { return ceilf(__fmul_rn(m, c)); }
+
+// Running reduction of one row by one thread.
 struct RunAcc {
-  float m;    // running raw max
-  float2 s;   // packed sum of 2^{(z - m) c}
-  int arg;    // first index of the max (greedy rows)
-  int bad;    // saw NaN
+  float m;   // running raw maximum (-inf: nothing yet)
+  float R;   // R(m) (0 while m = -inf)
+  float2 s;  // packed sum of 2^{z c - R} (softmax rows)
+  int arg;   // first index of the maximum (greedy rows)
+  int bad;   // saw NaN
   __device__ __forceinline__ void reset() {
     m = -INFINITY;
+    R = 0.0f;
     s = make_float2(0.0f, 0.0f);
     arg = 0x7fffffff;
     bad = 0;
@@ -41,19 +61,15 @@ struct RunAcc {
   __device__ __forceinline__ RowAcc row() const { return RowAcc{m, s.x + s.y, arg, bad}; }
 };
 
-// Move the running max to vm (> m), rescaling the sum.
-__device__ __forceinline__ void lift_max(RunAcc& a, float vm, float c) {
+// Move the running maximum up to tm (> m): new reference, rescale the sum.
+__device__ __forceinline__ void lift_ref(RunAcc& a, float tm, float c) {
+  const float Rn = ref_exp(tm, c);
   if (a.m != -INFINITY) {
-    const float f = ex2_approx((a.m - vm) * c);
+    const float f = exp2_int(a.R - Rn);
     a.s = __fmul2_rn(a.s, make_float2(f, f));
   }
-  a.m = vm;
-}
-
-// 2^{(z - m) c} for a pair of logits.
-__device__ __forceinline__ float2 exp_pair(float2 z, float2 nm, float2 cc) {
-  const float2 d = __fmul2_rn(__fadd2_rn(z, nm), cc);
-  return make_float2(ex2_approx(d.x), ex2_approx(d.y));
+  a.m = tm;
+  a.R = Rn;
 }
 
 template <bool kBf16>
@@ -62,9 +78,9 @@ struct Vec16;
 template <>
 struct Vec16<true> {  // 8 bf16
   static constexpr int kN = 8;
-  __device__ __forceinline__ static float vmax(const uint4& r) {
-    const uint32_t mm = hmax2_nan(hmax2_nan(r.x, r.y), hmax2_nan(r.z, r.w));
-    return max_nan(bf16_lo(mm), bf16_hi(mm));
+  static constexpr uint32_t kNegInf = 0xFF80FF80u;
+  __device__ __forceinline__ static uint32_t pmax(const uint4& r) {
+    return hmax2_nan(hmax2_nan(r.x, r.y), hmax2_nan(r.z, r.w));
   }
   __device__ __forceinline__ static float2 pair(const uint4& r, int k) {
     const uint32_t w = k == 0 ? r.x : (k == 1 ? r.y : (k == 2 ? r.z : r.w));
@@ -79,10 +95,7 @@ struct Vec16<true> {  // 8 bf16
 template <>
 struct Vec16<false> {  // 4 fp32
   static constexpr int kN = 4;
-  __device__ __forceinline__ static float vmax(const uint4& r) {
-    return max_nan(max_nan(__uint_as_float(r.x), __uint_as_float(r.y)),
-                   max_nan(__uint_as_float(r.z), __uint_as_float(r.w)));
-  }
+  static constexpr uint32_t kNegInf = 0xFF800000u;
   __device__ __forceinline__ static float2 pair(const uint4& r, int k) {
     return k == 0 ? make_float2(__uint_as_float(r.x), __uint_as_float(r.y))
                   : make_float2(__uint_as_float(r.z), __uint_as_float(r.w));
@@ -93,99 +106,82 @@ struct Vec16<false> {  // 4 fp32
   }
 };
 
+// Maximum of the thread's tile vectors (NaN if any element is NaN).
 template <bool kBf16>
-__device__ __forceinline__ void lse_vec(RunAcc& a, const uint4& r, float c) {
-  using V = Vec16<kBf16>;
-  const float vm = V::vmax(r);
-  if (vm != vm) {
-    a.bad = 1;
-    return;
-  }
-  if (vm == -INFINITY) return;
-  if (vm > a.m) lift_max(a, vm, c);
-  const float2 nm = make_float2(-a.m, -a.m), cc = make_float2(c, c);
+__device__ __forceinline__ float tile_max(const uint4 (&r)[kTileRegs]) {
   if constexpr (kBf16) {
-    const float2 e0 = exp_pair(V::pair(r, 0), nm, cc);
-    const float2 e1 = exp_pair(V::pair(r, 1), nm, cc);
-    const float2 e2 = exp_pair(V::pair(r, 2), nm, cc);
-    const float2 e3 = exp_pair(V::pair(r, 3), nm, cc);
-    a.s = __fadd2_rn(a.s, __fadd2_rn(__fadd2_rn(e0, e1), __fadd2_rn(e2, e3)));
+    uint32_t m = Vec16<true>::pmax(r[0]);
+#pragma unroll
+    for (int j = 1; j < kTileRegs; ++j) m = hmax2_nan(m, Vec16<true>::pmax(r[j]));
+    return max_nan(bf16_lo(m), bf16_hi(m));
   } else {
-    const float2 e0 = exp_pair(V::pair(r, 0), nm, cc);
-    const float2 e1 = exp_pair(V::pair(r, 1), nm, cc);
-    a.s = __fadd2_rn(a.s, __fadd2_rn(e0, e1));
+    float m = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < kTileRegs; ++j)
+      m = max_nan(max_nan(m, max_nan(__uint_as_float(r[j].x), __uint_as_float(r[j].y))),
+                  max_nan(__uint_as_float(r[j].z), __uint_as_float(r[j].w)));
+    return m;
   }
 }
 
+// Load the thread's vectors of the tile starting at vector kb; vectors at or
+// beyond k1 read as -inf.
 template <bool kBf16>
-__device__ __forceinline__ void argmax_vec(RunAcc& a, const uint4& r, int v0) {
+__device__ __forceinline__ void load_tile(const uint4* vp, int kb, int k1, uint4 (&r)[kTileRegs]) {
+  constexpr uint32_t ninf = Vec16<kBf16>::kNegInf;
+#pragma unroll
+  for (int j = 0; j < kTileRegs; ++j) {
+    const int k = kb + static_cast<int>(threadIdx.x) + j * kTileThreads;
+    r[j] = k < k1 ? ld_stream(vp + k) : make_uint4(ninf, ninf, ninf, ninf);
+  }
+}
+
+__device__ __forceinline__ float2 ex2_pair(float2 d) {
+  return make_float2(ex2_approx(d.x), ex2_approx(d.y));
+}
+
+// Fold a tile into a softmax-sum accumulator.
+template <bool kBf16>
+__device__ __forceinline__ void lse_tile(RunAcc& a, const uint4 (&r)[kTileRegs], float c) {
   using V = Vec16<kBf16>;
-  const float vm = V::vmax(r);
-  if (vm != vm) {
+  const float tm = tile_max<kBf16>(r);
+  if (tm != tm) {
     a.bad = 1;
     return;
   }
-  if (vm > a.m) {
-    a.m = vm;
-#pragma unroll
-    for (int e = V::kN - 1; e >= 0; --e)
-      if (V::at(r, e) == vm) a.arg = v0 + e;
-  }
-}
-
-// Sum of 2^{(z - m) c} over the elements of one vector (m fixed, finite).
-template <bool kBf16>
-__device__ __forceinline__ float2 exp_vec(const uint4& r, float2 nm, float2 cc) {
-  using V = Vec16<kBf16>;
-  if constexpr (kBf16) {
-    const float2 e0 = exp_pair(V::pair(r, 0), nm, cc);
-    const float2 e1 = exp_pair(V::pair(r, 1), nm, cc);
-    const float2 e2 = exp_pair(V::pair(r, 2), nm, cc);
-    const float2 e3 = exp_pair(V::pair(r, 3), nm, cc);
-    return __fadd2_rn(__fadd2_rn(e0, e1), __fadd2_rn(e2, e3));
-  } else {
-    return __fadd2_rn(exp_pair(V::pair(r, 0), nm, cc), exp_pair(V::pair(r, 1), nm, cc));
-  }
-}
-
-// Fold kR vectors of one thread (r[j] valid for j < n) into the running
-// accumulator: one max over all of them first, at most one rescale, then
-// independent exponentials (instruction-level parallelism across vectors).
-template <bool kBf16, int kR>
-__device__ __forceinline__ void lse_block(RunAcc& a, const uint4 (&r)[kR], int n, float c) {
-  using V = Vec16<kBf16>;
-  float vm = -INFINITY, mj[kR];
-  bool nan = false;
-#pragma unroll
-  for (int j = 0; j < kR; ++j) {
-    mj[j] = -INFINITY;
-    if (j < n) {
-      mj[j] = V::vmax(r[j]);
-      nan |= (mj[j] != mj[j]);
-      vm = fmaxf(vm, mj[j]);
-    }
-  }
-  if (nan) {
-    a.bad = 1;
-    return;
-  }
-  if (vm == -INFINITY) return;
-  if (vm > a.m) lift_max(a, vm, c);
-  const float2 nm = make_float2(-a.m, -a.m), cc = make_float2(c, c);
+  if (tm > a.m) lift_ref(a, tm, c);
+  const float2 nr = make_float2(-a.R, -a.R), cc = make_float2(c, c);
   float2 acc = make_float2(0.0f, 0.0f);
 #pragma unroll
-  for (int j = 0; j < kR; ++j)
-    // a vector whose largest term is below 2^-126 contributes only flushed
-    // zeros: skip its exponentials (same result)
-    if (j < n && (mj[j] - a.m) * c >= -126.0f) acc = __fadd2_rn(acc, exp_vec<kBf16>(r[j], nm, cc));
+  for (int j = 0; j < kTileRegs; ++j) {
+#pragma unroll
+    for (int k = 0; k < V::kN / 2; ++k)
+      acc = __fadd2_rn(acc, ex2_pair(__ffma2_rn(V::pair(r[j], k), cc, nr)));
+  }
   a.s = __fadd2_rn(a.s, acc);
 }
 
-template <bool kBf16, int kR>
-__device__ __forceinline__ void argmax_block(RunAcc& a, const uint4 (&r)[kR], int n, const int (&v0)[kR]) {
+// Fold a tile into a first-argmax accumulator; v0 is the row index of the
+// first element of the thread's vector j = 0, later vectors follow at
+// kTileThreads vectors' distance (increasing indices).
+template <bool kBf16>
+__device__ __forceinline__ void argmax_tile(RunAcc& a, const uint4 (&r)[kTileRegs], int v0) {
+  using V = Vec16<kBf16>;
+  const float tm = tile_max<kBf16>(r);
+  if (tm != tm) {
+    a.bad = 1;
+    return;
+  }
+  if (tm > a.m) {
+    a.m = tm;
+    int arg = 0x7fffffff;
 #pragma unroll
-  for (int j = 0; j < kR; ++j)
-    if (j < n) argmax_vec<kBf16>(a, r[j], v0[j]);
+    for (int j = kTileRegs - 1; j >= 0; --j)
+#pragma unroll
+      for (int e = V::kN - 1; e >= 0; --e)
+        if (V::at(r[j], e) == tm) arg = v0 + j * kTileThreads * V::kN + e;
+    a.arg = arg;
+  }
 }
 
 __device__ __forceinline__ void lse_scalar(RunAcc& a, float z, float c) {
@@ -193,9 +189,8 @@ __device__ __forceinline__ void lse_scalar(RunAcc& a, float z, float c) {
     a.bad = 1;
     return;
   }
-  if (z == -INFINITY) return;
-  if (z > a.m) lift_max(a, z, c);
-  a.s.x += ex2_approx((z - a.m) * c);
+  if (z > a.m) lift_ref(a, z, c);
+  a.s.x += ex2_approx(fmaf(z, c, -a.R));
 }
 
 __device__ __forceinline__ void argmax_scalar(RunAcc& a, float z, int v) {
@@ -203,14 +198,52 @@ __device__ __forceinline__ void argmax_scalar(RunAcc& a, float z, int v) {
     a.bad = 1;
     return;
   }
-  if (z > a.m) {
+  // the head elements are visited after the body: keep the lowest index on ties
+  if (z > a.m || (z == a.m && v < a.arg)) {
     a.m = z;
     a.arg = v;
   }
 }
 
-// Geometry of one row: unaligned head elements, 16-byte body vectors, tail;
-// the body is split into nseg segments, each staged in pieces of kStageVec.
+// Merge partial b into a.  Softmax rows: sums relative to R(m); greedy rows:
+// the larger maximum wins, ties keep the lower index.
+__device__ __forceinline__ void merge_ref(RowAcc& a, const RowAcc& b, bool argmax, float c) {
+  a.bad |= b.bad;
+  if (argmax) {
+    if (b.m > a.m || (b.m == a.m && b.arg < a.arg)) {
+      a.m = b.m;
+      a.arg = b.arg;
+    }
+    return;
+  }
+  float mh = a.m, sh = a.s, ml = b.m, sl = b.s;
+  if (ml > mh) {
+    mh = b.m;
+    sh = b.s;
+    ml = a.m;
+    sl = a.s;
+  }
+  if (ml != -INFINITY) sh += sl * exp2_int(ref_exp(ml, c) - ref_exp(mh, c));
+  a.m = mh;
+  a.s = sh;
+}
+
+__device__ __forceinline__ RowAcc shfl_down_acc(const RowAcc& a, int off) {
+  RowAcc o;
+  o.m = __shfl_down_sync(0xffffffffu, a.m, off);
+  o.s = __shfl_down_sync(0xffffffffu, a.s, off);
+  o.arg = __shfl_down_sync(0xffffffffu, a.arg, off);
+  o.bad = __shfl_down_sync(0xffffffffu, a.bad, off);
+  return o;
+}
+
+__device__ __forceinline__ void warp_merge(RowAcc& a, bool argmax, float c) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) merge_ref(a, shfl_down_acc(a, off), argmax, c);
+}
+
+// Geometry of one row: unaligned head elements, then 16-byte body vectors,
+// then the tail.
 template <bool kBf16>
 struct RowGeom {
   int head, nvec, tail0;
@@ -222,19 +255,8 @@ struct RowGeom {
     nvec = (V - head) / Vec16<kBf16>::kN;
     tail0 = head + nvec * Vec16<kBf16>::kN;
   }
-  // Vectors [k0, k1) of segment `seg` of `nseg`.
-  __device__ __forceinline__ void segment(int seg, int nseg, int& k0, int& k1) const {
-    const int cs = (nvec + nseg - 1) / nseg;
-    k0 = min(nvec, seg * cs);
-    k1 = min(nvec, k0 + cs);
-  }
-  __device__ __forceinline__ int stages(int seg, int nseg) const {
-    int k0, k1;
-    segment(seg, nseg, k0, k1);
-    return (k1 - k0 + kStageVec - 1) / kStageVec;
-  }
-  __device__ __forceinline__ const char* vec_ptr(const char* rp, int k) const {
-    return rp + static_cast<size_t>(head) * (kBf16 ? 2 : 4) + static_cast<size_t>(k) * 16;
+  __device__ __forceinline__ const uint4* body(const char* rp) const {
+    return reinterpret_cast<const uint4*>(rp + static_cast<size_t>(head) * (kBf16 ? 2 : 4));
   }
 };
 
