@@ -93,6 +93,11 @@ __device__ __forceinline__ unsigned ticket_release(unsigned* p) {
   asm volatile("atom.add.release.gpu.global.u32 %0, [%1], 1;" : "=r"(old) : "l"(p) : "memory");
   return old;
 }
+__device__ __forceinline__ unsigned ticket_add_release(unsigned* p, unsigned n) {
+  unsigned old;
+  asm volatile("atom.add.release.gpu.global.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(n) : "memory");
+  return old;
+}
 __device__ __forceinline__ void fence_acquire() {
   asm volatile("fence.acq_rel.gpu;" ::: "memory");
 }
@@ -263,6 +268,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
       : "r"(smem_addr(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Probe of phase `parity` that may suspend the thread for up to about
+// `ns` nanoseconds while the phase is incomplete (fewer polling instructions).
+__device__ __forceinline__ bool mbar_try_wait_for(uint64_t* bar, uint32_t parity, uint32_t ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_addr(bar)), "r"(parity), "r"(ns)
       : "memory");
   return ok != 0;
 }

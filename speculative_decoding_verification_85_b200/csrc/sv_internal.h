@@ -30,8 +30,8 @@ struct alignas(16) SeqInfo {
   float zmp;    // raw max of target row j
   float zmq;    // raw max of draft row j (residual)
   float c;      // log2(e) / T
-  float isp;    // 1 / (target row's scaled sum): p_v = 2^{(z_v - zmp) c} isp
-  float isq;    // 1 / (draft row's scaled sum)
+  float lsp;    // log2 of the target row's scaled sum: p_v = 2^{(z_v - zmp) c - lsp}
+  float lsq;    // log2 of the draft row's scaled sum
   float pad;
 };
 
@@ -80,9 +80,12 @@ struct MdParams {
 // fixed size at offset 0 (one slot per sequence, up to SV_MAX_BATCH), so their
 // position does not depend on the shape: every call leaves them at zero and a
 // later call of any shape finds zeroed counters.
-// Header: 256 reserved bytes, then the per-sequence row-kernel and
-// draw-kernel arrival counters.
+// Header: 256 bytes of control words, then the per-sequence row-kernel and
+// draw-kernel arrival counters.  Control word kHeaderError collects
+// device-side error bits; it is sticky (never cleared by a call).
 constexpr size_t kHeaderCtl = 256;
+constexpr int kHeaderError = 2;
+constexpr unsigned kErrStageTimeout = 1u;  // a bulk-copy wait gave up
 constexpr size_t kHeaderBytes = kHeaderCtl + 2 * static_cast<size_t>(SV_MAX_BATCH) * sizeof(unsigned);
 
 struct Layout {

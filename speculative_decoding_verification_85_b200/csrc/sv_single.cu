@@ -143,10 +143,10 @@ __device__ __noinline__ void decide_single(const Pass1Params& p, int b, const Ro
       si.j = j;
       si.c = c;
       si.zmp = rows[j].m;
-      si.isp = __frcp_rn(rows[j].s);
+      si.lsp = static_cast<float>(log2(static_cast<double>(rows[j].s)));
       if (j < g) {
         si.zmq = rows[g + 1 + j].m;
-        si.isq = __frcp_rn(rows[g + 1 + j].s);
+        si.lsq = static_cast<float>(log2(static_cast<double>(rows[g + 1 + j].s)));
       }
     }
     p.info[b] = si;
@@ -429,6 +429,7 @@ struct Block4<true> {
     const uint32_t x = w < 2 ? r.x : r.y;
     return (w & 1) ? bf16_hi(x) : bf16_lo(x);
   }
+  __device__ __forceinline__ void set_neg_inf() { r = make_uint2(0xFF80FF80u, 0xFF80FF80u); }
 };
 
 template <>
@@ -449,16 +450,64 @@ struct Block4<false> {
   __device__ __forceinline__ float at(int w) const {
     return w == 0 ? r.x : (w == 1 ? r.y : (w == 2 ? r.z : r.w));
   }
+  __device__ __forceinline__ void set_neg_inf() { r = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY); }
 };
 
+// Running winner of an exponential race: best weight / exponential pair and
+// index, and a slightly lowered copy of the winning ratio for the cheap
+// pre-test.
+struct Race {
+  float bw, be;
+  int bi;
+  float lo;  // bw / be (1 - 2^-20): a candidate with w <= lo t cannot win
+  __device__ __forceinline__ void reset() {
+    bw = 0.0f;
+    be = 1.0f;
+    bi = INT_MAX;
+    lo = 0.0f;
+  }
+  // Exact test of candidate v (weight w > 0, Philox word x).
+  __device__ __forceinline__ void offer(float w, uint32_t x, int v) {
+    const float e = exponential_from_bits(x);
+    if (race_better(w, e, v, bw, be, bi)) {
+      bw = w;
+      be = e;
+      bi = v;
+      lo = fmaxf(lo, __fdiv_rn(bw, be) * (1.0f - 0x1p-20f));
+    }
+  }
+};
+
+// Candidates of one Philox block (entries v0 .. v0 + 3).  Every entry runs the
+// cheap test: w > 0 and, since E >= t = 1 - U, w / t must beat the winner's
+// ratio (lowered, so the test never drops a possible winner); only entries
+// that pass take the logarithm.  The test is branch-free, so lanes of a warp
+// diverge only on the rare exact path.
+__device__ __forceinline__ void race_block(Race& race, const float (&w)[4], const uint4& rnd, int v0) {
+  bool pass[4];
+  bool any = false;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    pass[k] = (w[k] > 0.0f) & (w[k] > race.lo * gumbel_one_minus_u(word_of(rnd, k)));
+    any |= pass[k];
+  }
+  if (any) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      if (pass[k]) race.offer(w[k], word_of(rnd, k), v0 + k);
+  }
+}
+
 // Exponential race over Philox blocks [g0, g1) of the draw row(s): the winner
-// of w_v / E_v (E_v = -ln U_v) with w = max(p - q, 0) (residual) or
-// w = 2^{(z - max) c} (bonus).  Each thread loads all of its blocks before
-// using any of them.  A candidate is skipped without its logarithm when even
-// the bound E_v >= 1 - U_v cannot beat the current best.
+// of w_v / E_v (E_v = -ln U_v) with w = max(p - q, 0) (residual) or w = p
+// (bonus), p_v = 2^{(z_v - zmp) c - lsp}.  Two blocks per step, so that their
+// Philox chains interleave.  After every step the lanes of a warp share the
+// best lowered ratio: a candidate that cannot beat some lane's winner cannot
+// be the overall winner, so the shared value is a valid, much higher, bar for
+// the pre-test (each lane still reports its own best among what it tested).
 template <bool kBf16>
 __device__ __forceinline__ void race_chunk(const SingleParams& f, const SeqInfo& si, int b, int g0,
-                                           int g1, float& bw, float& be, int& bi) {
+                                           int g1, Race& race) {
   constexpr uintptr_t kVecAlign = kBf16 ? 8 : 16;
   const Pass1Params& p = f.p1;
   const char* trow = target_row<kBf16>(p, b, si.j);
@@ -466,51 +515,55 @@ __device__ __forceinline__ void race_chunk(const SingleParams& f, const SeqInfo&
   const char* drow = resid ? draft_row<kBf16>(p, b, si.j) : trow;
   const bool tvec = (reinterpret_cast<uintptr_t>(trow) % kVecAlign) == 0;
   const bool dvec = (reinterpret_cast<uintptr_t>(drow) % kVecAlign) == 0;
-  Block4<kBf16> zt[kDrawMaxBlocks], zd[kDrawMaxBlocks];
-  const int gb = g0 + static_cast<int>(threadIdx.x);
-#pragma unroll
-  for (int u = 0; u < kDrawMaxBlocks; ++u) {
-    const int g = gb + u * kDrawThreads;
+  const float c = si.c, zmp = si.zmp, zmq = si.zmq, lsp = si.lsp, lsq = si.lsq;
+  const int steps = (g1 - g0 + 2 * kDrawThreads - 1) / (2 * kDrawThreads);  // uniform
+  for (int it = 0; it < steps; ++it) {
+    const int g = g0 + it * 2 * kDrawThreads + static_cast<int>(threadIdx.x);
+    const int gh = g + kDrawThreads;
+    Block4<kBf16> t0, t1, d0, d1;
+    t0.set_neg_inf();
+    t1.set_neg_inf();
+    d0.set_neg_inf();
+    d1.set_neg_inf();
     if (g < g1) {
-      zt[u].load(trow, tvec, p.V, g);
-      if (resid) zd[u].load(drow, dvec, p.V, g);
+      t0.load(trow, tvec, p.V, g);
+      if (resid) d0.load(drow, dvec, p.V, g);
     }
-  }
+    if (gh < g1) {
+      t1.load(trow, tvec, p.V, gh);
+      if (resid) d1.load(drow, dvec, p.V, gh);
+    }
+    const uint4 r0 = keyed_block(p.seed, p.step, kTagGumbel, b, 0, si.j, g);
+    const uint4 r1 = keyed_block(p.seed, p.step, kTagGumbel, b, 0, si.j, gh);
+    float w0[4], w1[4];
 #pragma unroll
-  for (int u = 0; u < kDrawMaxBlocks; ++u) {
-    const int g = gb + u * kDrawThreads;
-    if (g >= g1) break;
-    const uint4 rnd = keyed_block(p.seed, p.step, kTagGumbel, b, 0, si.j, g);
-#pragma unroll
-    for (int w = 0; w < 4; ++w) {
-      float wt = ex2_approx((zt[u].at(w) - si.zmp) * si.c);
-      if (resid) wt = wt * si.isp - ex2_approx((zd[u].at(w) - si.zmq) * si.c) * si.isq;
-      if (!(wt > 0.0f)) continue;
-      const uint32_t x = word_of(rnd, w);
-      if (bw > 0.0f && wt * be <= bw * gumbel_one_minus_u(x)) continue;
-      const float e = exponential_from_bits(x);
-      const int v = 4 * g + w;
-      if (race_better(wt, e, v, bw, be, bi)) {
-        bw = wt;
-        be = e;
-        bi = v;
+    for (int k = 0; k < 4; ++k) {
+      w0[k] = ex2_approx(fmaf(t0.at(k) - zmp, c, -lsp));
+      w1[k] = ex2_approx(fmaf(t1.at(k) - zmp, c, -lsp));
+      if (resid) {
+        w0[k] -= ex2_approx(fmaf(d0.at(k) - zmq, c, -lsq));
+        w1[k] -= ex2_approx(fmaf(d1.at(k) - zmq, c, -lsq));
       }
     }
+    race_block(race, w0, r0, 4 * g);
+    race_block(race, w1, r1, 4 * gh);
+    float lo = race.lo;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) lo = fmaxf(lo, __shfl_xor_sync(0xffffffffu, lo, off));
+    race.lo = lo;
   }
 }
 
 // Fallback draw over a whole target row (the residual vanished: p_j == q_j
 // to rounding): bonus-style race over p_j, by one CTA.
 template <bool kBf16>
-__device__ void race_row(const SingleParams& f, SeqInfo si, int b, float& bw, float& be, int& bi) {
+__device__ void race_row(const SingleParams& f, SeqInfo si, int b, Race& race) {
   si.mode = kModeBonus;
-  const int nblocks = (f.p1.V + 3) / 4;
-  for (int g0 = 0; g0 < nblocks; g0 += kDrawMaxBlocks * kDrawThreads)
-    race_chunk<kBf16>(f, si, b, g0, min(nblocks, g0 + kDrawMaxBlocks * kDrawThreads), bw, be, bi);
+  race_chunk<kBf16>(f, si, b, 0, (f.p1.V + 3) / 4, race);
 }
 
 template <bool kBf16>
-__global__ void __launch_bounds__(kDrawThreads) draw_kernel(const __grid_constant__ SingleParams f) {
+__global__ void __launch_bounds__(kDrawThreads, kBf16 ? 5 : 4) draw_kernel(const __grid_constant__ SingleParams f) {
   __shared__ float4 scratch[kDrawThreads / 32];
   __shared__ int s_last;
   pdl_wait_and_release();  // the row kernel has completed: every decision is visible
@@ -525,17 +578,19 @@ __global__ void __launch_bounds__(kDrawThreads) draw_kernel(const __grid_constan
   si.zmp = w0.z;
   si.zmq = w0.w;
   si.c = w1.x;
-  si.isp = w1.y;
-  si.isq = w1.z;
+  si.lsp = w1.y;
+  si.lsq = w1.z;
   const bool draw = (si.mode == kModeResidual && si.j >= 0 && si.j < p.gamma) ||
                     (si.mode == kModeBonus && si.j == p.gamma);
   if (!draw) return;  // uniform: greedy or invalid sequence
   const int nblocks = (p.V + 3) / 4;
   const int g0 = chunk * (f.chunk2 / 4);
   const int g1 = min(nblocks, g0 + f.chunk2 / 4);
-  float bw = 0.0f, be = 1.0f;
-  int bi = INT_MAX;
-  race_chunk<kBf16>(f, si, b, g0, g1, bw, be, bi);
+  Race race;
+  race.reset();
+  race_chunk<kBf16>(f, si, b, g0, g1, race);
+  float bw = race.bw, be = race.be;
+  int bi = race.bi;
   race_reduce<kDrawThreads>(bw, be, bi, scratch);
   if (threadIdx.x == 0) {
     RacePartial* pp = f.part2 + static_cast<size_t>(b) * f.nc2 + chunk;
@@ -560,10 +615,11 @@ __global__ void __launch_bounds__(kDrawThreads) draw_kernel(const __grid_constan
   }
   race_reduce<kDrawThreads>(bw, be, bi, scratch);
   if (!(bw > 0.0f)) {  // uniform: race_reduce returns the winner to every thread
-    bw = 0.0f;
-    be = 1.0f;
-    bi = INT_MAX;
-    race_row<kBf16>(f, si, b, bw, be, bi);
+    race.reset();
+    race_row<kBf16>(f, si, b, race);
+    bw = race.bw;
+    be = race.be;
+    bi = race.bi;
     race_reduce<kDrawThreads>(bw, be, bi, scratch);
   }
   if (threadIdx.x == 0) p.out_tokens[static_cast<size_t>(b) * (p.gamma + 1) + si.j] = bi;
