@@ -164,6 +164,34 @@ int spec_verify_host(const void* target_logits, const void* draft_logits,
                      int32_t* out_tokens, float* out_target_logp, float* out_draft_logp,
                      void* staging, size_t staging_bytes, void* stream);
 
+/*
+ * spec_verify_noalloc -- spec_verify for callers that cannot allocate device
+ * memory at verification time (an engine that reserves almost all of the
+ * GPU's memory up front for weights and KV cache, or a decode path that must
+ * never enter an allocator).  Not an operation of the source pages: it is
+ * spec_verify with the same inputs, outputs and results, but the scratch
+ * space comes from a fixed array of SV_NOALLOC_MAX_WORKSPACE bytes in the
+ * library's own device memory (one per device, present once the library is
+ * loaded) instead of a caller workspace.  The call allocates nothing.
+ *   - Size limit: shapes whose spec_verify_workspace_size exceeds
+ *     SV_NOALLOC_MAX_WORKSPACE (8 MiB; for example B = 256, gamma = 4,
+ *     V = 151936 bf16 needs about 2.1 MB) return SV_ERR_WORKSPACE and launch
+ *     nothing; use spec_verify with a caller workspace for those.
+ *   - First call per device: it looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current) and clears its counter
+ *     header on `stream`.  Make that first call before any stream capture.
+ *   - Concurrency: all calls on one device share the array, so two calls
+ *     that may overlap on the GPU (different streams without ordering) race
+ *     and their results are undefined.  Order them on one stream.
+ */
+#define SV_NOALLOC_MAX_WORKSPACE (8u << 20)
+size_t spec_verify_noalloc_max_workspace(void);
+int spec_verify_noalloc(const void* target_logits, const void* draft_logits,
+                        const int32_t* draft_tokens, const float* temps, int B, int gamma,
+                        int V, int dtype, uint64_t seed, uint64_t step, int32_t* out_accept_len,
+                        int32_t* out_tokens, float* out_target_logp, float* out_draft_logp,
+                        void* stream);
+
 #ifdef __cplusplus
 }
 #endif

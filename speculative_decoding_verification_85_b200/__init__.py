@@ -9,10 +9,12 @@ device, raises.
 """
 from ._binding import (  # noqa: F401
     BF16, F32, SpecVerifyError, Verifier, lib, library_path, multidraft_workspace_size,
-    spec_verify, spec_verify_host, spec_verify_multidraft, staging_size, workspace_size,
+    spec_verify, spec_verify_host, spec_verify_multidraft, spec_verify_noalloc,
+    spec_verify_noalloc_max_workspace, staging_size, workspace_size,
 )
 
 __all__ = [
     "spec_verify", "spec_verify_multidraft", "spec_verify_host", "Verifier", "workspace_size",
     "multidraft_workspace_size", "staging_size", "SpecVerifyError", "lib", "library_path",
+    "spec_verify_noalloc", "spec_verify_noalloc_max_workspace",
 ]

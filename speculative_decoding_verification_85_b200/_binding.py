@@ -53,6 +53,11 @@ def lib() -> C.CDLL:
             L.spec_verify_host.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, u64, u64, vp, vp,
                                            vp, vp, vp, sz, vp]
             L.spec_verify_host.restype = i32
+            L.spec_verify_noalloc_max_workspace.argtypes = []
+            L.spec_verify_noalloc_max_workspace.restype = sz
+            L.spec_verify_noalloc.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, u64, u64, vp, vp,
+                                              vp, vp, vp]
+            L.spec_verify_noalloc.restype = i32
             _lib = L
     return _lib
 
@@ -196,6 +201,32 @@ def spec_verify_host(target, draft, tokens, temps, *, staging, seed: int = 0, st
                                   staging.numel() * staging.element_size(),
                                   _stream(staging.device, stream)))
     return out_accept_len, out_tokens, lp, lq
+
+
+def spec_verify_noalloc(target, draft, tokens, temps, *, seed: int = 0, step: int = 0,
+                        out_accept_len, out_tokens, out_target_logp=None, out_draft_logp=None,
+                        stream=None):
+    """spec_verify for callers that cannot allocate device memory while they
+    verify (memory reserved up front for weights and KV cache, or a decode
+    path that must not enter an allocator): the scratch space is a fixed
+    array inside the library (``spec_verify_noalloc_max_workspace()`` bytes
+    per device), so the call allocates nothing.  Every output tensor must be
+    passed in.  The first call on a device sets that array up (make it before
+    any stream capture); calls that may overlap on the GPU race."""
+    for t, n in ((target, "target"), (draft, "draft"), (tokens, "tokens"), (temps, "temps"),
+                 (out_accept_len, "out_accept_len"), (out_tokens, "out_tokens")):
+        _dev(t, n)
+    B, g1, V = target.shape
+    _check(lib().spec_verify_noalloc(_ptr(target), _ptr(draft), _ptr(tokens), _ptr(temps), B,
+                                     g1 - 1, V, _dt(target), seed, step, _ptr(out_accept_len),
+                                     _ptr(out_tokens), _ptr(out_target_logp),
+                                     _ptr(out_draft_logp), _stream(target.device, stream)))
+    return out_accept_len, out_tokens, out_target_logp, out_draft_logp
+
+
+def spec_verify_noalloc_max_workspace() -> int:
+    """Bytes of the fixed scratch array behind spec_verify_noalloc."""
+    return int(lib().spec_verify_noalloc_max_workspace())
 
 
 class Verifier:

@@ -61,3 +61,16 @@ def test_cpu_tensors_rejected():
     with pytest.raises(ValueError, match="CUDA"):
         sv.spec_verify(t, torch.zeros(1, 2, 8), torch.zeros(1, 2, dtype=torch.int32),
                        torch.ones(1))
+
+
+def test_noalloc_rejects_shapes_beyond_its_fixed_workspace():
+    """Host-side check, before any CUDA call: a shape whose workspace exceeds
+    the fixed array is refused with SV_ERR_WORKSPACE."""
+    L = sv.lib()
+    assert sv.spec_verify_noalloc_max_workspace() == 8 << 20
+    B, g, V = 2048, 8, 128256
+    assert sv.workspace_size(B, g, V, sv.BF16) > sv.spec_verify_noalloc_max_workspace()
+    rc = L.spec_verify_noalloc(None, None, None, None, B, g, V, sv.BF16, 0, 0, None, None, None,
+                               None, None)
+    assert rc == 4
+    assert b"fixed" in L.spec_verify_last_error()
