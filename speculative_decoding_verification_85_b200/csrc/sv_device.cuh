@@ -93,9 +93,12 @@ __device__ __forceinline__ unsigned ticket_release(unsigned* p) {
   asm volatile("atom.add.release.gpu.global.u32 %0, [%1], 1;" : "=r"(old) : "l"(p) : "memory");
   return old;
 }
-__device__ __forceinline__ unsigned ticket_add_release(unsigned* p, unsigned n) {
+// Arrival ticket with acquire-release semantics: releases this thread's
+// earlier stores and, for the last arriver, acquires everything the earlier
+// arrivers released (a CTA barrier then extends that to the whole CTA).
+__device__ __forceinline__ unsigned ticket_acq_rel(unsigned* p) {
   unsigned old;
-  asm volatile("atom.add.release.gpu.global.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(n) : "memory");
+  asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], 1;" : "=r"(old) : "l"(p) : "memory");
   return old;
 }
 __device__ __forceinline__ void fence_acquire() {

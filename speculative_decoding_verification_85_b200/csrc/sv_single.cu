@@ -36,14 +36,14 @@ __device__ __forceinline__ double accept_prob(double lp, double lq) {
 }
 
 // Warp 0 of the last-arriving CTA: validate, accept/reject, write outputs.
+// T is sequence b's temperature and x[0..gamma) its draft tokens (staged in
+// shared memory by the caller).
 template <bool kBf16>
-__device__ __noinline__ void decide_single(const Pass1Params& p, int b, const RowAcc* rows,
-                                           const float* zsel) {
+__device__ __noinline__ void decide_single(const Pass1Params& p, int b, float T, const int* x,
+                                           const RowAcc* rows, const float* zsel) {
   const int lane = threadIdx.x & 31;
   const int g = p.gamma;
-  const float T = __ldg(p.temps + b);
   const bool tvalid = (T >= 0.0f) && !isinf(T);
-  const int32_t* x = p.tokens + static_cast<size_t>(b) * g;
   int32_t* tok = p.out_tokens + static_cast<size_t>(b) * (g + 1);
 
   bool ok = tvalid;
@@ -52,7 +52,7 @@ __device__ __noinline__ void decide_single(const Pass1Params& p, int b, const Ro
   for (int h = 0; h < 2; ++h) {
     const int i = lane + 32 * h;
     if (i < g) {
-      xi[h] = __ldg(x + i);
+      xi[h] = x[i];
       ok = ok && xi[h] >= 0 && xi[h] < p.V;
     }
   }
@@ -143,10 +143,10 @@ __device__ __noinline__ void decide_single(const Pass1Params& p, int b, const Ro
       si.j = j;
       si.c = c;
       si.zmp = rows[j].m;
-      si.lsp = static_cast<float>(log2(static_cast<double>(rows[j].s)));
+      si.lsp = log2f(rows[j].s);
       if (j < g) {
         si.zmq = rows[g + 1 + j].m;
-        si.lsq = static_cast<float>(log2(static_cast<double>(rows[g + 1 + j].s)));
+        si.lsq = log2f(rows[g + 1 + j].s);
       }
     }
     p.info[b] = si;
@@ -166,7 +166,7 @@ struct SingleParams {
   RacePartial* part2;   // [B][nc2] draw partials
   unsigned* ticket2;    // [B] draw arrivals
   int nc2;              // draw CTAs per sequence
-  int chunk2;           // vocabulary entries per draw CTA (multiple of 4 * kDrawThreads)
+  int chunk2;           // vocabulary entries per draw CTA (a multiple of 4)
   int nseg;             // row segments per row (gridDim.y of the row kernel)
   int segvec;           // 16-byte vectors per row segment (multiple of kTileVec)
   float4* pairpart;     // [B][gamma + 1][nseg] x {target, draft} partials
@@ -193,78 +193,88 @@ __device__ __forceinline__ void pdl_wait_and_release() {
   asm volatile("griddepcontrol.launch_dependents;");
 }
 
-// Block reduction of the two rows' accumulators (one barrier); the result is
+// Empty partials: softmax rows carry R = -inf in the index slot.
+__device__ __forceinline__ RowAcc empty_lse_acc() {
+  return RowAcc{-INFINITY, 0.0f, __float_as_int(-INFINITY), 0};
+}
+__device__ __forceinline__ RowAcc empty_argmax_acc() { return RowAcc{-INFINITY, 0.0f, 0x7fffffff, 0}; }
+
+// Block reduction of the two rows' accumulators: a butterfly within each
+// warp, then warp 0 merges the 8 warp results of each row by a 3-step
+// butterfly (lanes 0-7 row A, lanes 8-15 row B).  One barrier; the result is
 // valid in thread 0.
-__device__ __forceinline__ void reduce_pair(RowAcc& A, RowAcc& B, bool argmaxA, float c,
-                                            RowAcc* scratch) {
+__device__ __forceinline__ void reduce_pair(RowAcc& A, RowAcc& B, bool argmaxA, RowAcc* scratch) {
+  constexpr int W = kRowThreads / 32;  // 8 warps
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  warp_merge(A, argmaxA, c);
-  warp_merge(B, false, c);
+  warp_merge(A, argmaxA);
+  warp_merge(B, false);
   if (lane == 0) {
-    scratch[2 * warp] = A;
-    scratch[2 * warp + 1] = B;
+    scratch[warp] = A;
+    scratch[W + warp] = B;
   }
   block_sync<kRowThreads>();
-  if (threadIdx.x == 0) {
-    for (int w = 1; w < kRowThreads / 32; ++w) {
-      merge_ref(A, scratch[2 * w], argmaxA, c);
-      merge_ref(B, scratch[2 * w + 1], false, c);
+  if (warp == 0) {
+    const bool rowB = lane >= W;
+    RowAcc v = lane < 2 * W ? scratch[lane] : empty_lse_acc();
+    group_merge<W>(v, rowB ? false : argmaxA);
+    const RowAcc vb = shfl_xor_acc(v, W);  // lane 0 receives lane 8's row-B result
+    if (lane == 0) {
+      A = v;
+      B = vb;
     }
   }
 }
 
-// The softmax sum relative to the row maximum, s = S 2^{R(m) - m c}, from a
-// sum S relative to the reference R(m) (fp64 scaling).
+// The softmax sum relative to the row maximum, s = S 2^{R - m c}, from a
+// merged softmax partial {m, S, R}.  R - m c lies in [0, 1) up to rounding
+// (R is the reference of the row maximum), so one ex2 of that small argument
+// (computed in fp64) keeps the relative error near 2^-22.
 __device__ __forceinline__ float sum_rel_max(const RowAcc& a, float c) {
-  if (!(a.m > -INFINITY) || isinf(a.m)) return a.s;  // invalid row: left to the decision
-  const double sh = exp2(static_cast<double>(ref_exp(a.m, c)) -
-                         static_cast<double>(a.m) * static_cast<double>(c));
-  return static_cast<float>(static_cast<double>(a.s) * sh);
+  const float R = __int_as_float(a.arg);
+  if (!isfinite(a.m) || !isfinite(R)) return a.s;  // invalid row: left to the decision
+  const float e = static_cast<float>(static_cast<double>(R) - static_cast<double>(a.m) * static_cast<double>(c));
+  return a.s * ex2_approx(e);
 }
 
-// Combine the nseg pair partials of every position of sequence b into the
+// Combine the nseg segment partials of every position of sequence b into the
 // row table rows[] (target rows 0..gamma, then draft rows), and pick up the
-// draft tokens' logits (zsel[2i], zsel[2i+1]).
-__device__ __forceinline__ void combine_pairs(const SingleParams& f, int b, RowAcc* rows,
-                                              float* zsel) {
+// draft tokens' logits (zsel[2i], zsel[2i+1]).  argmaxA and c describe the
+// sequence (greedy or softmax, c = log2(e) / T).
+__device__ __forceinline__ void combine_pairs(const SingleParams& f, int b, bool argmaxA, float c,
+                                              RowAcc* rows, float* zsel) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int g = f.p1.gamma;
-  const float T = __ldg(f.p1.temps + b);
-  const bool argmaxA = row_mode(T, true) == kRowArgmax;
-  const float c = row_mode(T, true) == kRowLse ? __fdiv_rn(kLog2e, T) : 0.0f;
   for (int i = warp; i <= g; i += kRowThreads / 32) {
-    RowAcc A{-INFINITY, 0.0f, 0x7fffffff, 0}, B{-INFINITY, 0.0f, 0x7fffffff, 0};
+    RowAcc A = argmaxA ? empty_argmax_acc() : empty_lse_acc(), B = empty_lse_acc();
+    float zt = __int_as_float(0x7fc00000), zd = zt;
     const float4* pp = f.pairpart + (static_cast<size_t>(b) * (g + 1) + i) * f.nseg * 2;
+    const float* zp = f.zx + (static_cast<size_t>(b) * g + i) * f.nseg * 2;
     for (int q = lane; q < f.nseg; q += 32) {
       const float4 a = __ldcg(pp + 2 * q), d = __ldcg(pp + 2 * q + 1);
-      merge_ref(A, RowAcc{a.x, a.y, __float_as_int(a.z), __float_as_int(a.w)}, argmaxA, c);
-      merge_ref(B, RowAcc{d.x, d.y, __float_as_int(d.z), __float_as_int(d.w)}, false, c);
+      merge_ref(A, RowAcc{a.x, a.y, __float_as_int(a.z), __float_as_int(a.w)}, argmaxA);
+      merge_ref(B, RowAcc{d.x, d.y, __float_as_int(d.z), __float_as_int(d.w)}, false);
+      if (i < g) {
+        // the draft token's logits: the one segment that holds it reports them
+        const float za = __ldcg(zp + 2 * q), zb = __ldcg(zp + 2 * q + 1);
+        if (za == za) zt = za;
+        if (zb == zb) zd = zb;
+      }
     }
-    warp_merge(A, argmaxA, c);
-    warp_merge(B, false, c);
+    warp_merge(A, argmaxA);
+    warp_merge(B, false);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      const float a = __shfl_xor_sync(0xffffffffu, zt, off);
+      const float d = __shfl_xor_sync(0xffffffffu, zd, off);
+      if (zt != zt) zt = a;
+      if (zd != zd) zd = d;
+    }
     if (lane == 0) {
       if (!argmaxA) A.s = sum_rel_max(A, c);
       B.s = sum_rel_max(B, c);
       rows[i] = A;
-      if (i < g) rows[g + 1 + i] = B;
-    }
-    if (i < g) {
-      // the draft token's logits: the one segment that holds it reports them
-      float zt = __int_as_float(0x7fc00000), zd = zt;
-      const float* zp = f.zx + (static_cast<size_t>(b) * g + i) * f.nseg * 2;
-      for (int q = lane; q < f.nseg; q += 32) {
-        const float a = __ldcg(zp + 2 * q), d = __ldcg(zp + 2 * q + 1);
-        if (a == a) zt = a;
-        if (d == d) zd = d;
-      }
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) {
-        const float a = __shfl_down_sync(0xffffffffu, zt, off);
-        const float d = __shfl_down_sync(0xffffffffu, zd, off);
-        if (zt != zt) zt = a;
-        if (zd != zd) zd = d;
-      }
-      if (lane == 0) {
+      if (i < g) {
+        rows[g + 1 + i] = B;
         zsel[2 * i] = zt;
         zsel[2 * i + 1] = zd;
       }
@@ -323,6 +333,7 @@ __global__ void __launch_bounds__(kRowThreads, 3) rows_kernel(const __grid_const
   __shared__ RowAcc scratch[2 * (kRowThreads / 32)];
   __shared__ float s_zx[2];
   __shared__ float s_zsel[2 * SV_MAX_GAMMA];
+  __shared__ int s_tok[SV_MAX_GAMMA];
   __shared__ int s_last;
   pdl_wait_and_release();
   const Pass1Params& p = f.p1;
@@ -343,6 +354,8 @@ __global__ void __launch_bounds__(kRowThreads, 3) rows_kernel(const __grid_const
     if (xt >= 0 && xt < p.V) xg = xt;
   }
   if (tid == 0) s_zx[0] = s_zx[1] = __int_as_float(0x7fc00000);  // NaN: "not in this segment"
+  // the sequence's draft tokens, for the decision if this CTA completes it
+  for (int k = tid; k < p.gamma; k += kRowThreads) s_tok[k] = __ldg(p.tokens + static_cast<size_t>(b) * p.gamma + k);
   block_sync<kRowThreads>();
 
   RunAcc accA, accB;
@@ -380,8 +393,8 @@ __global__ void __launch_bounds__(kRowThreads, 3) rows_kernel(const __grid_const
   if (loadB && (first || last))
     row_edges<kBf16>(rpB, p.V, gB, false, c, first, last, xg, &s_zx[1], accB);
 
-  RowAcc A = accA.row(), B = accB.row();
-  reduce_pair(A, B, argmaxA, c, scratch);
+  RowAcc A = argmaxA ? accA.argmax_row() : accA.lse_row(), B = accB.lse_row();
+  reduce_pair(A, B, argmaxA, scratch);
   if (tid == 0) {
     float4* pp = f.pairpart + ((static_cast<size_t>(b) * (p.gamma + 1) + i) * f.nseg + seg) * 2;
     pp[0] = make_float4(A.m, A.s, __int_as_float(A.arg), __int_as_float(A.bad));
@@ -391,16 +404,16 @@ __global__ void __launch_bounds__(kRowThreads, 3) rows_kernel(const __grid_const
       z[0] = s_zx[0];
       z[1] = s_zx[1];
     }
-    const unsigned tk = ticket_release(p.ticket + b);
+    // release this CTA's partial; the last arriver also acquires the others'
+    const unsigned tk = ticket_acq_rel(p.ticket + b);
     const unsigned arrivals = static_cast<unsigned>((p.gamma + 1) * f.nseg);
     s_last = (tk == arrivals - 1);
     if (s_last) p.ticket[b] = 0;  // leave the counter at zero for the next call
   }
-  block_sync<kRowThreads>();
+  block_sync<kRowThreads>();  // orders the other threads after thread 0's acquire
   if (!s_last) return;
-  fence_acquire();
-  combine_pairs(f, b, rows, s_zsel);
-  if (tid < 32) decide_single<kBf16>(p, b, rows, s_zsel);
+  combine_pairs(f, b, argmaxA, c, rows, s_zsel);
+  if (tid < 32) decide_single<kBf16>(p, b, T, s_tok, rows, s_zsel);
 }
 
 // -------------------------------------------------------------- draw kernel
@@ -545,6 +558,21 @@ __device__ __forceinline__ void race_chunk(const SingleParams& f, const SeqInfo&
         w1[k] -= ex2_approx(fmaf(d1.at(k) - zmq, c, -lsq));
       }
     }
+    if (it == 0) {
+      // warm start without logarithms: since -ln U <= (1 - U) / U, every
+      // candidate's ratio w / E is at least w U / t (t = 1 - U); the warp's
+      // largest such bound (lowered for rounding) is a valid first bar
+      float lb = 0.0f;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float ta = gumbel_one_minus_u(word_of(r0, k)), tb = gumbel_one_minus_u(word_of(r1, k));
+        lb = fmaxf(lb, __fdividef(w0[k] * (1.0f - ta), ta));
+        lb = fmaxf(lb, __fdividef(w1[k] * (1.0f - tb), tb));
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) lb = fmaxf(lb, __shfl_xor_sync(0xffffffffu, lb, off));
+      race.lo = fmaxf(race.lo, lb * (1.0f - 0x1p-20f));
+    }
     race_block(race, w0, r0, 4 * g);
     race_block(race, w1, r1, 4 * gh);
     float lo = race.lo;
@@ -595,13 +623,12 @@ __global__ void __launch_bounds__(kDrawThreads, kBf16 ? 5 : 4) draw_kernel(const
   if (threadIdx.x == 0) {
     RacePartial* pp = f.part2 + static_cast<size_t>(b) * f.nc2 + chunk;
     *reinterpret_cast<float4*>(pp) = make_float4(bw, be, __int_as_float(bi), 0.0f);
-    const unsigned t = ticket_release(f.ticket2 + b);
+    const unsigned t = ticket_acq_rel(f.ticket2 + b);
     s_last = (t == static_cast<unsigned>(f.nc2 - 1));
     if (s_last) f.ticket2[b] = 0;
   }
-  block_sync<kDrawThreads>();
+  block_sync<kDrawThreads>();  // orders the other threads after thread 0's acquire
   if (!s_last) return;
-  fence_acquire();
   bw = 0.0f;
   be = 1.0f;
   bi = INT_MAX;
@@ -638,7 +665,7 @@ int row_segments(int V, int dtype) { return body_tiles(V, dtype); }  // bound on
 
 int draw_chunks(int V, int dtype) {  // upper bound on draw CTAs per sequence
   (void)dtype;
-  return (V + 4 * kDrawThreads - 1) / (4 * kDrawThreads);
+  return (V + 255) / 256;
 }
 
 namespace {
@@ -667,6 +694,25 @@ int row_ctas_per_sm(bool bf16) {
              : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, rows_kernel<false>, kRowThreads, 0);
     if (e != cudaSuccess) (void)cudaGetLastError();
     slot = (e == cudaSuccess && n > 0) ? n : 3;
+  }
+  return slot;
+}
+
+// Resident draw-kernel CTAs per SM (occupancy query, cached per device).
+int draw_ctas_per_sm(bool bf16) {
+  static std::mutex mu;
+  static int cached[64][2];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 4;
+  std::lock_guard<std::mutex> lk(mu);
+  int& slot = cached[dev][bf16 ? 1 : 0];
+  if (slot == 0) {
+    int n = 0;
+    const cudaError_t e =
+        bf16 ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, draw_kernel<true>, kDrawThreads, 0)
+             : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, draw_kernel<false>, kDrawThreads, 0);
+    if (e != cudaSuccess) (void)cudaGetLastError();
+    slot = (e == cudaSuccess && n > 0) ? n : 4;
   }
   return slot;
 }
@@ -738,17 +784,22 @@ int launch_single(const void* target, const void* draft, const int32_t* tokens,
   f.zx = reinterpret_cast<float*>(ws + lay.resid);
   f.part2 = reinterpret_cast<RacePartial*>(ws + lay.part2);
   f.ticket2 = reinterpret_cast<unsigned*>(ws + lay.ticket2);
-  // Draw chunks: enough CTAs to cover the GPU about twice when the batch is
-  // small, at most kDrawMaxBlocks Philox blocks per thread.
-  const long long want = (2LL * sm_count() + B - 1) / B;
-  const int unit = 4 * kDrawThreads;  // entries per Philox block per thread
-  const int min_chunks = (V + unit * kDrawMaxBlocks - 1) / (unit * kDrawMaxBlocks);
-  long long nc2 = want > min_chunks ? want : min_chunks;
-  if (nc2 > lay.nc2) nc2 = lay.nc2;
-  int chunk = static_cast<int>((V + nc2 - 1) / nc2);
-  chunk = (chunk + unit - 1) / unit * unit;
-  f.chunk2 = chunk;
-  f.nc2 = (V + chunk - 1) / chunk;
+  // Draw chunks: a whole number of waves of the draw kernel over the GPU,
+  // with at most about kDrawMaxBlocks Philox blocks per thread; chunks are
+  // balanced within a sequence (in Philox blocks of 4 entries).
+  {
+    const long long nb = (V + 3) / 4;  // Philox blocks per row
+    const long long slots2 = static_cast<long long>(sm_count()) * draw_ctas_per_sm(bf16);
+    const long long per_cta = static_cast<long long>(kDrawMaxBlocks) * kDrawThreads;
+    const long long waves = (static_cast<long long>(B) * nb + per_cta * slots2 - 1) / (per_cta * slots2);
+    long long nc2 = waves * slots2 / B;
+    if (nc2 < 1) nc2 = 1;
+    if (nc2 > lay.nc2) nc2 = lay.nc2;
+    if (nc2 > nb) nc2 = nb;
+    const long long cb = (nb + nc2 - 1) / nc2;  // blocks per draw CTA
+    f.chunk2 = static_cast<int>(4 * cb);
+    f.nc2 = static_cast<int>((nb + cb - 1) / cb);
+  }
 
   const dim3 grid1(static_cast<unsigned>(B * (gamma + 1)), static_cast<unsigned>(f.nseg));
   cudaError_t e = bf16 ? launch_pdl(rows_kernel<true>, grid1, kRowThreads, stream, f)

@@ -36,9 +36,12 @@ __device__ __forceinline__ uint32_t hmax2_nan(uint32_t a, uint32_t b) {
   return d;
 }
 
-// Exact 2^d for an integral d <= 0 (0 below the normal range).
+// Exact 2^d for an integral d <= 0 (0 below the normal range, and for NaN).
+// The integer is read from the mantissa of d + 1.5 2^23 (no conversion unit).
 __device__ __forceinline__ float exp2_int(float d) {
-  return d < -126.0f ? 0.0f : __int_as_float((static_cast<int>(d) + 127) << 23);
+  if (!(d >= -126.0f)) return 0.0f;
+  const int k = __float_as_int(d + 12582912.0f) - 0x4B400000;
+  return __int_as_float((k + 127) << 23);
 }
 
 // Reference exponent R(m) = ceil(fl(m c)); the same operations everywhere.
@@ -58,7 +61,12 @@ struct RunAcc {
     arg = 0x7fffffff;
     bad = 0;
   }
-  __device__ __forceinline__ RowAcc row() const { return RowAcc{m, s.x + s.y, arg, bad}; }
+  // Greedy rows: {max, -, first index, bad}.
+  __device__ __forceinline__ RowAcc argmax_row() const { return RowAcc{m, 0.0f, arg, bad}; }
+  // Softmax rows: {max, S, R (in the index slot; -inf when empty), bad}.
+  __device__ __forceinline__ RowAcc lse_row() const {
+    return RowAcc{m, s.x + s.y, __float_as_int(m == -INFINITY ? -INFINITY : R), bad};
+  }
 };
 
 // Move the running maximum up to tm (> m): new reference, rescale the sum.
@@ -205,9 +213,11 @@ __device__ __forceinline__ void argmax_scalar(RunAcc& a, float z, int v) {
   }
 }
 
-// Merge partial b into a.  Softmax rows: sums relative to R(m); greedy rows:
-// the larger maximum wins, ties keep the lower index.
-__device__ __forceinline__ void merge_ref(RowAcc& a, const RowAcc& b, bool argmax, float c) {
+// Merge partial b into a.  Softmax rows ({m, S, R, bad}, R in the index
+// slot): the larger maximum, and the sums brought to the larger reference
+// by an exact power of two; greedy rows: the larger maximum wins, ties keep
+// the lower index.
+__device__ __forceinline__ void merge_ref(RowAcc& a, const RowAcc& b, bool argmax) {
   a.bad |= b.bad;
   if (argmax) {
     if (b.m > a.m || (b.m == a.m && b.arg < a.arg)) {
@@ -216,31 +226,33 @@ __device__ __forceinline__ void merge_ref(RowAcc& a, const RowAcc& b, bool argma
     }
     return;
   }
-  float mh = a.m, sh = a.s, ml = b.m, sl = b.s;
-  if (ml > mh) {
-    mh = b.m;
-    sh = b.s;
-    ml = a.m;
-    sl = a.s;
+  a.m = fmaxf(a.m, b.m);
+  const float Ra = __int_as_float(a.arg), Rb = __int_as_float(b.arg);
+  if (Rb > Ra) {
+    a.s = b.s + a.s * exp2_int(Ra - Rb);
+    a.arg = b.arg;
+  } else {
+    a.s += b.s * exp2_int(Rb - Ra);
   }
-  if (ml != -INFINITY) sh += sl * exp2_int(ref_exp(ml, c) - ref_exp(mh, c));
-  a.m = mh;
-  a.s = sh;
 }
 
-__device__ __forceinline__ RowAcc shfl_down_acc(const RowAcc& a, int off) {
+__device__ __forceinline__ RowAcc shfl_xor_acc(const RowAcc& a, int off) {
   RowAcc o;
-  o.m = __shfl_down_sync(0xffffffffu, a.m, off);
-  o.s = __shfl_down_sync(0xffffffffu, a.s, off);
-  o.arg = __shfl_down_sync(0xffffffffu, a.arg, off);
-  o.bad = __shfl_down_sync(0xffffffffu, a.bad, off);
+  o.m = __shfl_xor_sync(0xffffffffu, a.m, off);
+  o.s = __shfl_xor_sync(0xffffffffu, a.s, off);
+  o.arg = __shfl_xor_sync(0xffffffffu, a.arg, off);
+  o.bad = __shfl_xor_sync(0xffffffffu, a.bad, off);
   return o;
 }
 
-__device__ __forceinline__ void warp_merge(RowAcc& a, bool argmax, float c) {
+// Butterfly merge over groups of `width` lanes (every lane ends with its
+// group's result).
+template <int width>
+__device__ __forceinline__ void group_merge(RowAcc& a, bool argmax) {
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) merge_ref(a, shfl_down_acc(a, off), argmax, c);
+  for (int off = width / 2; off > 0; off >>= 1) merge_ref(a, shfl_xor_acc(a, off), argmax);
 }
+__device__ __forceinline__ void warp_merge(RowAcc& a, bool argmax) { group_merge<32>(a, argmax); }
 
 // Geometry of one row: unaligned head elements, then 16-byte body vectors,
 // then the tail.
