@@ -492,22 +492,22 @@ struct Race {
 };
 
 // Candidates of one Philox block (entries v0 .. v0 + 3).  Every entry runs the
-// cheap test: w > 0 and, since E >= t = 1 - U, w / t must beat the winner's
-// ratio (lowered, so the test never drops a possible winner); only entries
-// that pass take the logarithm.  The test is branch-free, so lanes of a warp
-// diverge only on the rare exact path.
+// cheap test w > lo t: since E >= t = 1 - U, w / t must beat the winner's
+// ratio (lowered, so the test never drops a possible winner; with lo >= 0 it
+// also rejects w <= 0).  Only entries that pass take the logarithm.  The test
+// is branch-free, so lanes of a warp diverge only on the rare exact path.
 __device__ __forceinline__ void race_block(Race& race, const float (&w)[4], const uint4& rnd, int v0) {
   bool pass[4];
   bool any = false;
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
-    pass[k] = (w[k] > 0.0f) & (w[k] > race.lo * gumbel_one_minus_u(word_of(rnd, k)));
+    pass[k] = w[k] > race.lo * gumbel_one_minus_u(word_of(rnd, k));
     any |= pass[k];
   }
   if (any) {
 #pragma unroll
     for (int k = 0; k < 4; ++k)
-      if (pass[k]) race.offer(w[k], word_of(rnd, k), v0 + k);
+      if (pass[k] && w[k] > 0.0f) race.offer(w[k], word_of(rnd, k), v0 + k);
   }
 }
 
@@ -548,14 +548,19 @@ __device__ __forceinline__ void race_chunk(const SingleParams& f, const SeqInfo&
     }
     const uint4 r0 = keyed_block(p.seed, p.step, kTagGumbel, b, 0, si.j, g);
     const uint4 r1 = keyed_block(p.seed, p.step, kTagGumbel, b, 0, si.j, gh);
+    // p_v = 2^{(z_v - zmp) c - lsp}, q_v likewise: the target and draft value
+    // of an entry travel as one packed pair
     float w0[4], w1[4];
+    const float2 nm = make_float2(-zmp, -zmq), cc = make_float2(c, c), nl = make_float2(-lsp, -lsq);
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
-      w0[k] = ex2_approx(fmaf(t0.at(k) - zmp, c, -lsp));
-      w1[k] = ex2_approx(fmaf(t1.at(k) - zmp, c, -lsp));
+      const float2 e0 = __ffma2_rn(__fadd2_rn(make_float2(t0.at(k), d0.at(k)), nm), cc, nl);
+      const float2 e1 = __ffma2_rn(__fadd2_rn(make_float2(t1.at(k), d1.at(k)), nm), cc, nl);
+      w0[k] = ex2_approx(e0.x);
+      w1[k] = ex2_approx(e1.x);
       if (resid) {
-        w0[k] -= ex2_approx(fmaf(d0.at(k) - zmq, c, -lsq));
-        w1[k] -= ex2_approx(fmaf(d1.at(k) - zmq, c, -lsq));
+        w0[k] -= ex2_approx(e0.y);
+        w1[k] -= ex2_approx(e1.y);
       }
     }
     if (it == 0) {
