@@ -70,21 +70,29 @@ def _source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def step_bytes(cfg: workloads.Config, temps: torch.Tensor) -> dict:
+def step_bytes(cfg: workloads.Config, temps: torch.Tensor, accept_len=None) -> dict:
     """Bytes of logits one step must read.
 
     formula: B (2 gamma + 1) V sizeof + B V sizeof (every row once, plus one
     residual row per sequence).  algorithmic: the rows the method needs --
-    greedy (T = 0) sequences need only their gamma + 1 target rows and no
-    draw; sampled sequences need all 2 gamma + 1 rows plus one row for the
-    draw.  The algorithmic figure is the one used for the roofline."""
+    a greedy (T = 0) sequence needs its gamma + 1 target rows and no draw; a
+    sampled sequence needs all 2 gamma + 1 rows once, and then the rows of its
+    draw again: two (target and draft row j) for a residual draw at j < gamma,
+    one (target row gamma) for the bonus draw.  The draw rows follow from the
+    step's accept lengths when they are given (otherwise one row is assumed).
+    The algorithmic figure is the one used for the roofline."""
     es = 2 if cfg.dtype == "bf16" else 4
     B, g, V = cfg.B, cfg.gamma, cfg.V
     formula = B * (2 * g + 1) * V * es + B * V * es
     t = temps.cpu().numpy()
-    greedy = int(np.sum(t == 0.0))
-    sampled = B - greedy
-    algo = (greedy * (g + 1) + sampled * (2 * g + 2)) * V * es
+    greedy = t == 0.0
+    rows = np.where(greedy, g + 1, 2 * g + 1).astype(np.int64)
+    if accept_len is None or cfg.multidraft:
+        draw = np.where(greedy, 0, 1)
+    else:
+        a = accept_len.cpu().numpy()
+        draw = np.where(greedy | (a < 0), 0, np.where(a < g, 2, 1))
+    algo = int(np.sum(rows + draw)) * V * es
     return {"formula": formula, "algorithmic": algo}
 
 
@@ -262,7 +270,6 @@ def run_ours(args, cfg):
     K, W = args.steps, args.warmup
     R = ring_size(cfg, K + W)
     sets = [workloads.make_step(cfg, s + 100000 * rank, device=dev) for s in range(R)]
-    bytes_info = step_bytes(cfg, sets[0].temps)
     dt = sv.BF16 if cfg.dtype == "bf16" else sv.F32
     B, g, V = cfg.B, cfg.gamma, cfg.V
     if cfg.multidraft:
@@ -328,6 +335,11 @@ def run_ours(args, cfg):
     acc_all = torch.cat([o[0] for o in outs]).float()
     valid = acc_all >= 0
     mean_len = float(acc_all[valid].mean()) if valid.any() else float("nan")
+
+    # algorithmic bytes per step, averaged over the ring's inputs and results
+    per = [step_bytes(cfg, sets[r].temps, outs[r][0]) for r in range(R)]
+    bytes_info = {"formula": per[0]["formula"],
+                  "algorithmic": int(round(sum(x["algorithmic"] for x in per) / R))}
 
     rows_total = _sum_over_ranks(cfg.rows_per_step * K, world, dev)
     value = rows_total / (ms_max / 1e3)
