@@ -48,8 +48,8 @@ __device__ __forceinline__ double step_weight(double w, double num, double den) 
 template <bool kBf16>
 __global__ void __launch_bounds__(kMdThreads) md_gbv_kernel(MdParams p) {
   constexpr size_t es = kBf16 ? 2 : 4;
-  __shared__ float s_mt[kMaxRowsPerSeq];  // fl32(row max / T)
-  __shared__ float s_is[kMaxRowsPerSeq];  // 1 / row sum
+  __shared__ float s_mt[kMaxRowsPerSeq];  // raw row maximum m
+  __shared__ float s_is[kMaxRowsPerSeq];  // 1 / s, s = sum_v 2^{(z_v - m) c}
   __shared__ int s_arg[kMaxRowsPerSeq];
   __shared__ int s_x[SV_MAX_DRAFTS * SV_MAX_GAMMA];
   __shared__ int s_H[SV_MAX_DRAFTS];
@@ -82,9 +82,9 @@ __global__ void __launch_bounds__(kMdThreads) md_gbv_kernel(MdParams p) {
     if (needed) {
       bool rv = !a.bad && isfinite(a.m);
       if (!greedy) {
-        s_mt[r] = __fdiv_rn(a.m, T);
+        s_mt[r] = a.m;
         s_is[r] = 1.0f / a.s;
-        rv = rv && isfinite(s_mt[r]);
+        rv = rv && isfinite(__fdiv_rn(a.m, T));
       }
       ok = ok && rv;
     }
@@ -122,15 +122,16 @@ __global__ void __launch_bounds__(kMdThreads) md_gbv_kernel(MdParams p) {
     return;
   }
 
-  // P_r(v) and Q_r(v) with the fp32 scaling of the CPU definition and an
-  // accurate exponential: p = exp(fl32(fl32(z/T) - fl32(max/T))) / S.
+  // P_r(v) and Q_r(v): p = 2^{(z - m) c} / s with c = log2(e) / T, the same
+  // MUFU exponential that built the row sums s (so each law sums to 1 to
+  // within the exponential's 2^-22 relative error), one subtraction, one
+  // multiply, one ex2 and one multiply per value.
+  const float cc = __fdiv_rn(kLog2e, T);
   auto prob_t = [&](int r, int v) -> float {
-    const float d = __fsub_rn(__fdiv_rn(logit_at<kBf16>(tgt + r * rowb, v), T), s_mt[r]);
-    return expf(d) * s_is[r];
+    return ex2_approx((logit_at<kBf16>(tgt + r * rowb, v) - s_mt[r]) * cc) * s_is[r];
   };
   auto prob_d = [&](int r, int v) -> float {
-    const float d = __fsub_rn(__fdiv_rn(logit_at<kBf16>(drf + r * rowb, v), T), s_mt[L + 1 + r]);
-    return expf(d) * s_is[L + 1 + r];
+    return ex2_approx((logit_at<kBf16>(drf + r * rowb, v) - s_mt[L + 1 + r]) * cc) * s_is[L + 1 + r];
   };
 
   // R <- P_0
