@@ -49,6 +49,38 @@ __device__ __forceinline__ uint4 keyed_block(uint64_t seed, uint32_t step, uint3
                        static_cast<uint32_t>(seed), static_cast<uint32_t>(seed >> 32));
 }
 
+// The same stream with the key schedule and the fixed counter words worked
+// out once, for many blocks that differ only in c0 (one draw race).
+struct PhiloxStream {
+  uint32_t k0[10], k1[10];  // round keys
+  uint32_t c1, c2, c3;      // counter words 1..3
+  __device__ __forceinline__ PhiloxStream(uint64_t seed, uint32_t step, uint32_t tag, uint32_t b,
+                                          uint32_t k, uint32_t pos) {
+    uint32_t a = static_cast<uint32_t>(seed), d = static_cast<uint32_t>(seed >> 32);
+#pragma unroll
+    for (int r = 0; r < 10; ++r) {
+      k0[r] = a;
+      k1[r] = d;
+      a += 0x9E3779B9u;
+      d += 0xBB67AE85u;
+    }
+    c1 = b;
+    c2 = step;
+    c3 = (tag << 24) | (k << 12) | pos;
+  }
+  __device__ __forceinline__ uint4 block(uint32_t c0) const {
+    uint4 c = make_uint4(c0, c1, c2, c3);
+#pragma unroll
+    for (int r = 0; r < 10; ++r) {
+      const uint64_t p0 = static_cast<uint64_t>(c.x) * 0xD2511F53u;
+      const uint64_t p1 = static_cast<uint64_t>(c.z) * 0xCD9E8D57u;
+      c = make_uint4(static_cast<uint32_t>(p1 >> 32) ^ c.y ^ k0[r], static_cast<uint32_t>(p1),
+                     static_cast<uint32_t>(p0 >> 32) ^ c.w ^ k1[r], static_cast<uint32_t>(p0));
+    }
+    return c;
+  }
+};
+
 __device__ __forceinline__ uint32_t word_of(const uint4& r, int w) {
   return w == 0 ? r.x : (w == 1 ? r.y : (w == 2 ? r.z : r.w));
 }

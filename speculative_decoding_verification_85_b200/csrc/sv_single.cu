@@ -529,6 +529,7 @@ __device__ __forceinline__ void race_chunk(const SingleParams& f, const SeqInfo&
   const bool tvec = (reinterpret_cast<uintptr_t>(trow) % kVecAlign) == 0;
   const bool dvec = (reinterpret_cast<uintptr_t>(drow) % kVecAlign) == 0;
   const float c = si.c, zmp = si.zmp, zmq = si.zmq, lsp = si.lsp, lsq = si.lsq;
+  const PhiloxStream ps(p.seed, p.step, kTagGumbel, b, 0, si.j);
   const int steps = (g1 - g0 + 2 * kDrawThreads - 1) / (2 * kDrawThreads);  // uniform
   for (int it = 0; it < steps; ++it) {
     const int g = g0 + it * 2 * kDrawThreads + static_cast<int>(threadIdx.x);
@@ -546,8 +547,8 @@ __device__ __forceinline__ void race_chunk(const SingleParams& f, const SeqInfo&
       t1.load(trow, tvec, p.V, gh);
       if (resid) d1.load(drow, dvec, p.V, gh);
     }
-    const uint4 r0 = keyed_block(p.seed, p.step, kTagGumbel, b, 0, si.j, g);
-    const uint4 r1 = keyed_block(p.seed, p.step, kTagGumbel, b, 0, si.j, gh);
+    const uint4 r0 = ps.block(g);
+    const uint4 r1 = ps.block(gh);
     // p_v = 2^{(z_v - zmp) c - lsp}, q_v likewise: the target and draft value
     // of an entry travel as one packed pair
     float w0[4], w1[4];
