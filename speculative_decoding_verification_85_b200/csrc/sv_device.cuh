@@ -118,14 +118,6 @@ __device__ __forceinline__ float max_nan(float a, float b) {
   return d;
 }
 
-// Arrival ticket with release semantics (orders this thread's earlier
-// stores before the increment), and the acquire fence a last arriver takes
-// before reading what the others published.
-__device__ __forceinline__ unsigned ticket_release(unsigned* p) {
-  unsigned old;
-  asm volatile("atom.add.release.gpu.global.u32 %0, [%1], 1;" : "=r"(old) : "l"(p) : "memory");
-  return old;
-}
 // Arrival ticket with acquire-release semantics: releases this thread's
 // earlier stores and, for the last arriver, acquires everything the earlier
 // arrivers released (a CTA barrier then extends that to the whole CTA).
@@ -133,9 +125,6 @@ __device__ __forceinline__ unsigned ticket_acq_rel(unsigned* p) {
   unsigned old;
   asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], 1;" : "=r"(old) : "l"(p) : "memory");
   return old;
-}
-__device__ __forceinline__ void fence_acquire() {
-  asm volatile("fence.acq_rel.gpu;" ::: "memory");
 }
 // 16-byte load of data read once (no L1 allocation).
 __device__ __forceinline__ uint4 ld_stream(const uint4* p) {
@@ -272,67 +261,6 @@ __device__ __forceinline__ double block_sum(double v, double* red) {
   }
   block_sync<kThreads>();
   return red[32];
-}
-
-}  // namespace sv
-
-namespace sv {
-
-// ---- shared-memory mbarrier and 1-D bulk copy (TMA engine), sm_90+ PTX ----
-__device__ __forceinline__ uint32_t smem_addr(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-__device__ __forceinline__ void mbar_init(uint64_t* bar, unsigned count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
-}
-__device__ __forceinline__ void mbar_fence_init() {
-  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-}
-__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes)
-               : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
-}
-// Non-blocking probe of the barrier's phase `parity`.
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_addr(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-// Probe of phase `parity` that may suspend the thread for up to about
-// `ns` nanoseconds while the phase is incomplete (fewer polling instructions).
-__device__ __forceinline__ bool mbar_try_wait_for(uint64_t* bar, uint32_t parity, uint32_t ns) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_addr(bar)), "r"(parity), "r"(ns)
-      : "memory");
-  return ok != 0;
-}
-// Order this thread's (and, after a barrier, the block's) earlier generic
-// shared-memory accesses before later async-proxy (bulk copy) accesses.
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-// Bulk global->shared copy of `bytes` (multiple of 16, both addresses 16-byte
-// aligned) completing on `bar`.  No cluster multicast.
-__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-          smem_addr(dst)),
-      "l"(src), "r"(bytes), "r"(smem_addr(bar))
-      : "memory");
 }
 
 }  // namespace sv

@@ -254,51 +254,6 @@ __device__ __forceinline__ bool pass1_chunk(const Pass1Params& p, int b, int r, 
   return publish_partial<kP1Threads>(p, b, r, chunk, a);
 }
 
-// The 16-byte-aligned body of chunk `chunk` of a row: vectors [k0, k1)
-// starting `head` elements into the row.
-template <bool kBf16>
-struct ChunkSpan {
-  int head, nvec, tail0, k0, k1;
-  __device__ __forceinline__ ChunkSpan(const char* rp, int V, int chunk, int nc) {
-    constexpr int es = kBf16 ? 2 : 4;
-    constexpr int kN = VecLoad<kBf16>::kN;
-    const uintptr_t addr = reinterpret_cast<uintptr_t>(rp);
-    head = static_cast<int>(((16u - (addr & 15u)) & 15u) / es);
-    if (head > V) head = V;
-    nvec = (V - head) / kN;
-    tail0 = head + nvec * kN;
-    const int cv = (nvec + nc - 1) / nc;
-    k0 = min(nvec, chunk * cv);
-    k1 = min(nvec, k0 + cv);
-  }
-  __device__ __forceinline__ const void* body(const char* rp) const {
-    return rp + static_cast<size_t>(head) * (kBf16 ? 2 : 4) + static_cast<size_t>(k0) * 16;
-  }
-  __device__ __forceinline__ uint32_t bytes() const { return static_cast<uint32_t>(k1 - k0) * 16u; }
-};
-
-// Same reduction as scan_chunk, with the chunk body already staged in shared
-// memory (`sm`, k1 - k0 vectors) and the head/tail scalars read from global.
-template <bool kBf16, int kMode, int kThreads>
-__device__ __forceinline__ void scan_staged(RowAcc& a, const char* rp, int V, int chunk, int nc,
-                                            const ChunkSpan<kBf16>& sp, const uint4* sm, float c) {
-  constexpr int kN = VecLoad<kBf16>::kN;
-  const int tid = threadIdx.x;
-  if (chunk == 0)
-    for (int v = tid; v < sp.head; v += kThreads) acc_scalar<kMode>(a, logit_at<kBf16>(rp, v), v, c);
-  const int n = sp.k1 - sp.k0;
-  const int base = sp.head + sp.k0 * kN;
-#pragma unroll 4
-  for (int k = tid; k < n; k += kThreads) {
-    float z[kN];
-    VecLoad<kBf16>::decode(sm[k], z);
-    acc_vector<kMode>(a, z, base + k * kN, c);
-  }
-  if (chunk == nc - 1)
-    for (int v = sp.tail0 + tid; v < V; v += kThreads)
-      acc_scalar<kMode>(a, logit_at<kBf16>(rp, v), v, c);
-}
-
 // Combine the nc chunk partials of every row of sequence b into rows[].
 // Called by all threads of the last-arriving CTA.
 template <int kThreads>
