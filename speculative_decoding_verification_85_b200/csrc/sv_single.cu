@@ -770,10 +770,12 @@ int launch_single(const void* target, const void* draft, const int32_t* tokens,
   p1.out_lq = out_lq;
   // Row segments: whole tiles, about kRowWaves waves of CTAs over the GPU but
   // at most kMaxSegTiles tiles per CTA; balanced so segments differ by at
-  // most one tile.
+  // most one tile.  Long segments spread each CTA's fixed cost (launch, block
+  // reduce, ticket) over more streaming; about three waves keep the last one
+  // mostly full.
   const bool bf16 = dtype == SV_BF16;
   {
-    constexpr int kRowWaves = 4, kMaxSegTiles = 8;
+    constexpr int kRowWaves = 3, kMaxSegTiles = 10;
     const int tiles = body_tiles(V, dtype);
     const long long pairs = static_cast<long long>(B) * (gamma + 1);
     const long long slots = static_cast<long long>(sm_count()) * row_ctas_per_sm(bf16);
