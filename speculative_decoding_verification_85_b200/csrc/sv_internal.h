@@ -14,8 +14,12 @@ constexpr int kP2Threads = 256;   // pass-2 CTA size
 constexpr int kMdThreads = 1024;  // multi-draft sequential kernel CTA size
 constexpr int kMaxRowsPerSeq = 2 * SV_MAX_GAMMA + 1;
 
-// Pass-1 partial of one (row, chunk): raw max, sum of 2^{(z - max) c}, first
-// argmax index (greedy rows), NaN seen.  16 bytes, stored as one vector.
+// Partial of one (row, chunk): raw max, scaled sum, index slot, NaN seen; 16
+// bytes, stored as one vector.  The multi-draft chunk pass keeps
+// s = sum 2^{(z - max) c} and the first argmax index (greedy rows); the
+// single-draft row kernel keeps S = sum 2^{z c - R} against an integer
+// reference R, carried as float bits in the index slot (softmax rows), or
+// the first argmax index (greedy rows).
 struct alignas(16) RowPartial {
   float m;
   float s;
@@ -80,12 +84,9 @@ struct MdParams {
 // fixed size at offset 0 (one slot per sequence, up to SV_MAX_BATCH), so their
 // position does not depend on the shape: every call leaves them at zero and a
 // later call of any shape finds zeroed counters.
-// Header: 256 bytes of control words, then the per-sequence row-kernel and
-// draw-kernel arrival counters.  Control word kHeaderError collects
-// device-side error bits; it is sticky (never cleared by a call).
+// Header: 256 reserved bytes (zero, unused by the current kernels), then the
+// per-sequence row-kernel and draw-kernel arrival counters.
 constexpr size_t kHeaderCtl = 256;
-constexpr int kHeaderError = 2;
-constexpr unsigned kErrStageTimeout = 1u;  // a bulk-copy wait gave up
 constexpr size_t kHeaderBytes = kHeaderCtl + 2 * static_cast<size_t>(SV_MAX_BATCH) * sizeof(unsigned);
 
 struct Layout {
@@ -95,7 +96,7 @@ struct Layout {
 
 Layout layout_single(int B, int gamma, int V, int dtype);
 int draw_chunks(int V, int dtype);   // bound on draw CTAs per sequence (sv_single.cu)
-int row_segments(int V, int dtype);  // row CTAs per row (sv_single.cu)
+int row_segments(int V, int dtype);  // bound on row segments per row (sv_single.cu)
 Layout layout_multi(int B, int K, int L, int V, int dtype);
 
 // Host helpers (sv_api.cu).

@@ -313,6 +313,8 @@ int launch_multi(const void* target, const void* draft, const int32_t* tokens,
   p1.ticket = reinterpret_cast<unsigned*>(ws + lay.ticket1);
   p1.rowstat = reinterpret_cast<RowPartial*>(ws + lay.rowstat);
   const long long grid1 = static_cast<long long>(B) * p1.rps * lay.nc;
+  if (grid1 > INT_MAX)
+    return set_error(SV_ERR_INVALID_ARG, "B x (2L+1) x V too large for one launch (%lld CTAs)", grid1);
   if (dtype == SV_BF16)
     pass1_multi_kernel<true><<<static_cast<unsigned>(grid1), kP1Threads, 0, stream>>>(p1);
   else

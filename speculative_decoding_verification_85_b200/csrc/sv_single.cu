@@ -17,8 +17,8 @@
 // per vocabulary entry; the CTA that completes a sequence combines.
 // Neither kernel waits on another CTA: all ordering is by arrival tickets and
 // by the launch dependency.
+#include <atomic>
 #include <climits>
-#include <mutex>
 
 #include "sv_device.cuh"
 #include "sv_internal.h"
@@ -675,52 +675,56 @@ int draw_chunks(int V, int dtype) {  // upper bound on draw CTAs per sequence
 }
 
 namespace {
+// A host query whose answer is fixed per device (SM count, occupancy), asked
+// once per device and kept.  The slots are atomics: threads that call at the
+// same time may both ask, and store the same value.
+template <typename Query>
+int per_device(std::atomic<int> (&slots)[64], int fallback, Query query) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return fallback;
+  int v = slots[dev].load(std::memory_order_relaxed);
+  if (v == 0) {
+    v = query(dev);
+    if (v <= 0) v = fallback;
+    slots[dev].store(v, std::memory_order_relaxed);
+  }
+  return v;
+}
+
 int sm_count() {
-  static int cached[64];
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-  if (cached[dev] == 0) {
+  static std::atomic<int> slots[64];
+  return per_device(slots, 148, [](int dev) {
     int n = 0;
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    cached[dev] = n > 0 ? n : 148;
-  }
-  return cached[dev];
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+      (void)cudaGetLastError();
+      return 0;
+    }
+    return n;
+  });
 }
 
-// Resident row-kernel CTAs per SM (occupancy query, cached per device).
+template <typename Kernel>
+int occupancy(Kernel kernel, int threads) {
+  int n = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, threads, 0) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return 0;
+  }
+  return n;
+}
+
+// Resident row-kernel CTAs per SM.
 int row_ctas_per_sm(bool bf16) {
-  static int cached[64][2];
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 3;
-  int& slot = cached[dev][bf16 ? 1 : 0];
-  if (slot == 0) {
-    int n = 0;
-    const cudaError_t e =
-        bf16 ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, rows_kernel<true>, kRowThreads, 0)
-             : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, rows_kernel<false>, kRowThreads, 0);
-    if (e != cudaSuccess) (void)cudaGetLastError();
-    slot = (e == cudaSuccess && n > 0) ? n : 3;
-  }
-  return slot;
+  static std::atomic<int> slots[2][64];
+  return bf16 ? per_device(slots[1], 3, [](int) { return occupancy(rows_kernel<true>, kRowThreads); })
+              : per_device(slots[0], 3, [](int) { return occupancy(rows_kernel<false>, kRowThreads); });
 }
 
-// Resident draw-kernel CTAs per SM (occupancy query, cached per device).
+// Resident draw-kernel CTAs per SM.
 int draw_ctas_per_sm(bool bf16) {
-  static std::mutex mu;
-  static int cached[64][2];
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 4;
-  std::lock_guard<std::mutex> lk(mu);
-  int& slot = cached[dev][bf16 ? 1 : 0];
-  if (slot == 0) {
-    int n = 0;
-    const cudaError_t e =
-        bf16 ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, draw_kernel<true>, kDrawThreads, 0)
-             : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, draw_kernel<false>, kDrawThreads, 0);
-    if (e != cudaSuccess) (void)cudaGetLastError();
-    slot = (e == cudaSuccess && n > 0) ? n : 4;
-  }
-  return slot;
+  static std::atomic<int> slots[2][64];
+  return bf16 ? per_device(slots[1], 4, [](int) { return occupancy(draw_kernel<true>, kDrawThreads); })
+              : per_device(slots[0], 4, [](int) { return occupancy(draw_kernel<false>, kDrawThreads); });
 }
 
 template <typename K>
@@ -809,6 +813,9 @@ int launch_single(const void* target, const void* draft, const int32_t* tokens,
     f.nc2 = static_cast<int>((nb + cb - 1) / cb);
   }
 
+  if (static_cast<long long>(B) * f.nc2 > INT_MAX)
+    return set_error(SV_ERR_INVALID_ARG, "B x V too large for one launch (draw grid %lld CTAs)",
+                     static_cast<long long>(B) * f.nc2);
   const dim3 grid1(static_cast<unsigned>(B * (gamma + 1)), static_cast<unsigned>(f.nseg));
   cudaError_t e = bf16 ? launch_pdl(rows_kernel<true>, grid1, kRowThreads, stream, f)
                        : launch_pdl(rows_kernel<false>, grid1, kRowThreads, stream, f);
