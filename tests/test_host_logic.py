@@ -126,7 +126,7 @@ def _cfg(**kw):
 def test_step_bytes_closed_forms():
     cfg = _cfg()
     es, B, g, V = 2, 4, 3, 1000
-    # the spec formula does not depend on temperatures or outcomes
+    # the headline byte formula does not depend on temperatures or outcomes
     f = bench.step_bytes(cfg, torch.zeros(B))["formula"]
     assert f == B * (2 * g + 1) * V * es + B * V * es
     # all greedy: gamma + 1 target rows each, no draw
