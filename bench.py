@@ -243,8 +243,8 @@ def run_reference(args, cfg):
     except AttributeError:
         cores = os.cpu_count() or 1
     threads = max(1, min(cores, cfg.B))
-    # warm-up steps are untimed
-    time_oracle(cfg, max(0, min(args.warmup, 1)), threads, 1e9)
+    # W untimed warm-up steps, as reported in the line
+    time_oracle(cfg, args.warmup, threads, 1e9)
     value, done, secs = time_oracle(cfg, args.steps, threads, args.ref_budget)
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
