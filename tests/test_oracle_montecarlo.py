@@ -221,3 +221,32 @@ def test_oracle_invariants(B, gamma, V, T, bf16, seed):
         assert np.array_equal(r["tokens"][b, :j], toks[b, :j])
         assert 0 <= r["tokens"][b, j] < V
         assert np.all(r["tokens"][b, j + 1:] == -1)
+
+
+@settings(max_examples=40, deadline=None)
+@given(B=st.integers(1, 3), K=st.sampled_from([1, 2, 5, 32]), L=st.sampled_from([1, 2, 7, 64]),
+       V=st.sampled_from([1, 2, 5, 17]), T=st.sampled_from([0.0, 0.1, 0.7, 1.0]),
+       bf16=st.booleans(), seed=st.integers(0, 2**31 - 1))
+def test_multidraft_oracle_invariants(B, K, L, V, T, bf16, seed):
+    """SpecTr-GBV, Algorithm 1, up to the largest K and L the interface takes:
+    0 <= tau <= L; with tau > 0 the output starts with the first tau tokens
+    of the reported draft; the emitted token is in range; padding is -1."""
+    rng = np.random.default_rng(seed)
+    tg = rng.normal(0, 2, (B, L + 1, V)).astype(np.float32)
+    dr = (tg[:, :L] + rng.normal(0, 1, (B, L, V))).astype(np.float32)
+    if bf16:
+        tg, dr = f32_to_bf16_bits(tg), f32_to_bf16_bits(dr)
+    # drafts share prefixes often (small V), which exercises the skip rules
+    toks = rng.integers(0, V, (B, K, L)).astype(np.int32)
+    r = oracle.verify_multidraft(tg, dr, toks, np.full(B, T, np.float32), seed=seed,
+                                 step=seed % 1000)
+    for b in range(B):
+        tau, a = int(r["accept_len"][b]), int(r["draft_index"][b])
+        assert 0 <= tau <= L
+        if tau > 0:
+            assert 0 <= a < K
+            assert np.array_equal(r["tokens"][b, :tau], toks[b, a, :tau])
+        else:
+            assert a == -1  # no draft's token was kept
+        assert 0 <= r["tokens"][b, tau] < V
+        assert np.all(r["tokens"][b, tau + 1:] == -1)
