@@ -88,6 +88,10 @@ def lib():
                                                 C.c_int, u64, u64, i64, i64, vp, vp, vp, vp,
                                                 C.POINTER(Rng)]
             L.svo_verify_multidraft.restype = C.c_int
+            L.svo_verify_multidraft_rows.argtypes = [vp, vp, vp, vp, i64, C.c_int, C.c_int, i64,
+                                                     C.c_int, C.c_int, u64, u64, i64, i64, vp, vp,
+                                                     vp, vp, C.POINTER(Rng)]
+            L.svo_verify_multidraft_rows.restype = C.c_int
             _lib = L
     return _lib
 
@@ -224,16 +228,21 @@ def verify(target, draft, tokens, temps, *, seed=0, step=0, rng=None, threads=1,
 
 
 def verify_multidraft(target, draft, tokens, temps, *, seed=0, step=0, rng=None, threads=1):
-    """Multi-draft verification.  target [B, L+1, V], draft [B, L, V], tokens
+    """Multi-draft verification.  target [B, L+1, V] and draft [B, L, V] shared
+    by the K drafts, or per-draft rows target [B, K, L+1, V] and draft
+    [B, K, L, V] (row (k, i) conditioned on draft k's own prefix); tokens
     [B, K, L].  Returns accept_len [B], tokens [B, L+1], draft_index [B], tie [B]."""
     target = np.ascontiguousarray(target)
     draft = np.ascontiguousarray(draft)
     tokens = np.ascontiguousarray(tokens, dtype=np.int32)
     temps = np.ascontiguousarray(temps, dtype=np.float32)
-    B, l1, V = target.shape
+    per_draft = target.ndim == 4
+    B, K = tokens.shape[0], tokens.shape[1]
+    l1, V = target.shape[-2], target.shape[-1]
     L_ = l1 - 1
-    K = tokens.shape[1]
-    assert draft.shape == (B, L_, V) and tokens.shape == (B, K, L_) and temps.shape == (B,)
+    lead = (B, K) if per_draft else (B,)
+    assert target.shape == lead + (L_ + 1, V) and draft.shape == lead + (L_, V)
+    assert tokens.shape == (B, K, L_) and temps.shape == (B,)
     dt = _dtype_code(target)
     assert _dtype_code(draft) == dt
     acc = np.empty(B, dtype=np.int32)
@@ -244,11 +253,12 @@ def verify_multidraft(target, draft, tokens, temps, *, seed=0, step=0, rng=None,
     Lb = lib()
 
     def run(r):
-        rc = Lb.svo_verify_multidraft(_ptr(target), _ptr(draft), _ptr(tokens), _ptr(temps), B, K,
-                                      L_, V, dt, seed, step, r[0], r[1], _ptr(acc), _ptr(tok),
-                                      _ptr(didx), _ptr(tie), rng_p)
+        rc = Lb.svo_verify_multidraft_rows(_ptr(target), _ptr(draft), _ptr(tokens), _ptr(temps),
+                                           B, K, L_, V, dt, int(per_draft), seed, step, r[0],
+                                           r[1], _ptr(acc), _ptr(tok), _ptr(didx), _ptr(tie),
+                                           rng_p)
         if rc != 0:
-            raise ValueError("svo_verify_multidraft rejected its arguments")
+            raise ValueError("svo_verify_multidraft_rows rejected its arguments")
 
     if rng is not None or threads <= 1:
         run((0, B))

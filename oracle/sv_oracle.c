@@ -383,13 +383,19 @@ static double step_weight(double w, double num, double den) {
 }
 
 static void seq_multi(const char* target, const char* draft, const int32_t* tokens,
-                      const float* temps, int K, int L, int64_t V, int dtype, int64_t b,
-                      const svo_rng* rng, int32_t* out_accept_len, int32_t* out_tokens,
-                      int32_t* out_draft_index, uint8_t* out_tie) {
+                      const float* temps, int K, int L, int64_t V, int dtype, int per_draft,
+                      int64_t b, const svo_rng* rng, int32_t* out_accept_len,
+                      int32_t* out_tokens, int32_t* out_draft_index, uint8_t* out_tie) {
   const size_t es = elem_size(dtype);
   const size_t rowb = (size_t)V * es;
-  const char* trow0 = target + (size_t)b * (size_t)(L + 1) * rowb;
-  const char* drow0 = draft + (size_t)b * (size_t)L * rowb;
+  /* Row sets: one shared by every draft, or one per draft (per_draft), in
+   * which case row (k, i) is conditioned on draft k's own prefix. */
+  const size_t nset = per_draft ? (size_t)K : 1u;
+  const char* trow0 = target + (size_t)b * nset * (size_t)(L + 1) * rowb;
+  const char* drow0 = draft + (size_t)b * nset * (size_t)L * rowb;
+#define SET(k) ((size_t)(per_draft ? (k) : 0))
+#define TROW(k, i) (trow0 + (SET(k) * (size_t)(L + 1) + (size_t)(i)) * rowb)
+#define DROW(k, i) (drow0 + (SET(k) * (size_t)L + (size_t)(i)) * rowb)
   const int32_t* xs = tokens + (size_t)b * (size_t)K * (size_t)L;
   int32_t* tok = out_tokens + (size_t)b * (size_t)(L + 1);
   uint8_t tie = 0;
@@ -408,47 +414,54 @@ static void seq_multi(const char* target, const char* draft, const int32_t* toke
     /* Reading (greedy): the target is the argmax at every position; the
      * accepted block is the longest draft prefix that matches it (first
      * draft on ties), and the correction is the argmax at tau. */
-    int64_t g[MAX_STEPS + 1];
-    for (int i = 0; i <= L; ++i) {
-      g[i] = svo_row_argmax(trow0 + (size_t)i * rowb, V, dtype);
-      if (g[i] < 0) return;
-    }
+    int64_t g[32][MAX_STEPS + 1]; /* argmax of row (set, i) */
+    for (size_t k = 0; k < nset; ++k)
+      for (int i = 0; i <= L; ++i) {
+        g[k][i] = svo_row_argmax(TROW(k, i), V, dtype);
+        if (g[k][i] < 0) return;
+      }
     int tau = 0, a = -1;
     for (int k = 0; k < K; ++k) {
       int n = 0;
-      while (n < L && (int64_t)xs[(size_t)k * L + n] == g[n]) ++n;
+      while (n < L && (int64_t)xs[(size_t)k * L + n] == g[SET(k)][n]) ++n;
       if (n > tau) {
         tau = n;
         a = k;
       }
     }
     for (int i = 0; i < tau; ++i) tok[i] = xs[(size_t)a * L + i];
-    tok[tau] = (int32_t)g[tau];
+    /* the correction is the argmax at tau of the accepted draft's rows (every
+     * draft's row 0 when nothing was accepted: they share the empty prefix) */
+    tok[tau] = (int32_t)g[SET(a < 0 ? 0 : a)][tau];
     out_accept_len[b] = tau;
     if (out_draft_index) out_draft_index[b] = a;
     return;
   }
 
-  /* Probability vectors P_0..P_L (target) and Q_0..Q_{L-1} (draft). */
-  double* P = (double*)malloc((size_t)(L + 1) * (size_t)V * sizeof(double));
-  double* Q = (double*)malloc((size_t)L * (size_t)V * sizeof(double));
+  /* Probability vectors P_0..P_L (target) and Q_0..Q_{L-1} (draft) of every
+   * row set. */
+  double* P = (double*)malloc(nset * (size_t)(L + 1) * (size_t)V * sizeof(double));
+  double* Q = (double*)malloc(nset * (size_t)L * (size_t)V * sizeof(double));
   double* R = (double*)malloc((size_t)V * sizeof(double));
   double* lw = (double*)malloc((size_t)V * sizeof(double));
   unsigned char* inH = (unsigned char*)calloc((size_t)V, 1);
   int ok = P && Q && R && lw && inH;
-  for (int i = 0; ok && i <= L; ++i)
-    ok = svo_row_logprobs(trow0 + (size_t)i * rowb, V, dtype, T, P + (size_t)i * V) == 0;
-  for (int i = 0; ok && i < L; ++i)
-    ok = svo_row_logprobs(drow0 + (size_t)i * rowb, V, dtype, T, Q + (size_t)i * V) == 0;
+  for (size_t k = 0; ok && k < nset; ++k) {
+    for (int i = 0; ok && i <= L; ++i)
+      ok = svo_row_logprobs(TROW(k, i), V, dtype, T, P + (k * (size_t)(L + 1) + i) * V) == 0;
+    for (int i = 0; ok && i < L; ++i)
+      ok = svo_row_logprobs(DROW(k, i), V, dtype, T, Q + (k * (size_t)L + i) * V) == 0;
+  }
   if (!ok) goto done;
-  for (size_t n = 0; n < (size_t)(L + 1) * (size_t)V; ++n) P[n] = exp(P[n]);
-  for (size_t n = 0; n < (size_t)L * (size_t)V; ++n) Q[n] = exp(Q[n]);
-#define PROW(i) (P + (size_t)(i) * (size_t)V)
-#define QROW(i) (Q + (size_t)(i) * (size_t)V)
+  for (size_t n = 0; n < nset * (size_t)(L + 1) * (size_t)V; ++n) P[n] = exp(P[n]);
+  for (size_t n = 0; n < nset * (size_t)L * (size_t)V; ++n) Q[n] = exp(Q[n]);
+  /* P_i and Q_i as seen by draft k (its own rows, or the shared ones) */
+#define PROW(k, i) (P + (SET(k) * (size_t)(L + 1) + (size_t)(i)) * (size_t)V)
+#define QROW(k, i) (Q + (SET(k) * (size_t)L + (size_t)(i)) * (size_t)V)
 
   int tau = 0, a = -1;
   double qH = 0.0; /* Q_tau mass of H */
-  memcpy(R, PROW(0), (size_t)V * sizeof(double));
+  memcpy(R, PROW(0, 0), (size_t)V * sizeof(double)); /* every draft shares the empty prefix */
 
   for (int k = 0; k < K; ++k) {
     if (tau == L) break;
@@ -457,19 +470,19 @@ static void seq_multi(const char* target, const char* draft, const int32_t* toke
     if (inH[x[tau]]) continue; /* rejected sub-block seen before */
 
     const double keep = 1.0 - qH;
-    const double qfirst = keep > 0.0 ? QROW(tau)[x[tau]] / keep : 0.0;
+    const double qfirst = keep > 0.0 ? QROW(k, tau)[x[tau]] / keep : 0.0;
     double w = 1.0, wbest = 1.0;
     int best = tau;
     for (int i = tau; i < L; ++i) {
       if (i == tau)
         w = step_weight(w, R[x[i]], qfirst);
       else
-        w = step_weight(w, PROW(i)[x[i]], QROW(i)[x[i]]);
+        w = step_weight(w, PROW(k, i)[x[i]], QROW(k, i)[x[i]]);
       double h;
       if (i < L - 1) {
         double A = 0.0;
-        const double* pn = PROW(i + 1);
-        const double* qn = QROW(i + 1);
+        const double* pn = PROW(k, i + 1);
+        const double* qn = QROW(k, i + 1);
         for (int64_t v = 0; v < V; ++v) {
           const double t = w * pn[v] - qn[v];
           if (t > 0.0) A += t;
@@ -495,19 +508,19 @@ static void seq_multi(const char* target, const char* draft, const int32_t* toke
       if (tau < L) {
         double Z = 0.0;
         for (int64_t v = 0; v < V; ++v) {
-          const double t = wbest * PROW(tau)[v] - QROW(tau)[v];
+          const double t = wbest * PROW(k, tau)[v] - QROW(k, tau)[v];
           R[v] = t > 0.0 ? t : 0.0;
           Z += R[v];
         }
         if (Z > 0.0)
           for (int64_t v = 0; v < V; ++v) R[v] /= Z;
         else
-          memcpy(R, PROW(tau), (size_t)V * sizeof(double));
+          memcpy(R, PROW(k, tau), (size_t)V * sizeof(double));
       }
     } else {
       double Z = 0.0;
       for (int64_t v = 0; v < V; ++v) {
-        const double qt = (inH[v] || keep <= 0.0) ? 0.0 : QROW(tau)[v] / keep;
+        const double qt = (inH[v] || keep <= 0.0) ? 0.0 : QROW(k, tau)[v] / keep;
         const double t = R[v] - qt;
         lw[v] = t > 0.0 ? t : 0.0;
         Z += lw[v];
@@ -515,14 +528,14 @@ static void seq_multi(const char* target, const char* draft, const int32_t* toke
       if (Z > 0.0)
         for (int64_t v = 0; v < V; ++v) R[v] = lw[v] / Z;
       inH[x[tau]] = 1;
-      qH += QROW(tau)[x[tau]];
+      qH += QROW(k, tau)[x[tau]];
     }
   }
 
   /* [GBV] termination: whole block accepted -> correction from the target
    * (row L); otherwise from the residual law R at tau. */
   if (tau == L) {
-    for (int64_t v = 0; v < V; ++v) lw[v] = log(PROW(L)[v]);
+    for (int64_t v = 0; v < V; ++v) lw[v] = log(PROW(a, L)[v]);
   } else {
     for (int64_t v = 0; v < V; ++v) lw[v] = R[v] > 0.0 ? log(R[v]) : -INFINITY;
   }
@@ -539,6 +552,9 @@ static void seq_multi(const char* target, const char* draft, const int32_t* toke
   }
 #undef PROW
 #undef QROW
+#undef TROW
+#undef DROW
+#undef SET
 done:
   free(P);
   free(Q);
@@ -552,6 +568,17 @@ int svo_verify_multidraft(const void* target, const void* draft, const int32_t* 
                           int dtype, uint64_t seed, uint64_t step, int64_t b_begin,
                           int64_t b_end, int32_t* out_accept_len, int32_t* out_tokens,
                           int32_t* out_draft_index, uint8_t* out_tie, const svo_rng* rng) {
+  return svo_verify_multidraft_rows(target, draft, tokens, temps, B, K, L, V, dtype, 0, seed,
+                                    step, b_begin, b_end, out_accept_len, out_tokens,
+                                    out_draft_index, out_tie, rng);
+}
+
+int svo_verify_multidraft_rows(const void* target, const void* draft, const int32_t* tokens,
+                               const float* temps, int64_t B, int K, int L, int64_t V,
+                               int dtype, int per_draft, uint64_t seed, uint64_t step,
+                               int64_t b_begin, int64_t b_end, int32_t* out_accept_len,
+                               int32_t* out_tokens, int32_t* out_draft_index,
+                               uint8_t* out_tie, const svo_rng* rng) {
   if (!target || !draft || !tokens || !temps || !out_accept_len || !out_tokens) return -1;
   if (B < 0 || K < 1 || K > 32 || L < 1 || L > MAX_STEPS || V < 1 || V > ((int64_t)1 << 31))
     return -1;
@@ -562,7 +589,7 @@ int svo_verify_multidraft(const void* target, const void* draft, const int32_t* 
   svo_rng def = {&pc, philox_coin, philox_categorical};
   if (!rng) rng = &def;
   for (int64_t b = b_begin; b < b_end; ++b)
-    seq_multi((const char*)target, (const char*)draft, tokens, temps, K, L, V, dtype, b, rng,
-              out_accept_len, out_tokens, out_draft_index, out_tie);
+    seq_multi((const char*)target, (const char*)draft, tokens, temps, K, L, V, dtype,
+              per_draft != 0, b, rng, out_accept_len, out_tokens, out_draft_index, out_tie);
   return 0;
 }

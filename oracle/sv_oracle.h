@@ -118,6 +118,21 @@ int svo_verify_multidraft(const void* target, const void* draft, const int32_t* 
                           int64_t b_end, int32_t* out_accept_len, int32_t* out_tokens,
                           int32_t* out_draft_index, uint8_t* out_tie, const svo_rng* rng);
 
+/* The same verification with a row set per draft when per_draft != 0:
+ * target [B, K, L+1, V] and draft [B, K, L, V], where row (k, i) holds the
+ * target / draft logits after draft k's own prefix x_k[0..i) (the
+ * prefix-conditioned use of the method; rows of drafts that share a prefix
+ * are then equal).  Draft k is weighed with its own rows; the residual law
+ * starts from row (0, 0) (every draft shares the empty prefix) and, after an
+ * advance, comes from the accepted draft's rows.  per_draft == 0 is
+ * svo_verify_multidraft. */
+int svo_verify_multidraft_rows(const void* target, const void* draft, const int32_t* tokens,
+                               const float* temps, int64_t B, int K, int L, int64_t V,
+                               int dtype, int per_draft, uint64_t seed, uint64_t step,
+                               int64_t b_begin, int64_t b_end, int32_t* out_accept_len,
+                               int32_t* out_tokens, int32_t* out_draft_index,
+                               uint8_t* out_tie, const svo_rng* rng);
+
 #ifdef __cplusplus
 }
 #endif

@@ -160,3 +160,73 @@ def product_law(P):
     for m in range(1, P.shape[0]):
         out = np.multiply.outer(out, P[m])
     return out
+
+
+# ---------------------------------------------------- prefix-conditioned model
+def prefix_model(V: int, L: int, seed: int):
+    """A small autoregressive target / draft pair: a logit row for every
+    prefix (target rows for prefixes of length 0..L, draft rows for 0..L-1),
+    the draft a noisy copy of the target."""
+    rng = np.random.default_rng(seed)
+    tctx, dctx = {}, {}
+    for n in range(L + 1):
+        for pre in itertools.product(range(V), repeat=n):
+            tctx[pre] = rng.normal(0.0, 1.5, V).astype(np.float32)
+            if n < L:
+                dctx[pre] = (tctx[pre] + rng.normal(0.0, 1.0, V)).astype(np.float32)
+    return tctx, dctx
+
+
+def per_draft_rows(tctx, dctx, drafts, L):
+    """Per-draft rows for drafts x_k: target row (k, i) = tctx[x_k[:i]],
+    draft row (k, i) = dctx[x_k[:i]]."""
+    tg = np.stack([np.stack([tctx[tuple(x[:i])] for i in range(L + 1)]) for x in drafts])
+    dr = np.stack([np.stack([dctx[tuple(x[:i])] for i in range(L)]) for x in drafts])
+    return tg, dr
+
+
+def multidraft_law_prefix_model(tctx, dctx, V, L, K, T, rows=per_draft_rows):
+    """Exact law of (tau, emitted tokens) with K i.i.d. drafts from the
+    prefix-conditioned draft model, verified with per-draft rows."""
+    q = {pre: np.exp(oracle.row_logprobs(r, T)) for pre, r in dctx.items()}
+    temps = np.array([T], dtype=np.float32)
+    blocks = list(itertools.product(range(V), repeat=L))
+    pblock = [float(np.prod([q[blk[:i]][blk[i]] for i in range(L)])) for blk in blocks]
+    law: dict = {}
+    for combo in itertools.product(range(len(blocks)), repeat=K):
+        wx = float(np.prod([pblock[c] for c in combo]))
+        if wx == 0.0:
+            continue
+        drafts = [blocks[c] for c in combo]
+        tg, dr = rows(tctx, dctx, drafts, L)
+        toks = np.array([drafts], dtype=np.int32)
+
+        def run(rng):
+            r = oracle.verify_multidraft(tg[None], dr[None], toks, temps, rng=rng)
+            t = int(r["accept_len"][0])
+            return t, tuple(int(v) for v in r["tokens"][0, : t + 1])
+
+        for w, key in leaves(run):
+            law[key] = law.get(key, 0.0) + wx * w
+    return law
+
+
+def prefix_target_law(tctx, V, L, T):
+    """Law of the target model over V^(L+1): prod_m P(seq[:m])(seq[m])."""
+    p = {pre: np.exp(oracle.row_logprobs(r, T)) for pre, r in tctx.items()}
+    full = np.zeros((V,) * (L + 1))
+    for seq in itertools.product(range(V), repeat=L + 1):
+        full[seq] = float(np.prod([p[seq[:m]][seq[m]] for m in range(L + 1)]))
+    return full, p
+
+
+def extend_prefix_law(law, p, V, L):
+    """Complete every emitted prefix with target draws from the
+    prefix-conditioned target for the later positions."""
+    full = np.zeros((V,) * (L + 1))
+    for (_, toks), w in law.items():
+        n = len(toks)
+        for rest in itertools.product(range(V), repeat=L + 1 - n):
+            seq = tuple(toks) + rest
+            full[seq] += w * float(np.prod([p[seq[:m]][seq[m]] for m in range(n, L + 1)]))
+    return full

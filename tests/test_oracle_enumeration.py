@@ -15,6 +15,7 @@ import pytest
 import oracle
 from tests.oracle_enum import (Script, extend_to_full, multidraft_law, product_law,
                                row_probs, single_draft_law)
+from tests import oracle_enum
 from workloads import f32_to_bf16_bits
 
 
@@ -142,3 +143,59 @@ def test_multidraft_accept_length_monotone_in_K():
     means = [_mean_len(multidraft_law(tg, dr, K, 1.0)) for K in (1, 2, 3)]
     assert means[0] <= means[1] + 1e-12 <= means[2] + 2e-12
     assert means[2] > means[0]
+
+
+# ------------------------------------------------ per-draft (prefix-conditioned) rows
+PREFIX_CASES = [(2, 1, 2, 1.0), (3, 1, 3, 0.8), (2, 2, 2, 1.0), (3, 2, 2, 0.7), (2, 2, 3, 1.2)]
+
+
+@pytest.mark.parametrize("V,L,K,T", PREFIX_CASES)
+def test_per_draft_rows_law_equals_prefix_conditioned_target(V, L, K, T):
+    """SpecTr-GBV, Algorithm 1 with each draft weighed by the rows of its own
+    prefix: with K i.i.d. drafts from an autoregressive draft model, the
+    emitted tokens (completed by the target for later positions) follow the
+    autoregressive target model exactly."""
+    tctx, dctx = oracle_enum.prefix_model(V, L, 3000 + 17 * V + 5 * L + K)
+    law = oracle_enum.multidraft_law_prefix_model(tctx, dctx, V, L, K, T)
+    want, p = oracle_enum.prefix_target_law(tctx, V, L, T)
+    full = oracle_enum.extend_prefix_law(law, p, V, L)
+    assert abs(full.sum() - 1.0) < 1e-12
+    np.testing.assert_allclose(full, want, rtol=0, atol=1e-12)
+
+
+def test_per_draft_enumeration_detects_rows_of_the_wrong_draft():
+    """Planted mistake: every draft weighed with draft 0's rows.  The law
+    drifts away from the target model, so the enumeration above has power."""
+    V, L, K, T = 3, 2, 2, 1.0
+    tctx, dctx = oracle_enum.prefix_model(V, L, 77)
+
+    def first_drafts_rows(tc, dc, drafts, L_):
+        tg, dr = oracle_enum.per_draft_rows(tc, dc, drafts, L_)
+        return np.repeat(tg[:1], len(drafts), axis=0), np.repeat(dr[:1], len(drafts), axis=0)
+
+    law = oracle_enum.multidraft_law_prefix_model(tctx, dctx, V, L, K, T, rows=first_drafts_rows)
+    want, p = oracle_enum.prefix_target_law(tctx, V, L, T)
+    full = oracle_enum.extend_prefix_law(law, p, V, L)
+    assert np.max(np.abs(full - want)) > 1e-4
+
+
+@pytest.mark.parametrize("T", [0.0, 0.4, 1.0])
+@pytest.mark.parametrize("bf16", [False, True])
+def test_per_draft_rows_with_equal_sets_match_shared_rows(T, bf16):
+    """Per-draft rows that are K copies of the shared rows give exactly the
+    shared-row result (same keyed randomness, same arithmetic)."""
+    rng = np.random.default_rng(11)
+    B, K, L, V = 4, 5, 4, 37
+    tg = rng.normal(0, 2, (B, L + 1, V)).astype(np.float32)
+    dr = (tg[:, :L] + rng.normal(0, 0.8, (B, L, V))).astype(np.float32)
+    if bf16:
+        tg, dr = f32_to_bf16_bits(tg), f32_to_bf16_bits(dr)
+    toks = rng.integers(0, V, (B, K, L)).astype(np.int32)
+    toks[:, 1:, :2] = toks[:, :1, :2]  # shared prefixes exercise the skip rules
+    temps = np.full(B, T, np.float32)
+    a = oracle.verify_multidraft(tg, dr, toks, temps, seed=9, step=4)
+    tgk = np.ascontiguousarray(np.repeat(tg[:, None], K, axis=1))
+    drk = np.ascontiguousarray(np.repeat(dr[:, None], K, axis=1))
+    b = oracle.verify_multidraft(tgk, drk, toks, temps, seed=9, step=4)
+    for key in ("accept_len", "tokens", "draft_index", "tie"):
+        assert np.array_equal(a[key], b[key]), key
