@@ -92,6 +92,18 @@ def lib():
                                                      C.c_int, C.c_int, u64, u64, i64, i64, vp, vp,
                                                      vp, vp, C.POINTER(Rng)]
             L.svo_verify_multidraft_rows.restype = C.c_int
+            L.svo_bandit_uniform.argtypes = [u64, u32, u32, u32, u32, C.c_int]
+            L.svo_bandit_uniform.restype = C.c_double
+            L.svo_gamma_sample.argtypes = [C.c_double, u64, u32, u32]
+            L.svo_gamma_sample.restype = C.c_double
+            L.svo_beta_sample.argtypes = [C.c_double, C.c_double, u64, u32, u32]
+            L.svo_beta_sample.restype = C.c_double
+            L.svo_ucb1_select.argtypes = [C.c_int, vp, vp]
+            L.svo_ucb1_select.restype = C.c_int
+            L.svo_thompson_select.argtypes = [C.c_int, vp, vp, u64, u32, vp]
+            L.svo_thompson_select.restype = C.c_int
+            L.svo_thompson_trial.argtypes = [C.c_double, u64, u32, u32]
+            L.svo_thompson_trial.restype = C.c_int
             _lib = L
     return _lib
 
@@ -266,3 +278,65 @@ def verify_multidraft(target, draft, tokens, temps, *, seed=0, step=0, rng=None,
         with ThreadPoolExecutor(threads) as ex:
             list(ex.map(run, _ranges(B, threads)))
     return {"accept_len": acc, "tokens": tok, "draft_index": didx, "tie": tie}
+
+
+# ------------------------------------------------------- draft selection bandit
+def gamma_sample(alpha: float, seed: int, round_: int, slot: int) -> float:
+    return lib().svo_gamma_sample(alpha, seed, round_, slot)
+
+
+def beta_sample(a: float, b: float, seed: int, round_: int, arm: int) -> float:
+    return lib().svo_beta_sample(a, b, seed, round_, arm)
+
+
+def bandit_uniform(seed: int, c0: int, round_: int, slot: int, tag: int, half: int = 0) -> float:
+    return lib().svo_bandit_uniform(seed, c0, round_, slot, tag, half)
+
+
+def ucb1_select(pulls, reward_sum) -> int:
+    n = np.ascontiguousarray(pulls, dtype=np.int64)
+    s = np.ascontiguousarray(reward_sum, dtype=np.float64)
+    return int(lib().svo_ucb1_select(len(n), _ptr(n), _ptr(s)))
+
+
+def thompson_select(succ, fail, seed: int, round_: int):
+    S = np.ascontiguousarray(succ, dtype=np.int64)
+    F = np.ascontiguousarray(fail, dtype=np.int64)
+    theta = np.empty(len(S), dtype=np.float64)
+    arm = int(lib().svo_thompson_select(len(S), _ptr(S), _ptr(F), seed, round_, _ptr(theta)))
+    return arm, theta
+
+
+def thompson_trial(reward: float, seed: int, round_: int, arm: int) -> bool:
+    return bool(lib().svo_thompson_trial(reward, seed, round_, arm))
+
+
+class BanditOracle:
+    """The selector's state machine, step by step: select() at select round
+    t_s, update(arm, reward) at update round t_u (both count from 0)."""
+
+    def __init__(self, K: int, policy: str = "ucb1", seed: int = 0):
+        self.K, self.policy, self.seed = K, policy, seed
+        self.pulls = np.zeros(K, np.int64)
+        self.sums = np.zeros(K, np.float64)
+        self.succ = np.zeros(K, np.int64)
+        self.fail = np.zeros(K, np.int64)
+        self.t_s = self.t_u = 0
+
+    def select(self) -> int:
+        if self.policy == "ucb1":
+            arm = ucb1_select(self.pulls, self.sums)
+        else:
+            arm, _ = thompson_select(self.succ, self.fail, self.seed, self.t_s)
+        self.t_s += 1
+        return arm
+
+    def update(self, arm: int, reward: float) -> None:
+        self.pulls[arm] += 1
+        self.sums[arm] += reward
+        if self.policy != "ucb1":
+            if thompson_trial(reward, self.seed, self.t_u, arm):
+                self.succ[arm] += 1
+            else:
+                self.fail[arm] += 1
+        self.t_u += 1

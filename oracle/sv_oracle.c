@@ -593,3 +593,122 @@ int svo_verify_multidraft_rows(const void* target, const void* draft, const int3
               per_draft != 0, b, rng, out_accept_len, out_tokens, out_draft_index, out_tie);
   return 0;
 }
+
+/* ---------------------------------------------------------------------------
+ * Draft selection as a K-armed bandit ([FS] Methodology s.2): before each
+ * decoding step one draft model (an arm) is chosen from the acceptance
+ * history alone; the reward of a step is its fraction of accepted draft
+ * tokens, in [0, 1].  Two policies, as the page lists them:
+ *  - UCB1 (Auer, Cesa-Bianchi, Fischer, "Finite-time Analysis of the
+ *    Multiarmed Bandit Problem", 2002): every arm once, in index order; then
+ *    the arm with the largest mean reward + sqrt(2 ln n / n_j), n the number
+ *    of pulls so far; ties go to the lower index.
+ *  - Thompson Sampling for rewards in [0, 1] (Agrawal, Goyal, "Analysis of
+ *    Thompson Sampling for the Multi-armed Bandit Problem", 2012): a
+ *    Beta(S_j + 1, F_j + 1) draw per arm, the largest draw wins (ties to the
+ *    lower index); a reward r counts as a success with probability r (one
+ *    Bernoulli trial), else as a failure.
+ * Randomness: Philox4x32-10 keyed by the seed; counter (c0, round, slot,
+ * tag << 24) with tag 5 for the Beta draws (slot = 2 arm + {0: X, 1: Y} of
+ * Beta = X / (X + Y) with X, Y Gamma) and tag 6 for the success trials
+ * (slot = arm).  A uniform in (0, 1) takes two words w0, w1 of a block:
+ * m = ((w0 << 32) | w1) >> 12, u = (2m + 1) 2^-53, exact in fp64.
+ * Gamma(alpha >= 1) by Marsaglia and Tsang ("A Simple Method for Generating
+ * Gamma Variables", 2000): d = alpha - 1/3, c = 1 / sqrt(9 d); repeat
+ * z ~ N(0, 1), v = (1 + c z)^3 while v <= 0 or
+ * ln u >= z^2 / 2 + d - d v + d ln v; return d v.  Iteration i takes u1, u2
+ * from Philox block c0 = i (word pairs 0-1 and 2-3), z = sqrt(-2 ln u1)
+ * cos(2 pi u2) (Box-Muller), and u from block c0 = i + 2^31 (words 0-1).  At
+ * most 64 iterations (then d is returned; each is accepted with probability
+ * above 0.95).
+ * ------------------------------------------------------------------------ */
+#define BANDIT_TAG_BETA 5u
+#define BANDIT_TAG_TRIAL 6u
+#define GAMMA_MAX_ITERS 64
+#define TWO_PI 6.283185307179586476925 /* 2 pi, rounded to the nearest double */
+
+static double u01_pair(uint32_t w0, uint32_t w1) {
+  const uint64_t m = ((((uint64_t)w0) << 32) | (uint64_t)w1) >> 12;
+  return (double)(2u * m + 1u) * 0x1p-53;
+}
+
+static void bandit_block(uint64_t seed, uint32_t c0, uint32_t round, uint32_t slot, uint32_t tag,
+                         uint32_t out[4]) {
+  const uint32_t ctr[4] = {c0, round, slot, tag << 24};
+  const uint32_t key[2] = {(uint32_t)seed, (uint32_t)(seed >> 32)};
+  svo_philox4x32_10(ctr, key, out);
+}
+
+double svo_bandit_uniform(uint64_t seed, uint32_t c0, uint32_t round, uint32_t slot, uint32_t tag,
+                          int half) {
+  uint32_t w[4];
+  bandit_block(seed, c0, round, slot, tag, w);
+  return half ? u01_pair(w[2], w[3]) : u01_pair(w[0], w[1]);
+}
+
+double svo_gamma_sample(double alpha, uint64_t seed, uint32_t round, uint32_t slot) {
+  if (!(alpha >= 1.0)) return NAN;
+  const double d = alpha - 1.0 / 3.0;
+  const double c = 1.0 / sqrt(9.0 * d);
+  for (uint32_t i = 0; i < GAMMA_MAX_ITERS; ++i) {
+    uint32_t w[4], w3[4];
+    bandit_block(seed, i, round, slot, BANDIT_TAG_BETA, w);
+    bandit_block(seed, i + 0x80000000u, round, slot, BANDIT_TAG_BETA, w3);
+    const double u1 = u01_pair(w[0], w[1]);
+    const double u2 = u01_pair(w[2], w[3]);
+    const double u = u01_pair(w3[0], w3[1]);
+    const double z = sqrt(-2.0 * log(u1)) * cos(TWO_PI * u2);
+    const double t = 1.0 + c * z;
+    if (t <= 0.0) continue;
+    const double v = t * t * t;
+    if (log(u) < 0.5 * z * z + d - d * v + d * log(v)) return d * v;
+  }
+  return d;
+}
+
+double svo_beta_sample(double a, double b, uint64_t seed, uint32_t round, uint32_t arm) {
+  const double x = svo_gamma_sample(a, seed, round, 2u * arm);
+  const double y = svo_gamma_sample(b, seed, round, 2u * arm + 1u);
+  return x / (x + y);
+}
+
+int svo_ucb1_select(int K, const int64_t* pulls, const double* reward_sum) {
+  if (K < 1 || !pulls || !reward_sum) return -1;
+  int64_t n = 0;
+  for (int j = 0; j < K; ++j) {
+    if (pulls[j] == 0) return j; /* every arm once, in index order */
+    n += pulls[j];
+  }
+  int best = 0;
+  double best_v = -INFINITY;
+  for (int j = 0; j < K; ++j) {
+    const double mean = reward_sum[j] / (double)pulls[j];
+    const double v = mean + sqrt(2.0 * log((double)n) / (double)pulls[j]);
+    if (v > best_v) {
+      best_v = v;
+      best = j;
+    }
+  }
+  return best;
+}
+
+int svo_thompson_select(int K, const int64_t* succ, const int64_t* fail, uint64_t seed,
+                        uint32_t round, double* theta) {
+  if (K < 1 || !succ || !fail) return -1;
+  int best = 0;
+  double best_v = -INFINITY;
+  for (int j = 0; j < K; ++j) {
+    const double t = svo_beta_sample((double)succ[j] + 1.0, (double)fail[j] + 1.0, seed, round,
+                                     (uint32_t)j);
+    if (theta) theta[j] = t;
+    if (t > best_v) {
+      best_v = t;
+      best = j;
+    }
+  }
+  return best;
+}
+
+int svo_thompson_trial(double reward, uint64_t seed, uint32_t round, uint32_t arm) {
+  return svo_bandit_uniform(seed, 0u, round, arm, BANDIT_TAG_TRIAL, 0) < reward ? 1 : 0;
+}

@@ -133,6 +133,26 @@ int svo_verify_multidraft_rows(const void* target, const void* draft, const int3
                                int32_t* out_tokens, int32_t* out_draft_index,
                                uint8_t* out_tie, const svo_rng* rng);
 
+/* ---- draft selection bandit ([FS] Methodology s.2) -------------------
+ * Rewards are fractions of accepted draft tokens, in [0, 1].
+ * svo_bandit_uniform: uniform in (0, 1) from Philox block (c0, round, slot,
+ *   tag << 24), word pair 0-1 (half = 0) or 2-3 (half = 1).
+ * svo_gamma_sample: Gamma(alpha, 1), alpha >= 1 (Marsaglia-Tsang), NaN for
+ *   alpha < 1.  svo_beta_sample: X / (X + Y), X ~ Gamma(a) on slot 2 arm,
+ *   Y ~ Gamma(b) on slot 2 arm + 1.
+ * svo_ucb1_select: UCB1 arm for pulls[K] and reward sums[K] (-1 on bad args).
+ * svo_thompson_select: Thompson arm for successes / failures [K] at `round`;
+ *   theta[K] (may be NULL) receives the Beta draws.
+ * svo_thompson_trial: 1 if a reward counts as a success at update `round`. */
+double svo_bandit_uniform(uint64_t seed, uint32_t c0, uint32_t round, uint32_t slot, uint32_t tag,
+                          int half);
+double svo_gamma_sample(double alpha, uint64_t seed, uint32_t round, uint32_t slot);
+double svo_beta_sample(double a, double b, uint64_t seed, uint32_t round, uint32_t arm);
+int svo_ucb1_select(int K, const int64_t* pulls, const double* reward_sum);
+int svo_thompson_select(int K, const int64_t* succ, const int64_t* fail, uint64_t seed,
+                        uint32_t round, double* theta);
+int svo_thompson_trial(double reward, uint64_t seed, uint32_t round, uint32_t arm);
+
 #ifdef __cplusplus
 }
 #endif
