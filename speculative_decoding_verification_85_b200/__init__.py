@@ -5,10 +5,11 @@ kernels, ``include/spec_verify.h``); this package is a thin ctypes binding
 that marshals torch tensors (device memory, the current stream) into that ABI.
 It performs no computation of its own and has no CPU fallback: importing it
 without the built library, or calling it on tensors that are not on a CUDA
-device, raises.
+device, raises.  The same library holds the host-side draft selector
+(``include/sv_bandit.h``, native C++), bound here as ``Bandit``.
 """
 from ._binding import (  # noqa: F401
-    BF16, F32, SpecVerifyError, Verifier, lib, library_path, multidraft_workspace_size,
+    BF16, F32, Bandit, SpecVerifyError, Verifier, lib, library_path, multidraft_workspace_size,
     spec_verify, spec_verify_host, spec_verify_multidraft, spec_verify_noalloc,
     spec_verify_noalloc_max_workspace, staging_size, workspace_size,
 )
@@ -16,5 +17,5 @@ from ._binding import (  # noqa: F401
 __all__ = [
     "spec_verify", "spec_verify_multidraft", "spec_verify_host", "Verifier", "workspace_size",
     "multidraft_workspace_size", "staging_size", "SpecVerifyError", "lib", "library_path",
-    "spec_verify_noalloc", "spec_verify_noalloc_max_workspace",
+    "spec_verify_noalloc", "spec_verify_noalloc_max_workspace", "Bandit",
 ]

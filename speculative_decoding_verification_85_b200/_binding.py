@@ -58,6 +58,18 @@ def lib() -> C.CDLL:
             L.spec_verify_noalloc.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, u64, u64, vp, vp,
                                               vp, vp, vp]
             L.spec_verify_noalloc.restype = i32
+            L.sv_bandit_create.argtypes = [i32, i32, u64]
+            L.sv_bandit_create.restype = vp
+            L.sv_bandit_destroy.argtypes = [vp]
+            L.sv_bandit_destroy.restype = None
+            L.sv_bandit_select.argtypes = [vp, C.POINTER(C.c_int)]
+            L.sv_bandit_select.restype = i32
+            L.sv_bandit_update.argtypes = [vp, i32, C.c_double]
+            L.sv_bandit_update.restype = i32
+            L.sv_bandit_update_accept.argtypes = [vp, i32, vp, i32, i32]
+            L.sv_bandit_update_accept.restype = i32
+            L.sv_bandit_stats.argtypes = [vp, vp, vp]
+            L.sv_bandit_stats.restype = i32
             _lib = L
     return _lib
 
@@ -251,3 +263,48 @@ class Verifier:
         ws = self._workspace(multidraft_workspace_size(B, tokens.shape[1], l1 - 1, V,
                                                        _dt(target)))
         return spec_verify_multidraft(target, draft, tokens, temps, workspace=ws, **kw)
+
+
+class Bandit:
+    """Online draft selection (include/sv_bandit.h): K arms, policy "ucb1" or
+    "thompson".  select() gives the arm (draft model) for the next step;
+    update(arm, reward) or update_from_accept(arm, accept_len, gamma) records
+    the outcome.  Host-side by design: accept_len is read from the host (a
+    device tensor is copied back, B int32 values)."""
+
+    POLICIES = {"ucb1": 0, "thompson": 1}
+
+    def __init__(self, K: int, policy: str = "ucb1", seed: int = 0):
+        if policy not in self.POLICIES:
+            raise ValueError(f"policy must be one of {sorted(self.POLICIES)}")
+        self.K = K
+        self._h = lib().sv_bandit_create(K, self.POLICIES[policy], seed)
+        if not self._h:
+            raise SpecVerifyError(1, lib().spec_verify_last_error().decode())
+
+    def select(self) -> int:
+        arm = C.c_int(-1)
+        _check(lib().sv_bandit_select(self._h, C.byref(arm)))
+        return arm.value
+
+    def update(self, arm: int, reward: float) -> None:
+        _check(lib().sv_bandit_update(self._h, arm, float(reward)))
+
+    def update_from_accept(self, arm: int, accept_len, gamma: int) -> None:
+        a = torch.as_tensor(accept_len).to("cpu", torch.int32).contiguous()
+        _check(lib().sv_bandit_update_accept(self._h, arm, a.data_ptr() if a.numel() else None,
+                                             a.numel(), gamma))
+
+    def stats(self):
+        pulls = torch.zeros(self.K, dtype=torch.int64)
+        sums = torch.zeros(self.K, dtype=torch.float64)
+        _check(lib().sv_bandit_stats(self._h, pulls.data_ptr(), sums.data_ptr()))
+        return pulls, sums
+
+    def close(self) -> None:
+        if getattr(self, "_h", None):
+            lib().sv_bandit_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        self.close()

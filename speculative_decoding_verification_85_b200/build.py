@@ -15,7 +15,8 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libspecverify.so")
-SOURCES = sorted(glob.glob(os.path.join(HERE, "csrc", "*.cu")))
+SOURCES = sorted(glob.glob(os.path.join(HERE, "csrc", "*.cu")) +
+                 glob.glob(os.path.join(HERE, "host", "*.cpp")))
 DEPS = SOURCES + sorted(glob.glob(os.path.join(HERE, "csrc", "*.cuh")) +
                         glob.glob(os.path.join(HERE, "csrc", "*.h")) +
                         glob.glob(os.path.join(ROOT, "include", "*.h")))
@@ -23,7 +24,7 @@ NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = [
     "-O3", "-std=c++17", "-lineinfo",
     "-gencode", "arch=compute_100a,code=sm_100a",
-    "-Xcompiler", "-fPIC,-O2", "-shared", "--expt-relaxed-constexpr",
+    "-Xcompiler", "-fPIC,-O2,-ffp-contract=off", "-shared", "--expt-relaxed-constexpr",
     "-I" + os.path.join(ROOT, "include"), "-I" + os.path.join(HERE, "csrc"),
 ]
 
