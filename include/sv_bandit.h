@@ -20,8 +20,9 @@
  * round t and tag 5 (slots 2j, 2j + 1 for the two Gamma variates of arm j,
  * Marsaglia-Tsang with Box-Muller normals), the success trial of update call
  * number t uses round t, slot j and tag 6.  A uniform is (2m + 1) 2^-53 with
- * m the top 52 bits of two Philox words.  Results are therefore a function of
- * (K, policy, seed, the sequence of calls).
+ * m the top 52 bits of two Philox words (the round counters wrap modulo
+ * 2^32).  Results are therefore a function of (K, policy, seed, the sequence
+ * of calls).
  *
  * Memory and threads: a handle owns its state (O(K) bytes, no device
  * memory); calls on one handle are serialised internally.  Errors return a
