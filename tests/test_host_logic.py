@@ -164,3 +164,26 @@ def test_rows_per_step():
     assert workloads.get(1).rows_per_step == 16 * 5
     assert workloads.get(3).rows_per_step == 8 * 4 * 5
     assert workloads.get(4).rows_per_step == 256 * 4
+
+
+def test_clock_summary_from_sampled_rows(tmp_path):
+    """The bench's clock record: median SM clock under load, the maximum,
+    and every throttle reason seen active during the timed region."""
+    rows = [
+        "0, 1965, 1965, 300.5, 0x0, Not Active, Not Active, Not Active, Not Active, 0",
+        "0, 1900, 1965, 610.0, 0x4, Not Active, Not Active, Not Active, Active, 98",
+        "0, 1950, 1965, 640.2, 0x0, Not Active, Not Active, Not Active, Not Active, 100",
+        "0, 1965, 1965, 655.9, 0x0, Not Active, Not Active, Not Active, Not Active, 100",
+        "garbage line",
+    ]
+    p = tmp_path / "clk.csv"
+    p.write_text("\n".join(rows) + "\n")
+    c = bench.ClockSampler(0)
+    c.path = str(p)
+    s = c.summary()
+    assert s["sm_mhz"] == 1950.0  # median of the three samples with load
+    assert s["sm_max_mhz"] == 1965.0 and s["samples"] == 3
+    assert s["reasons"] == ["sw_power_cap"] and s["power_w_max"] == 655.9
+    c2 = bench.ClockSampler(0)
+    c2.path = str(tmp_path / "missing.csv")
+    assert c2.summary()["reasons"] == ["unavailable"]
