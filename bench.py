@@ -46,7 +46,8 @@ import workloads  # noqa: E402
 METRIC = ("verified draft rows/s and achieved HBM GB/s vs B200 peak "
           "(spec_verify, 1 GPU)")
 UNIT = "rows/s"
-DEFAULT_CONFIG = "c1_b16_g5_v32000_bf16"
+DEFAULT_CONFIG = "c4_b256_g4_v151936_bf16"
+NOMINAL_HBM_GBS = 8000.0  # B200 HBM3e, nominal (DGX figure)
 L2_BYTES = 126 * 2**20
 
 
@@ -96,27 +97,38 @@ def step_bytes(cfg: workloads.Config, temps: torch.Tensor, accept_len=None) -> d
     return {"formula": formula, "algorithmic": algo}
 
 
+def gpu_ident(dev) -> str:
+    """nvidia-smi's id of a torch device: its UUID ("GPU-..."), so that the
+    sampler watches the GPU this process uses whatever CUDA_VISIBLE_DEVICES
+    remaps (nvidia-smi ignores that variable and counts physical GPUs)."""
+    u = str(torch.cuda.get_device_properties(dev).uuid)
+    return u if u.startswith("GPU-") else "GPU-" + u
+
+
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms, for one GPU
+    named by its nvidia-smi id (UUID)."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap,"
               "utilization.gpu")
 
-    def __init__(self, index: int):
-        self.index = index
+    def __init__(self, ident: str):
+        self.ident = str(ident)
         self.proc = None
         self.path = None
+
+    def command(self) -> list:
+        return ["nvidia-smi", "-i", self.ident, f"--query-gpu={self.FIELDS}",
+                "--format=csv,noheader,nounits", "-lms", "200"]
 
     def __enter__(self):
         fd, self.path = tempfile.mkstemp(suffix=".csv")
         os.close(fd)
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
-                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            self.proc = subprocess.Popen(self.command(), stdout=open(self.path, "w"),
+                                         stderr=subprocess.DEVNULL)
         except FileNotFoundError:
             self.proc = None
         time.sleep(0.3)
@@ -141,7 +153,8 @@ class ClockSampler:
                         rows.append(p)
             os.unlink(self.path)
         if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0,
+                    "gpu": self.ident}
 
         def num(x):
             try:
@@ -156,7 +169,7 @@ class ClockSampler:
                           if r[5 + i].lower().startswith("active")})
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(num(r[2]) for r in rows),
                 "reasons": reasons, "samples": len(load),
-                "power_w_max": max(num(r[3]) for r in rows)}
+                "power_w_max": max(num(r[3]) for r in rows), "gpu": self.ident}
 
 
 def _dist_init():
@@ -203,22 +216,38 @@ def _sum_over_ranks(x: float, world: int, device) -> float:
     return float(t.item())
 
 
-def ring_size(cfg: workloads.Config, total_steps: int) -> int:
+def ring_size(cfg: workloads.Config) -> int:
+    """Distinct resident input sets the timed steps cycle through: at least 8
+    and at least 4x the L2 size in total, whatever the step count, capped
+    near 24 GB of device memory."""
     es = 2 if cfg.dtype == "bf16" else 4
     per = cfg.B * (2 * cfg.gamma + 1) * cfg.V * es
-    need = max(8, -(-4 * L2_BYTES // per))  # at least 8 sets and 4x the L2 size
-    cap = max(2, int(24e9 // per))          # at most ~24 GB of inputs
-    return int(max(2, min(total_steps, need, cap)))
+    need = max(8, -(-4 * L2_BYTES // per))
+    cap = max(2, int(24e9 // per))
+    return int(max(2, min(need, cap)))
 
 
 # ------------------------------------------------------------------- oracle
+REF_SAMPLE_B = 32  # sequences per oracle step on the large workloads (bounded CPU sample)
+
+
+def oracle_batch(cfg) -> int:
+    """Sequences per step in the oracle's timed sample: the whole batch, or
+    the first REF_SAMPLE_B sequences of it (same recipe, same temperatures)
+    on the workloads whose full step would take the single-threaded oracle
+    seconds."""
+    return min(cfg.B, REF_SAMPLE_B)
+
+
 def time_oracle(cfg, sample_steps: int, threads: int, budget_s: float, rank: int = 0):
     """Run the oracle on up to `sample_steps` steps (stopping after
-    `budget_s`); return (rows/s, steps done, seconds)."""
+    `budget_s`); return (rows/s, steps done, seconds, sequences per step)."""
     import oracle
+    Bs = oracle_batch(cfg)
+    rows_per = cfg.rows_per_step // cfg.B * Bs
     done, t_total, rows = 0, 0.0, 0
     for s in range(sample_steps):
-        st = workloads.make_step(cfg, s + 100000 * rank, device="cpu")
+        st = workloads.make_step(cfg, s + 100000 * rank, device="cpu", B=Bs)
         tg, dr, tok, tm = workloads.host_inputs(st)
         t0 = time.perf_counter()
         if cfg.multidraft:
@@ -226,11 +255,11 @@ def time_oracle(cfg, sample_steps: int, threads: int, budget_s: float, rank: int
         else:
             oracle.verify(tg, dr, tok, tm, seed=rank, step=s, threads=threads)
         t_total += time.perf_counter() - t0
-        rows += cfg.rows_per_step
+        rows += rows_per
         done += 1
         if t_total >= budget_s:
             break
-    return rows / t_total, done, t_total
+    return rows / t_total, done, t_total, Bs
 
 
 def run_reference(args, cfg):
@@ -242,10 +271,10 @@ def run_reference(args, cfg):
         cores = len(os.sched_getaffinity(0))
     except AttributeError:
         cores = os.cpu_count() or 1
-    threads = max(1, min(cores, cfg.B))
+    threads = max(1, min(cores, oracle_batch(cfg)))
     # W untimed warm-up steps, as reported in the line
     time_oracle(cfg, args.warmup, threads, 1e9)
-    value, done, secs = time_oracle(cfg, args.steps, threads, args.ref_budget)
+    value, done, secs, Bs = time_oracle(cfg, args.steps, threads, args.ref_budget)
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
         "steps": done, "warmup": args.warmup, "ms_per_step": 1e3 * secs / done,
@@ -253,7 +282,8 @@ def run_reference(args, cfg):
         "data": "synthetic", "config": {"workload": cfg.name, "B": cfg.B, "gamma": cfg.gamma,
                                         "V": cfg.V, "K": cfg.K or None, "logits": cfg.dtype},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
-                         "sample": f"{done} full steps of {cfg.name} (requested {args.steps}), "
+                         "sample": f"{done} steps of {cfg.name} (requested {args.steps}), "
+                                   f"{Bs} of its {cfg.B} sequences per step, "
                                    f"sequences split over {threads} host threads"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -268,7 +298,7 @@ def run_ours(args, cfg):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     K, W = args.steps, args.warmup
-    R = ring_size(cfg, K + W)
+    R = ring_size(cfg)
     sets = [workloads.make_step(cfg, s + 100000 * rank, device=dev) for s in range(R)]
     dt = sv.BF16 if cfg.dtype == "bf16" else sv.F32
     B, g, V = cfg.B, cfg.gamma, cfg.V
@@ -312,7 +342,7 @@ def run_ours(args, cfg):
     stream.synchronize()
 
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(dev.index) as clk:
+    with ClockSampler(gpu_ident(dev)) as clk:
         # soak so the clocks sampled below reflect this load
         t_end = time.time() + args.soak
         while time.time() < t_end:
@@ -393,9 +423,10 @@ def run_ours(args, cfg):
     # ---- CPU baseline: the oracle on a bounded sample (rank 0, N = 1 only)
     cpu = None
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
-        v, done, secs = time_oracle(cfg, args.cpu_steps, 1, args.cpu_budget)
+        v, done, secs, Bs = time_oracle(cfg, args.cpu_steps, 1, args.cpu_budget)
         cpu = {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle",
-               "sample": f"{done} full steps of {cfg.name}, single-threaded, {secs:.1f} s"}
+               "sample": f"{done} steps of {cfg.name}, {Bs} of its {cfg.B} sequences per "
+                         f"step, single-threaded, {secs:.1f} s"}
 
     if rank == 0:
         line = {
@@ -405,7 +436,8 @@ def run_ours(args, cfg):
             "config": {"workload": cfg.name, "B": cfg.B, "gamma": cfg.gamma, "V": cfg.V,
                        "K": cfg.K or None, "logits": cfg.dtype,
                        "inputs": f"ring of {R} distinct resident input sets "
-                                 f"({R * bytes_info['formula'] / 1e9:.2f} GB > L2); "
+                                 f"({R * bytes_info['formula'] / 1e9:.2f} GB, "
+                                 f"{R * bytes_info['formula'] / L2_BYTES:.1f}x L2); "
                                  "no L2 flush needed",
                        "launch": "K steps captured in one CUDA graph, replayed",
                        "parallelism": f"batch-sharded replicas x{world}"},
@@ -414,10 +446,18 @@ def run_ours(args, cfg):
                                     if cfg.multidraft else "rows_kernel + draw_kernel (whole step)"),
                          "achieved": algo_gbs, "peak": peak, "unit": "GB/s",
                          "frac": algo_gbs / peak, "traffic": traffic,
-                         "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)",
+                         "peak_source": (f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)"
+                                         if peak_kind == "measured" else
+                                         "fallback (an earlier copy-bandwidth measurement on "
+                                         "this pool; MEASURED_PEAKS.json absent)"),
+                         "peak_nominal": NOMINAL_HBM_GBS,
+                         "frac_nominal": algo_gbs / NOMINAL_HBM_GBS,
                          "algorithmic_bytes_per_launch": bytes_info["algorithmic"],
                          "formula_bytes_per_step": bytes_info["formula"],
-                         "formula_gbs": bytes_info["formula"] / (ms / K / 1e3) / 1e9},
+                         "formula_gbs": bytes_info["formula"] / (ms / K / 1e3) / 1e9,
+                         "formula_frac": bytes_info["formula"] / (ms / K / 1e3) / 1e9 / peak,
+                         "formula_frac_nominal":
+                             bytes_info["formula"] / (ms / K / 1e3) / 1e9 / NOMINAL_HBM_GBS},
             "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches_per_replay,
             "clocks": clocks,
             "accept": {"mean_accept_len": mean_len,

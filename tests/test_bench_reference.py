@@ -9,7 +9,8 @@ import subprocess
 import sys
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-ARGS = ["--impl", "reference", "--steps", "2", "--warmup", "3", "--ref-budget", "5"]
+ARGS = ["--impl", "reference", "--config", "c1_b16_g5_v32000_bf16", "--steps", "2", "--warmup",
+        "3", "--ref-budget", "5"]
 
 
 def _json_lines(out: str):
@@ -32,6 +33,17 @@ def _check_line(d: dict, n_gpus: int):
     assert e2e["h2d_bytes_per_step"] == 0 and e2e["d2h_bytes_per_step"] == 0
     # the rate is the workload's verified rows over the timed seconds
     assert abs(d["value"] * d["ms_per_step"] / 1e3 - 16 * 5) < 1e-6 * 16 * 5
+
+
+def test_default_workload_is_the_largest_single_gpu_one():
+    sys.path.insert(0, ROOT)
+    import bench
+    import workloads
+    assert bench.DEFAULT_CONFIG == "c4_b256_g4_v151936_bf16"
+    big = max(workloads.CONFIGS, key=lambda c: c.B * (2 * c.gamma + 1) * c.V)
+    assert bench.DEFAULT_CONFIG == big.name
+    # the oracle's timed sample of it is a bounded subset of whole sequences
+    assert bench.oracle_batch(big) == 32 and bench.oracle_batch(workloads.get(1)) == 16
 
 
 def test_reference_arm_single_process():
