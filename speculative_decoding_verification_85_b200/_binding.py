@@ -104,6 +104,13 @@ def _stream(device, stream):
     return C.c_void_p(stream.cuda_stream)
 
 
+def _on(device):
+    """The C library works on the current CUDA device (its device checks and
+    per-device caches ask cudaGetDevice): make the tensors' device current for
+    the call."""
+    return torch.cuda.device(device)
+
+
 def workspace_size(B: int, gamma: int, V: int, dtype: int) -> int:
     return int(lib().spec_verify_workspace_size(B, gamma, V, dtype))
 
@@ -149,10 +156,12 @@ def spec_verify(target, draft, tokens, temps, *, seed: int = 0, step: int = 0, w
         out_draft_logp = torch.empty((B, g), dtype=torch.float32, device=dev)
     if workspace is None:
         workspace = _zeroed(workspace_size(B, g, V, dt), dev)
-    _check(lib().spec_verify(_ptr(target), _ptr(draft), _ptr(tokens), _ptr(temps), B, g, V, dt,
-                             seed, step, _ptr(out_accept_len), _ptr(out_tokens),
-                             _ptr(out_target_logp), _ptr(out_draft_logp), _ptr(workspace),
-                             workspace.numel() * workspace.element_size(), _stream(dev, stream)))
+    with _on(dev):
+            _check(lib().spec_verify(_ptr(target), _ptr(draft), _ptr(tokens), _ptr(temps), B, g, V,
+                                 dt, seed, step, _ptr(out_accept_len), _ptr(out_tokens),
+                                 _ptr(out_target_logp), _ptr(out_draft_logp), _ptr(workspace),
+                                 workspace.numel() * workspace.element_size(),
+                                 _stream(dev, stream)))
     return out_accept_len, out_tokens, out_target_logp, out_draft_logp
 
 
@@ -182,11 +191,13 @@ def spec_verify_multidraft(target, draft, tokens, temps, *, seed: int = 0, step:
         out_draft_index = torch.empty(B, dtype=torch.int32, device=dev)
     if workspace is None:
         workspace = _zeroed(multidraft_workspace_size(B, K, L, V, dt), dev)
-    _check(lib().spec_verify_multidraft(_ptr(target), _ptr(draft), _ptr(tokens), _ptr(temps), B,
-                                        K, L, V, dt, seed, step, _ptr(out_accept_len),
-                                        _ptr(out_tokens), _ptr(out_draft_index), _ptr(workspace),
-                                        workspace.numel() * workspace.element_size(),
-                                        _stream(dev, stream)))
+    with _on(dev):
+        _check(lib().spec_verify_multidraft(_ptr(target), _ptr(draft), _ptr(tokens), _ptr(temps),
+                                            B, K, L, V, dt, seed, step, _ptr(out_accept_len),
+                                            _ptr(out_tokens), _ptr(out_draft_index),
+                                            _ptr(workspace),
+                                            workspace.numel() * workspace.element_size(),
+                                            _stream(dev, stream)))
     return out_accept_len, out_tokens, out_draft_index
 
 
@@ -207,11 +218,12 @@ def spec_verify_host(target, draft, tokens, temps, *, staging, seed: int = 0, st
         out_tokens = torch.empty((B, g + 1), dtype=torch.int32, pin_memory=True)
     lp = torch.empty((B, g), dtype=torch.float32, pin_memory=True) if with_logprobs else None
     lq = torch.empty((B, g), dtype=torch.float32, pin_memory=True) if with_logprobs else None
-    _check(lib().spec_verify_host(_ptr(target), _ptr(draft), _ptr(tokens), _ptr(temps), B, g, V,
-                                  dt, seed, step, _ptr(out_accept_len), _ptr(out_tokens),
-                                  _ptr(lp), _ptr(lq), _ptr(staging),
-                                  staging.numel() * staging.element_size(),
-                                  _stream(staging.device, stream)))
+    with _on(staging.device):
+        _check(lib().spec_verify_host(_ptr(target), _ptr(draft), _ptr(tokens), _ptr(temps), B, g,
+                                      V, dt, seed, step, _ptr(out_accept_len), _ptr(out_tokens),
+                                      _ptr(lp), _ptr(lq), _ptr(staging),
+                                      staging.numel() * staging.element_size(),
+                                      _stream(staging.device, stream)))
     return out_accept_len, out_tokens, lp, lq
 
 
@@ -229,10 +241,12 @@ def spec_verify_noalloc(target, draft, tokens, temps, *, seed: int = 0, step: in
                  (out_accept_len, "out_accept_len"), (out_tokens, "out_tokens")):
         _dev(t, n)
     B, g1, V = target.shape
-    _check(lib().spec_verify_noalloc(_ptr(target), _ptr(draft), _ptr(tokens), _ptr(temps), B,
-                                     g1 - 1, V, _dt(target), seed, step, _ptr(out_accept_len),
-                                     _ptr(out_tokens), _ptr(out_target_logp),
-                                     _ptr(out_draft_logp), _stream(target.device, stream)))
+    with _on(target.device):
+        _check(lib().spec_verify_noalloc(_ptr(target), _ptr(draft), _ptr(tokens), _ptr(temps), B,
+                                         g1 - 1, V, _dt(target), seed, step,
+                                         _ptr(out_accept_len), _ptr(out_tokens),
+                                         _ptr(out_target_logp), _ptr(out_draft_logp),
+                                         _stream(target.device, stream)))
     return out_accept_len, out_tokens, out_target_logp, out_draft_logp
 
 

@@ -68,6 +68,10 @@ extern "C" int spec_verify_noalloc(const void* target_logits, const void* draft_
                                    int32_t* out_accept_len, int32_t* out_tokens,
                                    float* out_target_logp, float* out_draft_logp, void* stream) {
   const size_t need = spec_verify_workspace_size(B, gamma, V, dtype);
+  if (B > 0 && need == 0)  // a bad shape: spec_verify reports it before any CUDA work
+    return spec_verify(target_logits, draft_logits, draft_tokens, temps, B, gamma, V, dtype, seed,
+                       step, out_accept_len, out_tokens, out_target_logp, out_draft_logp, nullptr,
+                       0, stream);
   if (B > 0 && need > SV_NOALLOC_MAX_WORKSPACE)
     return set_error(SV_ERR_WORKSPACE,
                      "spec_verify_noalloc: this shape needs %zu bytes of workspace, more than "

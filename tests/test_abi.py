@@ -74,3 +74,18 @@ def test_noalloc_rejects_shapes_beyond_its_fixed_workspace():
                                None, None)
     assert rc == 4
     assert b"fixed" in L.spec_verify_last_error()
+
+
+def test_noalloc_reports_bad_shapes_before_any_device_setup():
+    """A bad shape (gamma out of range) is reported as SV_ERR_INVALID_ARG, as
+    spec_verify reports it: the no-alloc entry point neither looks up its
+    fixed array nor queues its first-call clear (no CUDA device is needed)."""
+    L = sv.lib()
+    for g in (0, 65):
+        rc = L.spec_verify_noalloc(None, None, None, None, 1, g, 100, sv.BF16, 0, 0, None, None,
+                                   None, None, None)
+        assert rc == 1
+        assert b"draft length" in L.spec_verify_last_error()
+    rc = L.spec_verify_noalloc(None, None, None, None, 1, 4, 100, 9, 0, 0, None, None, None,
+                               None, None)
+    assert rc == 1 and b"dtype" in L.spec_verify_last_error()
