@@ -199,6 +199,44 @@ typedef struct {
   uint64_t seed, step;
 } philox_ctx;
 
+/* Tie rule T for a single-draft draw (a reading: the pages fix no tolerance
+ * for the draw).  A draw is logged as a Gumbel near-tie when another
+ * candidate's score could overtake the winner's once every weight carries
+ * the error of an fp32 evaluation of the probabilities: score s_v =
+ * ln w_v + G_v carries u_v = GUMBEL_TIE_BAND / 2 + (eta_p p_v + eta_q q_v) /
+ * w_v, with eta = 2e-6 + 2e-7 |ln prob| the relative error of a probability
+ * evaluated as 2^(fp32 exponent) from temperature-scaled fp32 logits and an
+ * fp32 row sum, and w_v = p_v - q_v (residual) or p_v (bonus, q = 0).  For a
+ * well-conditioned weight this is the fixed band (gap < GUMBEL_TIE_BAND); a
+ * residual weight of two nearly equal probabilities is ill-conditioned, and
+ * its band widens by (p + q) / (p - q).  lq == NULL: bonus draw. */
+static double prob_eta(double lp) { return 2e-6 + 2e-7 * fabs(lp); }
+
+static int draw_fragile(const double* lw, const double* lp, const double* lq, int64_t V,
+                        const philox_ctx* pc, uint32_t b, uint32_t pos, int64_t y) {
+  if (y < 0) return 0;
+  double sy = -INFINITY, uy = 0.0, other = -INFINITY;
+  for (int64_t v = 0; v < V; ++v) {
+    if (lw[v] == -INFINITY) continue;
+    const uint32_t x = svo_stream_word(pc->seed, pc->step, SVO_TAG_GUMBEL, b, 0, pos,
+                                       (uint32_t)(v >> 2), (uint32_t)(v & 3));
+    const double E = -log1p(-(1.0 - svo_u01_gumbel(x)));
+    const double score = lw[v] - log(E);
+    const double p = exp(lp[v]);
+    const double q = lq ? exp(lq[v]) : 0.0;
+    const double w = exp(lw[v]);
+    double u = 0.5 * GUMBEL_TIE_BAND;
+    u += (prob_eta(lp[v]) * p + (lq ? prob_eta(lq[v]) * q : 0.0)) / w;
+    if (v == y) {
+      sy = score;
+      uy = u;
+    } else if (score + u > other) {
+      other = score + u;
+    }
+  }
+  return other >= sy - uy;
+}
+
 static int philox_coin(void* ctx, double h, uint32_t tag, uint32_t b, uint32_t k,
                        uint32_t pos, double* gap) {
   const philox_ctx* c = (const philox_ctx*)ctx;
@@ -228,7 +266,8 @@ static double accept_prob(double lp, double lq) {
 
 static void seq_single(const char* target, const char* draft, const int32_t* tokens,
                        const float* temps, int gamma, int64_t V, int dtype, int64_t b,
-                       const svo_rng* rng, int32_t* out_accept_len, int32_t* out_tokens,
+                       const svo_rng* rng, const philox_ctx* pc, int32_t* out_accept_len,
+                       int32_t* out_tokens,
                        double* out_lp, double* out_lq, uint8_t* out_tie) {
   const size_t es = elem_size(dtype);
   const size_t rowb = (size_t)V * es;
@@ -307,11 +346,13 @@ static void seq_single(const char* target, const char* draft, const int32_t* tok
     return;
   }
   svo_row_logprobs(trow0 + (size_t)j * rowb, V, dtype, T, lpr);
+  int residual = 0;
   if (j < gamma) {
     /* Residual max(p_j - q_j, 0).  Reading: if it is identically zero (p_j
      * == q_j to rounding), draw from p_j. */
     svo_row_logprobs(drow0 + (size_t)j * rowb, V, dtype, T, lqr);
-    if (svo_residual_logw(lpr, lqr, V, lw) == 0) memcpy(lw, lpr, (size_t)V * sizeof(double));
+    residual = svo_residual_logw(lpr, lqr, V, lw) != 0;
+    if (!residual) memcpy(lw, lpr, (size_t)V * sizeof(double));
   } else {
     /* Every draft token accepted: bonus token from the target row gamma. */
     memcpy(lw, lpr, (size_t)V * sizeof(double));
@@ -319,6 +360,8 @@ static void seq_single(const char* target, const char* draft, const int32_t* tok
   double gap = INFINITY;
   const int64_t y = rng->categorical(rng->ctx, lw, V, SVO_TAG_GUMBEL, (uint32_t)b, (uint32_t)j, &gap);
   if (gap < GUMBEL_TIE_BAND) tie |= SVO_TIE_GUMBEL;
+  if (pc && draw_fragile(lw, lpr, residual ? lqr : NULL, V, pc, (uint32_t)b, (uint32_t)j, y))
+    tie |= SVO_TIE_GUMBEL;
   free(lw);
   free(lpr);
   free(lqr);
@@ -345,10 +388,11 @@ int svo_verify(const void* target, const void* draft, const int32_t* tokens,
   if (b_begin < 0 || b_end > B || b_begin > b_end) return -1;
   philox_ctx pc = {seed, step};
   svo_rng def = {&pc, philox_coin, philox_categorical};
+  const philox_ctx* tie_ctx = rng ? NULL : &pc; /* the draw tie rule needs the Philox stream */
   if (!rng) rng = &def;
   for (int64_t b = b_begin; b < b_end; ++b)
     seq_single((const char*)target, (const char*)draft, tokens, temps, gamma, V, dtype, b, rng,
-               out_accept_len, out_tokens, out_lp, out_lq, out_tie);
+               tie_ctx, out_accept_len, out_tokens, out_lp, out_lq, out_tie);
   return 0;
 }
 
