@@ -77,3 +77,42 @@ def test_select_update_cost(capsys):
         with capsys.disabled():
             print(f"\nbandit {policy}: {us:.2f} us per select + update (K = 3, via ctypes)")
         assert us < 200.0
+
+
+# ------------------------------------------- library-only pins (no oracle)
+def test_ucb1_pull_count_bound_from_the_index():
+    """UCB1 with deterministic rewards (arm 0 always 0.9, arm 1 always 0.1):
+    from the index mean + sqrt(2 ln n / n_j), arm 1 is pulled only while
+    sqrt(2 ln n / n_1) >= 0.8 + sqrt(2 ln n / n_0), so after n pulls
+    2 ln n / (0.8 + sqrt(2 ln n / n_0))^2 - 1 <= n_1 <= 2 ln n / 0.64 + 1."""
+    b = sv.Bandit(2, "ucb1", 0)
+    n = 10000
+    for _ in range(n):
+        a = b.select()
+        b.update(a, 0.9 if a == 0 else 0.1)
+    pulls, _ = b.stats()
+    n0, n1 = int(pulls[0]), int(pulls[1])
+    assert n0 + n1 == n
+    lo = 2 * np.log(n) / (0.8 + np.sqrt(2 * np.log(n) / n0)) ** 2 - 1
+    hi = 2 * np.log(n) / 0.64 + 1
+    assert lo <= n1 <= hi, (n1, lo, hi)
+
+
+def test_thompson_choice_frequency_is_the_beta_comparison():
+    """Thompson Sampling with successes / failures S = (3, 2), F = (1, 2):
+    each select draws Beta(S_j + 1, F_j + 1) per arm independently and picks
+    the larger, so arm 0 wins with probability P(X > Y), X ~ Beta(4, 2),
+    Y ~ Beta(3, 3) (numerical integral).  Rewards 1 and 0 are always a
+    success and a failure."""
+    from scipy import integrate, stats
+    b = sv.Bandit(2, "thompson", 99)
+    for arm, r in ((0, 1.0), (0, 1.0), (0, 1.0), (0, 0.0), (1, 1.0), (1, 1.0), (1, 0.0),
+                   (1, 0.0)):
+        b.update(arm, r)
+    X, Y = stats.beta(4, 2), stats.beta(3, 3)
+    p, _ = integrate.quad(lambda x: X.pdf(x) * Y.cdf(x), 0.0, 1.0)
+    n = 4000
+    wins = sum(b.select() == 0 for _ in range(n))
+    sd = np.sqrt(p * (1 - p) / n)
+    assert abs(wins / n - p) < 4.5 * sd, (wins / n, p)
+    assert b.stats()[0].tolist() == [4, 4]  # select alone changes no statistics
