@@ -298,7 +298,7 @@ def run_ours(args, cfg):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     K, W = args.steps, args.warmup
-    R = ring_size(cfg)
+    R = args.sets if args.sets else ring_size(cfg)
     sets = [workloads.make_step(cfg, s + 100000 * rank, device=dev) for s in range(R)]
     dt = sv.BF16 if cfg.dtype == "bf16" else sv.F32
     B, g, V = cfg.B, cfg.gamma, cfg.V
@@ -386,30 +386,47 @@ def run_ours(args, cfg):
         except Exception:
             traffic = None
 
-    # ---- e2e through the host-buffer entry point (single-draft workloads)
+    # ---- e2e through the host-buffer entry point (single-draft workloads):
+    # every step uploads its inputs from pinned host memory, verifies and
+    # downloads its outputs; two staging buffers on two streams in turn, so one
+    # step's upload overlaps the previous step's verification and download
     e2e = None
     if not cfg.multidraft:
-        staging = torch.zeros(sv.staging_size(B, g, V, dt), dtype=torch.uint8, device=dev)
+        nst = 2
+        stagings = [torch.zeros(sv.staging_size(B, g, V, dt), dtype=torch.uint8, device=dev)
+                    for _ in range(nst)]
+        streams = [stream, torch.cuda.Stream(device=dev)]
         nh = 2
         host = []
-        for s in range(nh):
-            st = sets[s]
+        for s_ in range(nh):
+            st = sets[s_]
             host.append([x.cpu().pin_memory() for x in (st.target, st.draft, st.tokens,
                                                         st.temps)])
-        acc_h = torch.empty(B, dtype=torch.int32, pin_memory=True)
-        tok_h = torch.empty((B, g + 1), dtype=torch.int32, pin_memory=True)
-        for i in range(min(W, 3) + 1):
-            sv.spec_verify_host(*host[i % nh], staging=staging, seed=seed, step=i,
-                                out_accept_len=acc_h, out_tokens=tok_h, stream=stream)
+        outs_h = [(torch.empty(B, dtype=torch.int32, pin_memory=True),
+                   torch.empty((B, g + 1), dtype=torch.int32, pin_memory=True))
+                  for _ in range(nst)]
+
+        def e2e_step(i):
+            k = i % nst
+            sv.spec_verify_host(*host[i % nh], staging=stagings[k], seed=seed, step=i,
+                                out_accept_len=outs_h[k][0], out_tokens=outs_h[k][1],
+                                stream=streams[k], wait=False)
+
+        for i in range(max(W, 3)):
+            e2e_step(i)
+        torch.cuda.synchronize(dev)
         ke = K
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        done1 = torch.cuda.Event()
         _barrier(world, local)
         torch.cuda.synchronize(dev)
-        e0.record(stream)
+        e0.record(streams[0])
+        streams[1].wait_event(e0)
         for i in range(ke):
-            sv.spec_verify_host(*host[i % nh], staging=staging, seed=seed, step=i,
-                                out_accept_len=acc_h, out_tokens=tok_h, stream=stream)
-        e1.record(stream)
+            e2e_step(i)
+        done1.record(streams[1])
+        streams[0].wait_event(done1)
+        e1.record(streams[0])
         torch.cuda.synchronize(dev)
         _barrier(world, local)
         ems = _max_over_ranks(e0.elapsed_time(e1), world, dev)
@@ -418,7 +435,9 @@ def run_ours(args, cfg):
         d2h = B * 4 + B * (g + 1) * 4
         e2e = {"value": _sum_over_ranks(cfg.rows_per_step * ke, world, dev) / (ems / 1e3),
                "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-               "ms_per_step": ems / ke, "path": "spec_verify_host (pinned host buffers)"}
+               "ms_per_step": ems / ke, "h2d_gbs": h2d / (ems / ke / 1e3) / 1e9,
+               "path": "spec_verify_host_async (pinned host buffers; two staging buffers "
+                       "on two streams in turn)"}
 
     # ---- CPU baseline: the oracle on a bounded sample (rank 0, N = 1 only)
     cpu = None
@@ -482,8 +501,16 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=10.0)
     ap.add_argument("--ref-budget", type=float, default=60.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="run the workload with this many sequences instead of its own B "
+                         "(small profiling captures; not a bench line)")
+    ap.add_argument("--sets", type=int, default=None,
+                    help="distinct input sets in the ring (default: at least 4x L2)")
     args = ap.parse_args()
     cfg = workloads.get(args.config)
+    if args.batch is not None and args.batch != cfg.B:
+        import dataclasses
+        cfg = dataclasses.replace(cfg, B=args.batch, name=f"{cfg.name}@B{args.batch}")
     if args.steps is None:
         args.steps = 1000 if cfg.index in (1, 3) else (200 if cfg.index == 2 else
                                                          (100 if cfg.index == 4 else 1000))

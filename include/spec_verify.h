@@ -149,6 +149,30 @@ int spec_verify_multidraft(const void* target_logits, const void* draft_logits,
                            void* stream);
 
 /*
+ * spec_verify_multidraft_rows -- multi-draft verification with a row set per
+ * draft, the prefix-conditioned use of SpecTr-GBV (Methodology, Algorithm 1:
+ * K i.i.d. draft sequences, each verified against the target's
+ * distributions after its own prefix).
+ *
+ * Inputs (device): target_logits [B, K, L+1, V] -- row (k, i) holds the
+ * target logits after draft k's own prefix x_k[0..i); draft_logits
+ * [B, K, L, V] likewise; draft_tokens [B, K, L]; temps [B].  Outputs and
+ * workspace (spec_verify_multidraft_workspace_size) as spec_verify_multidraft.
+ * Draft k is weighed with its own rows; the residual law starts from row set
+ * 0 (every draft shares the empty prefix) and, after an advance, comes from
+ * the accepted draft's rows; the whole-block correction is drawn from row L
+ * of the accepted draft.  With K equal copies of one row set the results are
+ * those of spec_verify_multidraft.  K (2L + 1) must not exceed 256 (row
+ * statistics kept per sequence): larger shapes return SV_ERR_UNSUPPORTED.
+ */
+int spec_verify_multidraft_rows(const void* target_logits, const void* draft_logits,
+                                const int32_t* draft_tokens, const float* temps, int B, int K,
+                                int L, int V, int dtype, uint64_t seed, uint64_t step,
+                                int32_t* out_accept_len, int32_t* out_tokens,
+                                int32_t* out_draft_index, void* workspace,
+                                size_t workspace_bytes, void* stream);
+
+/*
  * spec_verify_host -- spec_verify on HOST buffers, for callers whose logits
  * live in host memory.  The inputs are copied host->device into `staging`
  * (device memory, at least spec_verify_host_staging_size bytes, 256-byte
@@ -163,6 +187,23 @@ int spec_verify_host(const void* target_logits, const void* draft_logits,
                      int V, int dtype, uint64_t seed, uint64_t step, int32_t* out_accept_len,
                      int32_t* out_tokens, float* out_target_logp, float* out_draft_logp,
                      void* staging, size_t staging_bytes, void* stream);
+
+/*
+ * spec_verify_host_async -- spec_verify_host without the final
+ * synchronisation: the input copies, the verification and the output copies
+ * are enqueued on `stream` and the call returns; the host outputs are valid
+ * once the stream has reached that point.  With pinned host buffers, two
+ * staging buffers used on two streams in turn let one step's upload overlap
+ * the previous step's verification and download.  A staging buffer must not
+ * be reused before the work enqueued on it has finished (order it on its
+ * stream); the argument checks and errors are those of spec_verify_host.
+ */
+int spec_verify_host_async(const void* target_logits, const void* draft_logits,
+                           const int32_t* draft_tokens, const float* temps, int B, int gamma,
+                           int V, int dtype, uint64_t seed, uint64_t step,
+                           int32_t* out_accept_len, int32_t* out_tokens, float* out_target_logp,
+                           float* out_draft_logp, void* staging, size_t staging_bytes,
+                           void* stream);
 
 /*
  * spec_verify_noalloc -- spec_verify for callers that cannot allocate device

@@ -48,11 +48,15 @@ def lib() -> C.CDLL:
             L.spec_verify_multidraft.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, u64, u64,
                                                  vp, vp, vp, vp, sz, vp]
             L.spec_verify_multidraft.restype = i32
+            L.spec_verify_multidraft_rows.argtypes = list(L.spec_verify_multidraft.argtypes)
+            L.spec_verify_multidraft_rows.restype = i32
             L.spec_verify_host_staging_size.argtypes = [i32, i32, i32, i32]
             L.spec_verify_host_staging_size.restype = sz
             L.spec_verify_host.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, u64, u64, vp, vp,
                                            vp, vp, vp, sz, vp]
             L.spec_verify_host.restype = i32
+            L.spec_verify_host_async.argtypes = list(L.spec_verify_host.argtypes)
+            L.spec_verify_host_async.restype = i32
             L.spec_verify_noalloc_max_workspace.argtypes = []
             L.spec_verify_noalloc_max_workspace.restype = sz
             L.spec_verify_noalloc.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, u64, u64, vp, vp,
@@ -168,16 +172,26 @@ def spec_verify(target, draft, tokens, temps, *, seed: int = 0, step: int = 0, w
 def spec_verify_multidraft(target, draft, tokens, temps, *, seed: int = 0, step: int = 0,
                            workspace=None, out_accept_len=None, out_tokens=None,
                            out_draft_index=None, stream=None):
-    """Multi-draft verification: target [B, L+1, V], draft [B, L, V], tokens
-    [B, K, L] int32, temps [B].  Returns (accept_len, tokens [B, L+1], draft_index)."""
+    """Multi-draft verification: target [B, L+1, V], draft [B, L, V] shared by
+    the K drafts, tokens [B, K, L] int32, temps [B]; or, with a row set per
+    draft (the prefix-conditioned use), target [B, K, L+1, V] and draft
+    [B, K, L, V].  Returns (accept_len, tokens [B, L+1], draft_index)."""
     for t, n in ((target, "target"), (draft, "draft"), (tokens, "tokens"), (temps, "temps")):
         _dev(t, n)
-    B, l1, V = target.shape
+    per_draft = target.dim() == 4
+    if per_draft:
+        B, Kt, l1, V = target.shape
+    else:
+        B, l1, V = target.shape
     L = l1 - 1
     K = tokens.shape[1]
     dt = _dt(target)
-    if draft.dtype != target.dtype or tuple(draft.shape) != (B, L, V):
-        raise ValueError("draft must match target's dtype and be [B, L, V]")
+    lead = (B, K) if per_draft else (B,)
+    if per_draft and Kt != K:
+        raise ValueError("per-draft rows: target [B, K, L+1, V] with K = tokens.shape[1]")
+    if draft.dtype != target.dtype or tuple(draft.shape) != lead + (L, V):
+        raise ValueError("draft must match target's dtype and be [B, L, V] ([B, K, L, V] with "
+                         "a row set per draft)")
     if tokens.dtype != torch.int32 or tuple(tokens.shape) != (B, K, L):
         raise ValueError("tokens must be int32 [B, K, L]")
     if temps.dtype != torch.float32 or tuple(temps.shape) != (B,):
@@ -191,21 +205,24 @@ def spec_verify_multidraft(target, draft, tokens, temps, *, seed: int = 0, step:
         out_draft_index = torch.empty(B, dtype=torch.int32, device=dev)
     if workspace is None:
         workspace = _zeroed(multidraft_workspace_size(B, K, L, V, dt), dev)
+    fn = lib().spec_verify_multidraft_rows if per_draft else lib().spec_verify_multidraft
     with _on(dev):
-        _check(lib().spec_verify_multidraft(_ptr(target), _ptr(draft), _ptr(tokens), _ptr(temps),
-                                            B, K, L, V, dt, seed, step, _ptr(out_accept_len),
-                                            _ptr(out_tokens), _ptr(out_draft_index),
-                                            _ptr(workspace),
-                                            workspace.numel() * workspace.element_size(),
-                                            _stream(dev, stream)))
+        _check(fn(_ptr(target), _ptr(draft), _ptr(tokens), _ptr(temps), B, K, L, V, dt, seed,
+                  step, _ptr(out_accept_len), _ptr(out_tokens), _ptr(out_draft_index),
+                  _ptr(workspace), workspace.numel() * workspace.element_size(),
+                  _stream(dev, stream)))
     return out_accept_len, out_tokens, out_draft_index
 
 
 def spec_verify_host(target, draft, tokens, temps, *, staging, seed: int = 0, step: int = 0,
-                     out_accept_len=None, out_tokens=None, stream=None, with_logprobs=False):
+                     out_accept_len=None, out_tokens=None, stream=None, with_logprobs=False,
+                     wait: bool = True):
     """spec_verify on host (preferably pinned) CPU tensors through the C ABI's
     host-buffer entry point; `staging` is a zero-initialised CUDA uint8 tensor
-    of at least staging_size(...) bytes.  Synchronous."""
+    of at least staging_size(...) bytes.  wait=True returns after the outputs
+    have arrived (spec_verify_host); wait=False only enqueues the copies and
+    the verification on the stream (spec_verify_host_async): the outputs are
+    valid once the stream has reached that point."""
     B, g1, V = target.shape
     g = g1 - 1
     dt = _dt(target)
@@ -218,12 +235,11 @@ def spec_verify_host(target, draft, tokens, temps, *, staging, seed: int = 0, st
         out_tokens = torch.empty((B, g + 1), dtype=torch.int32, pin_memory=True)
     lp = torch.empty((B, g), dtype=torch.float32, pin_memory=True) if with_logprobs else None
     lq = torch.empty((B, g), dtype=torch.float32, pin_memory=True) if with_logprobs else None
+    fn = lib().spec_verify_host if wait else lib().spec_verify_host_async
     with _on(staging.device):
-        _check(lib().spec_verify_host(_ptr(target), _ptr(draft), _ptr(tokens), _ptr(temps), B, g,
-                                      V, dt, seed, step, _ptr(out_accept_len), _ptr(out_tokens),
-                                      _ptr(lp), _ptr(lq), _ptr(staging),
-                                      staging.numel() * staging.element_size(),
-                                      _stream(staging.device, stream)))
+        _check(fn(_ptr(target), _ptr(draft), _ptr(tokens), _ptr(temps), B, g, V, dt, seed, step,
+                  _ptr(out_accept_len), _ptr(out_tokens), _ptr(lp), _ptr(lq), _ptr(staging),
+                  staging.numel() * staging.element_size(), _stream(staging.device, stream)))
     return out_accept_len, out_tokens, lp, lq
 
 
@@ -273,7 +289,7 @@ class Verifier:
         return spec_verify(target, draft, tokens, temps, workspace=ws, **kw)
 
     def verify_multidraft(self, target, draft, tokens, temps, **kw):
-        B, l1, V = target.shape
+        B, l1, V = target.shape[0], target.shape[-2], target.shape[-1]
         ws = self._workspace(multidraft_workspace_size(B, tokens.shape[1], l1 - 1, V,
                                                        _dt(target)))
         return spec_verify_multidraft(target, draft, tokens, temps, workspace=ws, **kw)

@@ -17,13 +17,6 @@ thread_local char g_err[512] = "no error";
 constexpr size_t kAlign = 256;
 size_t up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
-// Pass-1 chunk: about 16 KB of logits per CTA (8192 bf16 / 4096 fp32).
-int chunks_per_row(int V, int dtype) {
-  const int per = dtype == SV_BF16 ? 8192 : 4096;
-  int nc = (V + per - 1) / per;
-  return nc < 1 ? 1 : nc;
-}
-
 bool sizes_ok(int B, int g, int V, int dtype) {
   return B >= 0 && B <= SV_MAX_BATCH && g >= 1 && g <= SV_MAX_GAMMA && V >= 1 && (dtype == SV_F32 || dtype == SV_BF16);
 }
@@ -73,38 +66,38 @@ Layout layout_single(int B, int gamma, int V, int dtype) {
   l.nc2 = draw_chunks(V, dtype);
   l.ctl = 0;
   l.ticket1 = kHeaderCtl;
-  l.ticket2 = kHeaderCtl + static_cast<size_t>(SV_MAX_BATCH) * sizeof(unsigned);
+  l.ticket2 = kHeaderCtl + kSeqSlots;
+  l.ready = kHeaderCtl + 2 * kSeqSlots;
+  l.bar = kHeaderCtl + 3 * kSeqSlots;
   size_t off = kHeaderBytes;
   l.part1 = off;  // row-pair partials: [B][gamma + 1][nseg] x 2 x 16 bytes
-  off += up(static_cast<size_t>(B) * (gamma + 1) * l.nc * 2 * sizeof(RowPartial));
+  off += up(static_cast<size_t>(B) * (gamma + 1) * l.nc * 2 * sizeof(float4));
   l.info = off;
   off += up(static_cast<size_t>(B) * sizeof(SeqInfo));
   l.part2 = off;
   off += up(static_cast<size_t>(B) * l.nc2 * sizeof(RacePartial));
   l.resid = off;  // the draft tokens' gathered logits: [B][gamma][nseg][2] fp32
   off += up(static_cast<size_t>(B) * gamma * l.nc * 2 * sizeof(float));
-  l.rowstat = 0;
   l.total = off;
   return l;
 }
 
 Layout layout_multi(int B, int K, int L, int V, int dtype) {
   (void)K;
+  (void)L;
+  (void)dtype;
   Layout l{};
-  l.nc = chunks_per_row(V, dtype);
+  l.nc = 0;
   l.nc2 = 0;
-  const size_t rps = static_cast<size_t>(2 * L + 1);
   l.ctl = 0;
   l.ticket1 = kHeaderCtl;
-  l.ticket2 = kHeaderCtl + static_cast<size_t>(SV_MAX_BATCH) * sizeof(unsigned);
+  l.ticket2 = kHeaderCtl + kSeqSlots;
+  l.ready = kHeaderCtl + 2 * kSeqSlots;
+  l.bar = kHeaderCtl + 3 * kSeqSlots;
   size_t off = kHeaderBytes;
-  l.part1 = off;
-  off += up(static_cast<size_t>(B) * rps * l.nc * sizeof(RowPartial));
-  l.rowstat = off;
-  off += up(static_cast<size_t>(B) * rps * sizeof(RowPartial));
-  l.resid = off;
-  off += up(static_cast<size_t>(B) * static_cast<size_t>(V) * sizeof(float));
-  l.info = l.part2 = 0;
+  l.resid = off;  // residual laws R (two per sequence) when they do not fit on chip
+  off += up(multidraft_global_bytes(B, V));
+  l.part1 = l.info = l.part2 = 0;
   l.total = off;
   return l;
 }
@@ -179,11 +172,11 @@ int spec_verify(const void* target_logits, const void* draft_logits, const int32
                        lay, static_cast<cudaStream_t>(stream));
 }
 
-int spec_verify_multidraft(const void* target_logits, const void* draft_logits,
+static int multidraft_call(const void* target_logits, const void* draft_logits,
                            const int32_t* draft_tokens, const float* temps, int B, int K, int L,
-                           int V, int dtype, uint64_t seed, uint64_t step, int32_t* out_accept_len,
-                           int32_t* out_tokens, int32_t* out_draft_index, void* workspace,
-                           size_t workspace_bytes, void* stream) {
+                           int V, int dtype, int per_draft, uint64_t seed, uint64_t step,
+                           int32_t* out_accept_len, int32_t* out_tokens, int32_t* out_draft_index,
+                           void* workspace, size_t workspace_bytes, void* stream) {
   if (K < 1 || K > SV_MAX_DRAFTS)
     return set_error(SV_ERR_INVALID_ARG, "K must be in [1, %d] (got %d)", SV_MAX_DRAFTS, K);
   const bool shape_ok = B > 0 && sizes_ok(B, L, V, dtype);
@@ -191,10 +184,35 @@ int spec_verify_multidraft(const void* target_logits, const void* draft_logits,
   int rc = check_common(target_logits, draft_logits, draft_tokens, temps, B, L, V, dtype, step,
                         out_accept_len, out_tokens, workspace, workspace_bytes, lay.total);
   if (rc != SV_OK || B == 0) return rc;
+  if (per_draft && K > multidraft_max_row_sets(L))
+    return set_error(SV_ERR_UNSUPPORTED,
+                     "per-draft rows: at most %d drafts of length %d (got K = %d)",
+                     multidraft_max_row_sets(L), L, K);
   if ((rc = check_device()) != SV_OK) return rc;
-  return launch_multi(target_logits, draft_logits, draft_tokens, temps, B, K, L, V, dtype, seed,
-                      step, out_accept_len, out_tokens, out_draft_index, workspace, lay,
-                      static_cast<cudaStream_t>(stream));
+  return launch_multi(target_logits, draft_logits, draft_tokens, temps, B, K, L, V, dtype,
+                      per_draft, seed, step, out_accept_len, out_tokens, out_draft_index,
+                      workspace, lay, static_cast<cudaStream_t>(stream));
+}
+
+int spec_verify_multidraft(const void* target_logits, const void* draft_logits,
+                           const int32_t* draft_tokens, const float* temps, int B, int K, int L,
+                           int V, int dtype, uint64_t seed, uint64_t step, int32_t* out_accept_len,
+                           int32_t* out_tokens, int32_t* out_draft_index, void* workspace,
+                           size_t workspace_bytes, void* stream) {
+  return multidraft_call(target_logits, draft_logits, draft_tokens, temps, B, K, L, V, dtype, 0,
+                         seed, step, out_accept_len, out_tokens, out_draft_index, workspace,
+                         workspace_bytes, stream);
+}
+
+int spec_verify_multidraft_rows(const void* target_logits, const void* draft_logits,
+                                const int32_t* draft_tokens, const float* temps, int B, int K,
+                                int L, int V, int dtype, uint64_t seed, uint64_t step,
+                                int32_t* out_accept_len, int32_t* out_tokens,
+                                int32_t* out_draft_index, void* workspace, size_t workspace_bytes,
+                                void* stream) {
+  return multidraft_call(target_logits, draft_logits, draft_tokens, temps, B, K, L, V, dtype, 1,
+                         seed, step, out_accept_len, out_tokens, out_draft_index, workspace,
+                         workspace_bytes, stream);
 }
 
 // ------------------------------------------------------------- host buffers
@@ -235,11 +253,13 @@ size_t spec_verify_host_staging_size(int B, int gamma, int V, int dtype) {
   return host_layout(B, gamma, V, dtype).total;
 }
 
-int spec_verify_host(const void* target_logits, const void* draft_logits,
-                     const int32_t* draft_tokens, const float* temps, int B, int gamma, int V,
-                     int dtype, uint64_t seed, uint64_t step, int32_t* out_accept_len,
-                     int32_t* out_tokens, float* out_target_logp, float* out_draft_logp,
-                     void* staging, size_t staging_bytes, void* stream) {
+// The host-buffer path without the final synchronisation: copies in, the
+// verification, copies out, all enqueued on `stream`.
+static int host_enqueue(const void* target_logits, const void* draft_logits,
+                        const int32_t* draft_tokens, const float* temps, int B, int gamma, int V,
+                        int dtype, uint64_t seed, uint64_t step, int32_t* out_accept_len,
+                        int32_t* out_tokens, float* out_target_logp, float* out_draft_logp,
+                        void* staging, size_t staging_bytes, cudaStream_t s) {
   if (B < 0 || !sizes_ok(B, gamma, V, dtype))
     return check_common(target_logits, draft_logits, draft_tokens, temps, B, gamma, V, dtype, step,
                         out_accept_len, out_tokens, staging, staging_bytes, 0);
@@ -254,7 +274,6 @@ int spec_verify_host(const void* target_logits, const void* draft_logits,
   if (step >> 32) return set_error(SV_ERR_INVALID_ARG, "step must be < 2^32");
   int rc = check_device();
   if (rc != SV_OK) return rc;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
   char* st = static_cast<char*>(staging);
   const size_t es = dtype == SV_BF16 ? 2 : 4;
   const size_t nt = static_cast<size_t>(B) * (gamma + 1) * static_cast<size_t>(V) * es;
@@ -281,9 +300,34 @@ int spec_verify_host(const void* target_logits, const void* draft_logits,
     e = cudaMemcpyAsync(out_target_logp, st + h.lp, nx, cudaMemcpyDeviceToHost, s);
   if (e == cudaSuccess && out_draft_logp)
     e = cudaMemcpyAsync(out_draft_logp, st + h.lq, nx, cudaMemcpyDeviceToHost, s);
-  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   if (e != cudaSuccess) return set_error(SV_ERR_CUDA, "device->host copy: %s", cudaGetErrorString(e));
   return SV_OK;
+}
+
+int spec_verify_host(const void* target_logits, const void* draft_logits,
+                     const int32_t* draft_tokens, const float* temps, int B, int gamma, int V,
+                     int dtype, uint64_t seed, uint64_t step, int32_t* out_accept_len,
+                     int32_t* out_tokens, float* out_target_logp, float* out_draft_logp,
+                     void* staging, size_t staging_bytes, void* stream) {
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int rc = host_enqueue(target_logits, draft_logits, draft_tokens, temps, B, gamma, V, dtype,
+                              seed, step, out_accept_len, out_tokens, out_target_logp,
+                              out_draft_logp, staging, staging_bytes, s);
+  if (rc != SV_OK || B == 0) return rc;
+  const cudaError_t e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return set_error(SV_ERR_CUDA, "device->host copy: %s", cudaGetErrorString(e));
+  return SV_OK;
+}
+
+int spec_verify_host_async(const void* target_logits, const void* draft_logits,
+                           const int32_t* draft_tokens, const float* temps, int B, int gamma,
+                           int V, int dtype, uint64_t seed, uint64_t step,
+                           int32_t* out_accept_len, int32_t* out_tokens, float* out_target_logp,
+                           float* out_draft_logp, void* staging, size_t staging_bytes,
+                           void* stream) {
+  return host_enqueue(target_logits, draft_logits, draft_tokens, temps, B, gamma, V, dtype, seed,
+                      step, out_accept_len, out_tokens, out_target_logp, out_draft_logp, staging,
+                      staging_bytes, static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

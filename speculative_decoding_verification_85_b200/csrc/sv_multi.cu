@@ -1,40 +1,117 @@
 // sv_multi.cu -- multi-draft verification, "SpecTr-GBV: Multi-Draft Block
 // Verification Accelerating Speculative Decoding", Methodology, Algorithm 1.
 //
-// Pass 1 is the single-draft row pass (sv_rows.cuh) over the L+1 target and
-// L draft rows of each sequence; its last CTA per sequence publishes the
-// combined row statistics.  The sequential part -- drafts visited in order,
-// sub-block weights w, acceptance h = A / (A + 1 - w) with
-// A = sum_v max(w P_{i+1}(v) - Q_{i+1}(v), 0), the residual law R at tau and
-// the rejected set H -- runs in one CTA per sequence; every V-wide quantity
-// (A, the residual update, the final race) is a block reduction.
+// One thread-block cluster of kMdC CTAs per sequence; CTA `rank` owns the
+// vocabulary slice [rank * slice, (rank + 1) * slice).  Every V-wide quantity
+// of the algorithm is a sum (or a race) over the slices: each CTA reduces its
+// slice, writes its partial into every CTA's exchange buffer through
+// distributed shared memory, and after one cluster barrier every CTA adds the
+// kMdC partials in rank order -- so every CTA holds the same value and takes
+// the same decisions, with no further communication.  The steps:
+//   1. row statistics (maximum, softmax sum, first argmax) of the L + 1 target
+//      and L draft rows (one exchange);
+//   2. the residual law R = P_0 and its sum (one exchange);
+//   3. per draft k, in index order: the sub-block weights w_i (scalars), all
+//      sums A_i = sum_v max(w_i P_{i+1}(v) - Q_{i+1}(v), 0) of the draft in one
+//      pass (one exchange), the acceptance coins h_i = A_i / (A_i + 1 - w_i)
+//      (h_{L-1} = w_{L-1}) with the longest accepted sub-block kept, then the
+//      update of R -- on an advance R <- norm(max(w P_tau - Q_tau, 0)), on a
+//      rejection R <- norm(max(R - Q~, 0)) with Q~ the draft law at tau
+//      conditioned on not being in the rejected set H (one exchange);
+//   4. the correction token: an exponential race over R at tau, or over P_L
+//      when the whole block was accepted (one exchange).
+// When a slice's rows and R fit in shared memory they are staged there once
+// (bulk copies); otherwise every pass reads them from global memory.
 //
 // Reading of the unprinted equations (as in the CPU definition): greedy
 // block-verification weights; the longest accepted sub-block wins; on a
-// rejection the draft law at tau is conditioned on not being in H and
-// R <- norm(max(R - Q~, 0)); on an advance R <- norm(max(w P_tau - Q_tau, 0)).
-// A token in H has R = 0 after its rejection, so the residual update needs
-// no membership test; H only decides which later drafts are skipped.
+// rejection the draft law at tau is conditioned on not being in H.  A token in
+// H has R = 0 after its rejection, so the residual update needs no membership
+// test; H only decides which later drafts are skipped.
+#include <cooperative_groups.h>
+
+#include <atomic>
 #include <climits>
 
 #include "sv_device.cuh"
 #include "sv_internal.h"
 #include "sv_rows.cuh"
 
+namespace cg = cooperative_groups;
+
 namespace sv {
 
-template <bool kBf16>
-__global__ void __launch_bounds__(kP1Threads) pass1_multi_kernel(Pass1Params p) {
-  __shared__ RowAcc rows[kMaxRowsPerSeq];
-  const int item = blockIdx.x;
-  const int rowg = item / p.nc;
-  const int chunk = item - rowg * p.nc;
-  const int b = rowg / p.rps;
-  const int r = rowg - b * p.rps;
-  if (!pass1_chunk<kBf16>(p, b, r, chunk)) return;
-  combine_rows<kP1Threads>(p, b, rows);
-  for (int q = threadIdx.x; q < p.rps; q += kP1Threads)
-    store_partial(p.rowstat + static_cast<size_t>(b) * p.rps + q, rows[q]);
+constexpr int kMdC = 8;                          // CTAs per cluster (one sequence)
+constexpr int kMdT = 256;                        // threads per CTA
+constexpr int kMdW = kMdT / 32;
+constexpr int kXBatch = 128;                     // row statistics per exchange
+constexpr int kXSlot = 2 * kXBatch;              // doubles per rank in an exchange buffer
+constexpr int kMaxStatRows = 256;                // row statistics per sequence (all row sets)
+constexpr int kMaxDraftTokens = SV_MAX_DRAFTS * SV_MAX_GAMMA;
+static_assert(SV_MAX_GAMMA <= kXSlot, "an exchange carries every A_i of a draft");
+
+struct MdcParams {
+  const void* target;  // [B][nsets][L + 1][V]
+  const void* draft;   // [B][nsets][L][V]
+  const int32_t* tokens;
+  const float* temps;
+  int B, K, L, V;
+  int per_draft;    // 1: a row set per draft (nsets = K); 0: one shared set
+  uint64_t seed;
+  uint32_t step;
+  int slice;        // vocabulary entries per CTA (a multiple of 8)
+  int rowstride;    // bytes per staged row slice in shared memory (local variant)
+  float* Rws;       // [B][2][V] residual laws in global memory (global variant)
+  int32_t* accept_len;
+  int32_t* out_tokens;
+  int32_t* out_draft_index;
+};
+
+// Fixed part of the dynamic shared memory (the local variant adds the R
+// buffers and the staged rows after it).
+struct alignas(16) MdSmem {
+  double xb[2][kMdC][kXSlot];          // exchange buffers (written by every rank)
+  float4 wpart[kMdW][kXBatch];         // per-warp row statistics of a batch
+  double wred[kMdW][SV_MAX_GAMMA];     // per-warp partial sums
+  double res[kXSlot];                  // results of the last exchange
+  float m[kMaxStatRows];               // row maxima
+  float is[kMaxStatRows];              // 1 / s, s = sum_v 2^{(z_v - m) c}
+  int arg[kMaxStatRows];               // first argmax (greedy target rows)
+  double w[SV_MAX_GAMMA];              // the current draft's sub-block weights
+  int tok[kMaxDraftTokens];            // draft tokens [K][L]
+  float2 zg[kMaxDraftTokens];          // target / draft logit at each draft token
+  int H[SV_MAX_DRAFTS];                // rejected tokens at tau
+  float4 race[kMdW];
+  uint64_t bar;                        // staging barrier
+  double Rn, qH, keep, wbest;
+  int tau, a, nH, skip, best, rcur;
+};
+
+constexpr size_t kMdFixed = (sizeof(MdSmem) + 127) / 128 * 128;
+
+// The kMdC partials of an exchange, in rank order: thread t < nv contributes
+// `mine` as slot t of buffer `buf` to every CTA; after the cluster barrier
+// thread t adds slot t over the ranks into sm.res[t]; ends with a CTA barrier.
+template <typename Cl>
+__device__ __forceinline__ void exchange(Cl& cl, MdSmem& sm, int buf, int nv, double mine) {
+  const int tid = threadIdx.x;
+  const int rank = static_cast<int>(cl.block_rank());
+  if (tid < nv)
+    for (int q = 0; q < kMdC; ++q) *cl.map_shared_rank(&sm.xb[buf][rank][tid], q) = mine;
+  cl.sync();
+  if (tid < nv) {
+    double s = 0.0;
+    for (int q = 0; q < kMdC; ++q) s += sm.xb[buf][q][tid];
+    sm.res[tid] = s;
+  }
+  __syncthreads();
+}
+
+// One value slot v of a CTA-wide sum: each warp's total lands in sm.wred[warp][v].
+__device__ __forceinline__ void warp_sum_to(MdSmem& sm, int v, double x) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) x += __shfl_down_sync(0xffffffffu, x, off);
+  if ((threadIdx.x & 31) == 0) sm.wred[threadIdx.x >> 5][v] = x;
 }
 
 __device__ __forceinline__ double step_weight(double w, double num, double den) {
@@ -45,303 +122,595 @@ __device__ __forceinline__ double step_weight(double w, double num, double den) 
   return (w > 0.0 && num > 0.0) ? 1.0 : 0.0;
 }
 
-template <bool kBf16>
-__global__ void __launch_bounds__(kMdThreads) md_gbv_kernel(MdParams p) {
+template <bool kBf16, bool kLocal>
+__global__ void __launch_bounds__(kMdT) md_cluster_kernel(const __grid_constant__ MdcParams p) {
   constexpr size_t es = kBf16 ? 2 : 4;
-  __shared__ float s_mt[kMaxRowsPerSeq];  // raw row maximum m
-  __shared__ float s_is[kMaxRowsPerSeq];  // 1 / s, s = sum_v 2^{(z_v - m) c}
-  __shared__ int s_arg[kMaxRowsPerSeq];
-  __shared__ int s_x[SV_MAX_DRAFTS * SV_MAX_GAMMA];
-  __shared__ int s_H[SV_MAX_DRAFTS];
-  __shared__ double s_red[33];
-  __shared__ float4 s_race[kMdThreads / 32];
-  __shared__ int s_tau, s_a, s_nH, s_skip, s_best;
-  __shared__ double s_qH, s_Rn, s_w, s_wbest, s_keep, s_qfirst;
-
-  const int b = blockIdx.x;
-  const int tid = threadIdx.x;
+  extern __shared__ __align__(128) char dyn[];
+  MdSmem& sm = *reinterpret_cast<MdSmem*>(dyn);
+  cg::cluster_group cl = cg::this_cluster();
+  const int rank = static_cast<int>(cl.block_rank());
+  const int b = blockIdx.x / kMdC;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int K = p.K, L = p.L, V = p.V, rps = 2 * L + 1;
+  const int nsets = p.per_draft ? K : 1;
+  const int v0 = rank * p.slice;
+  const int n = max(0, min(V - v0, p.slice));  // entries of this slice
   const float T = __ldg(p.temps + b);
-  const char* tgt = static_cast<const char*>(p.target) +
-                    static_cast<size_t>(b) * (L + 1) * static_cast<size_t>(V) * es;
-  const char* drf = static_cast<const char*>(p.draft) +
-                    static_cast<size_t>(b) * L * static_cast<size_t>(V) * es;
-  const size_t rowb = static_cast<size_t>(V) * es;
-  float* R = p.R + static_cast<size_t>(b) * V;
-  int32_t* tok = p.out_tokens + static_cast<size_t>(b) * (L + 1);
-
   const bool tvalid = (T >= 0.0f) && !isinf(T);
   const bool greedy = tvalid && T == 0.0f;
-  bool ok = tvalid;
-  for (int r = tid; r < rps; r += kMdThreads) {
-    const RowAcc a = load_partial(p.rowstat + static_cast<size_t>(b) * rps + r);
-    s_arg[r] = a.arg;
-    s_mt[r] = 0.0f;
-    s_is[r] = 0.0f;
-    const bool needed = tvalid && (!greedy || r <= L);
-    if (needed) {
-      bool rv = !a.bad && isfinite(a.m);
-      if (!greedy) {
-        s_mt[r] = a.m;
-        s_is[r] = 1.0f / a.s;
-        rv = rv && isfinite(__fdiv_rn(a.m, T));
-      }
-      ok = ok && rv;
+  // the rows a sequence needs, numbered q = set * nrows + r: per row set the
+  // target rows 0..L, then (softmax rows only) the draft rows 0..L-1 as r = L+1..2L
+  const int nrows = greedy ? L + 1 : rps;
+  const int nq = nsets * nrows;
+  const size_t rowb = static_cast<size_t>(V) * es;
+  const char* tgt = static_cast<const char*>(p.target) + static_cast<size_t>(b) * nsets * (L + 1) * rowb;
+  const char* drf = static_cast<const char*>(p.draft) + static_cast<size_t>(b) * nsets * L * rowb;
+  auto grow = [&](int q) -> const char* {  // global row q
+    const int set = q / nrows, r = q - set * nrows;
+    return r <= L ? tgt + (static_cast<size_t>(set) * (L + 1) + r) * rowb
+                  : drf + (static_cast<size_t>(set) * L + (r - L - 1)) * rowb;
+  };
+  auto qt = [&](int set, int i) { return set * nrows + i; };          // target row i of a set
+  auto qd = [&](int set, int i) { return set * nrows + L + 1 + i; };  // draft row i of a set
+  float* Rb[2];
+  char* srows = nullptr;
+  if constexpr (kLocal) {
+    Rb[0] = reinterpret_cast<float*>(dyn + kMdFixed);
+    Rb[1] = Rb[0] + p.slice;
+    srows = dyn + kMdFixed + 2 * static_cast<size_t>(p.slice) * sizeof(float);
+  } else {
+    Rb[0] = p.Rws + static_cast<size_t>(b) * 2 * V + v0;
+    Rb[1] = Rb[0] + V;
+  }
+  // logit e (0 <= e < n) of row q of this slice
+  auto zrow = [&](int q, int e) -> float {
+    if constexpr (kLocal) {
+      const char* sp = srows + static_cast<size_t>(q) * p.rowstride +
+                       (reinterpret_cast<uintptr_t>(grow(q) + static_cast<size_t>(v0) * es) & 15u);
+      if constexpr (kBf16)
+        return __uint_as_float(static_cast<uint32_t>(reinterpret_cast<const uint16_t*>(sp)[e]) << 16);
+      else
+        return reinterpret_cast<const float*>(sp)[e];
+    } else {
+      return logit_at<kBf16>(grow(q), static_cast<int64_t>(v0) + e);
     }
-  }
-  for (int n = tid; n < K * L; n += kMdThreads) {
-    const int xv = __ldg(p.tokens + static_cast<size_t>(b) * K * L + n);
-    s_x[n] = xv;
-    ok = ok && xv >= 0 && xv < V;
-  }
-  ok = __syncthreads_and(ok);
-  if (!ok) {
-    for (int i = tid; i <= L; i += kMdThreads) tok[i] = -1;
-    if (tid == 0) {
-      p.accept_len[b] = -1;
-      if (p.out_draft_index) p.out_draft_index[b] = -1;
-    }
-    return;
-  }
+  };
 
+  // ---- draft tokens and their logits; staging of the slice's rows
+  bool stage_ok = true;
+  if (tid == 0) {
+    mbar_init(&sm.bar, 1);
+    mbar_init_fence();
+  }
+  __syncthreads();
+  for (int t = tid; t < K * L; t += kMdT) {
+    const int x = __ldg(p.tokens + static_cast<size_t>(b) * K * L + t);
+    const int k = t / L, i = t - k * L, set = p.per_draft ? k : 0;
+    sm.tok[t] = x;
+    float2 z = make_float2(__int_as_float(0x7fc00000), __int_as_float(0x7fc00000));
+    if (tvalid && !greedy && x >= 0 && x < V) {
+      z.x = logit_at<kBf16>(grow(qt(set, i)), x);
+      z.y = logit_at<kBf16>(grow(qd(set, i)), x);
+    }
+    sm.zg[t] = z;
+  }
+  if constexpr (kLocal) {
+    if (tvalid) {
+      // rows start at the same offset modulo 16 in shared and in global memory,
+      // so the aligned body of each row slice is one bulk copy
+      if (tid == 0) {
+        uint32_t total = 0;
+        for (int q = 0; q < nq; ++q) {
+          const uintptr_t ga = reinterpret_cast<uintptr_t>(grow(q) + static_cast<size_t>(v0) * es);
+          const uint32_t hb = min(static_cast<uint32_t>((16u - (ga & 15u)) & 15u), static_cast<uint32_t>(n * es));
+          total += (static_cast<uint32_t>(n * es) - hb) / 16u * 16u;
+        }
+        if (total) {
+          mbar_arrive_expect_tx(&sm.bar, total);
+          for (int q = 0; q < nq; ++q) {
+            const char* g = grow(q) + static_cast<size_t>(v0) * es;
+            const uintptr_t ga = reinterpret_cast<uintptr_t>(g);
+            const uint32_t hb = min(static_cast<uint32_t>((16u - (ga & 15u)) & 15u), static_cast<uint32_t>(n * es));
+            const uint32_t body = (static_cast<uint32_t>(n * es) - hb) / 16u * 16u;
+            char* sdst = srows + static_cast<size_t>(q) * p.rowstride + (ga & 15u);
+            if (body) bulk_g2s(sdst + hb, g + hb, body, &sm.bar);
+          }
+        } else {
+          mbar_arrive(&sm.bar);
+        }
+      }
+      // the unaligned head and tail of each row slice, as scalars
+      for (int q = 0; q < nq; ++q) {
+        const char* g = grow(q) + static_cast<size_t>(v0) * es;
+        const uintptr_t ga = reinterpret_cast<uintptr_t>(g);
+        const int hb = min(static_cast<int>((16u - (ga & 15u)) & 15u), static_cast<int>(n * es));
+        const int body = (static_cast<int>(n * es) - hb) / 16 * 16;
+        char* sdst = srows + static_cast<size_t>(q) * p.rowstride + (ga & 15u);
+        const int h = hb / static_cast<int>(es), t0 = (hb + body) / static_cast<int>(es);
+        for (int e = tid; e < h; e += kMdT) memcpy(sdst + e * es, g + e * es, es);
+        for (int e = t0 + tid; e < n; e += kMdT) memcpy(sdst + e * es, g + e * es, es);
+      }
+      // if the copies never completed, the slice's rows count as bad (NaN)
+      // and the whole sequence is reported invalid
+      stage_ok = mbar_wait(&sm.bar, 0);
+    }
+  }
+  __syncthreads();
+
+  // ---- 1. row statistics: slice partials, one exchange per batch of rows,
+  // merged in rank order
+  int buf = 0;
+  bool row_ok = true;
+  {
+    const float c = tvalid && !greedy ? __fdiv_rn(kLog2e, T) : 0.0f;
+    for (int q0 = 0; q0 < nq; q0 += kXBatch) {
+      const int nb = min(kXBatch, nq - q0);
+      for (int j = 0; j < nb; ++j) {
+        RowAcc a{-INFINITY, 0.0f, 0x7fffffff, stage_ok ? 0 : 1};
+        if (tvalid)
+          for (int e = tid; e < n; e += kMdT) {
+            const float z = zrow(q0 + j, e);
+            if (greedy) acc_scalar<kRowArgmax>(a, z, v0 + e, c); else acc_scalar<kRowLse>(a, z, v0 + e, c);
+          }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+          RowAcc o;
+          o.m = __shfl_down_sync(0xffffffffu, a.m, off);
+          o.s = __shfl_down_sync(0xffffffffu, a.s, off);
+          o.arg = __shfl_down_sync(0xffffffffu, a.arg, off);
+          o.bad = __shfl_down_sync(0xffffffffu, a.bad, off);
+          if (greedy) acc_merge<kRowArgmax>(a, o, c); else acc_merge<kRowLse>(a, o, c);
+        }
+        if (lane == 0) sm.wpart[warp][j] = make_float4(a.m, a.s, __int_as_float(a.arg), __int_as_float(a.bad));
+      }
+      __syncthreads();
+      if (tid < nb) {
+        RowAcc a{-INFINITY, 0.0f, 0x7fffffff, 0};
+        for (int w = 0; w < kMdW; ++w) {
+          const float4 x = sm.wpart[w][tid];
+          const RowAcc o{x.x, x.y, __float_as_int(x.z), __float_as_int(x.w)};
+          if (greedy) acc_merge<kRowArgmax>(a, o, c); else acc_merge<kRowLse>(a, o, c);
+        }
+        const float4 v = make_float4(a.m, a.s, __int_as_float(a.arg), __int_as_float(a.bad));
+        for (int r = 0; r < kMdC; ++r)
+          *reinterpret_cast<float4*>(cl.map_shared_rank(&sm.xb[buf][rank][2 * tid], r)) = v;
+      }
+      cl.sync();
+      if (tid < nb) {
+        RowAcc a{-INFINITY, 0.0f, 0x7fffffff, 0};
+        for (int r = 0; r < kMdC; ++r) {
+          const float4 x = *reinterpret_cast<const float4*>(&sm.xb[buf][r][2 * tid]);
+          const RowAcc o{x.x, x.y, __float_as_int(x.z), __float_as_int(x.w)};
+          if (greedy) acc_merge<kRowArgmax>(a, o, c); else acc_merge<kRowLse>(a, o, c);
+        }
+        const int q = q0 + tid;
+        sm.m[q] = a.m;
+        sm.is[q] = greedy ? 0.0f : 1.0f / a.s;
+        sm.arg[q] = a.arg;
+        bool rv = !a.bad && isfinite(a.m);
+        if (!greedy) rv = rv && isfinite(__fdiv_rn(a.m, T));
+        row_ok = row_ok && rv;
+      }
+      buf ^= 1;
+      __syncthreads();  // wpart is reused by the next batch
+    }
+  }
+  // validity: temperature, rows, tokens (the same in every CTA of the cluster)
+  bool ok = tvalid && row_ok;
+  for (int t = tid; t < K * L; t += kMdT) ok = ok && sm.tok[t] >= 0 && sm.tok[t] < V;
+  ok = __syncthreads_and(ok);
+  int32_t* tok = p.out_tokens + static_cast<size_t>(b) * (L + 1);
+  if (!ok) {
+    if (rank == 0) {
+      for (int i = tid; i <= L; i += kMdT) tok[i] = -1;
+      if (tid == 0) {
+        p.accept_len[b] = -1;
+        if (p.out_draft_index) p.out_draft_index[b] = -1;
+      }
+    }
+    return;  // every CTA returns here: no one touches another CTA's memory any more
+  }
   if (greedy) {
-    if (tid == 0) {
+    // the accepted block is the longest draft prefix that matches the target
+    // argmaxes of its row set (first draft on ties); the correction is the
+    // argmax at tau of the accepted draft's rows (of row set 0 when nothing
+    // was accepted: every draft shares the empty prefix)
+    if (rank == 0 && tid == 0) {
       int tau = 0, a = -1;
       for (int k = 0; k < K; ++k) {
-        int n = 0;
-        while (n < L && s_x[k * L + n] == s_arg[n]) ++n;
-        if (n > tau) {
-          tau = n;
+        const int set = p.per_draft ? k : 0;
+        int m = 0;
+        while (m < L && sm.tok[k * L + m] == sm.arg[qt(set, m)]) ++m;
+        if (m > tau) {
+          tau = m;
           a = k;
         }
       }
-      for (int i = 0; i <= L; ++i) tok[i] = i < tau ? s_x[a * L + i] : (i == tau ? s_arg[tau] : -1);
+      const int sa = p.per_draft && a >= 0 ? a : 0;
+      for (int i = 0; i <= L; ++i)
+        tok[i] = i < tau ? sm.tok[a * L + i] : (i == tau ? sm.arg[qt(sa, tau)] : -1);
       p.accept_len[b] = tau;
       if (p.out_draft_index) p.out_draft_index[b] = a;
     }
     return;
   }
 
-  // P_r(v) and Q_r(v): p = 2^{(z - m) c} / s with c = log2(e) / T, the same
-  // MUFU exponential that built the row sums s (so each law sums to 1 to
-  // within the exponential's 2^-22 relative error), one subtraction, one
-  // multiply, one ex2 and one multiply per value.
+  // P and Q of row q at entry e: 2^{(z - m_q) c} / s_q with c = log2(e) / T, the
+  // same MUFU exponential that built the row sums (each law sums to 1 to
+  // within its 2^-22 relative error); one subtraction, one multiply, one ex2
+  // and one multiply per value.
   const float cc = __fdiv_rn(kLog2e, T);
-  auto prob_t = [&](int r, int v) -> float {
-    return ex2_approx((logit_at<kBf16>(tgt + r * rowb, v) - s_mt[r]) * cc) * s_is[r];
-  };
-  auto prob_d = [&](int r, int v) -> float {
-    return ex2_approx((logit_at<kBf16>(drf + r * rowb, v) - s_mt[L + 1 + r]) * cc) * s_is[L + 1 + r];
+  auto prob = [&](int q, int e) -> float { return ex2_approx((zrow(q, e) - sm.m[q]) * cc) * sm.is[q]; };
+  auto prob_x = [&](int q, float z) -> float { return ex2_approx((z - sm.m[q]) * cc) * sm.is[q]; };
+  auto exch1 = [&](double x) {  // one value: CTA sum, then cluster sum into sm.res[0]
+    warp_sum_to(sm, 0, x);
+    __syncthreads();
+    double loc = 0.0;
+    if (tid == 0)
+      for (int w = 0; w < kMdW; ++w) loc += sm.wred[w][0];
+    exchange(cl, sm, buf, 1, loc);
+    buf ^= 1;
   };
 
-  // R <- P_0
+  // ---- 2. R <- P_0 (row set 0: every draft shares the empty prefix)
   {
     double loc = 0.0;
-    for (int v = tid; v < V; v += kMdThreads) {
-      const float pv = prob_t(0, v);
-      R[v] = pv;
+    for (int e = tid; e < n; e += kMdT) {
+      const float pv = prob(qt(0, 0), e);
+      Rb[0][e] = pv;
       loc += pv;
     }
-    const double tot = block_sum<kMdThreads>(loc, s_red);
+    exch1(loc);
     if (tid == 0) {
-      s_Rn = tot;
-      s_tau = 0;
-      s_a = -1;
-      s_nH = 0;
-      s_qH = 0.0;
+      sm.Rn = sm.res[0];
+      sm.tau = 0;
+      sm.a = -1;
+      sm.nH = 0;
+      sm.qH = 0.0;
+      sm.rcur = 0;
     }
+    __syncthreads();
   }
-  __syncthreads();
 
+  // ---- 3. the drafts in index order
   for (int k = 0; k < K; ++k) {
-    __syncthreads();  // every thread is done with the previous draft's shared state
+    const int set = p.per_draft ? k : 0;
     if (tid == 0) {
-      const int tau = s_tau;
+      const int tau = sm.tau;
       int skip = tau == L ? 2 : 0;
-      const int* x = s_x + k * L;
+      const int* x = sm.tok + k * L;
       if (!skip && tau > 0) {
-        const int* xa = s_x + s_a * L;
+        const int* xa = sm.tok + sm.a * L;
         for (int i = 0; i < tau; ++i)
           if (x[i] != xa[i]) skip = 1;
       }
       if (!skip)
-        for (int h = 0; h < s_nH; ++h)
-          if (s_H[h] == x[tau]) skip = 1;
-      s_skip = skip;
+        for (int h = 0; h < sm.nH; ++h)
+          if (sm.H[h] == x[tau]) skip = 1;
+      sm.skip = skip;
       if (!skip) {
-        const double keep = 1.0 - s_qH;
-        s_keep = keep;
-        s_qfirst = keep > 0.0 ? static_cast<double>(prob_d(tau, x[tau])) / keep : 0.0;
-        s_w = 1.0;
-        s_wbest = 1.0;
-        s_best = tau;
+        const double keep = 1.0 - sm.qH;
+        sm.keep = keep;
+        const double qfirst = keep > 0.0 ? static_cast<double>(prob_x(qd(set, tau), sm.zg[k * L + tau].y)) / keep : 0.0;
+        // R at the draft's token: read from the CTA that owns that entry
+        const int xt = x[tau], owner = xt / p.slice, eo = xt - owner * p.slice;
+        float rx;
+        if constexpr (kLocal) {
+          const float* Rl = reinterpret_cast<const float*>(dyn + kMdFixed) + sm.rcur * p.slice;
+          rx = cl.map_shared_rank(Rl, owner)[eo];
+        } else {
+          rx = p.Rws[static_cast<size_t>(b) * 2 * V + static_cast<size_t>(sm.rcur) * V + xt];
+          (void)eo;
+        }
+        double w = 1.0;
+        for (int i = tau; i < L; ++i) {
+          double num, den;
+          if (i == tau) {
+            num = static_cast<double>(rx) / sm.Rn;
+            den = qfirst;
+          } else {
+            num = prob_x(qt(set, i), sm.zg[k * L + i].x);
+            den = prob_x(qd(set, i), sm.zg[k * L + i].y);
+          }
+          w = step_weight(w, num, den);
+          sm.w[i] = w;
+        }
       }
     }
     __syncthreads();
-    if (s_skip == 2) break;
-    if (s_skip) continue;
-    const int tau = s_tau;
-    const int* x = s_x + k * L;
-    for (int i = tau; i < L; ++i) {
-      if (tid == 0) {
-        double num, den;
-        if (i == tau) {
-          num = static_cast<double>(R[x[i]]) / s_Rn;
-          den = s_qfirst;
+    if (sm.skip == 2) break;
+    if (sm.skip) continue;
+    const int tau = sm.tau;
+    const int* x = sm.tok + k * L;
+    // all of the draft's sums A_i, i = tau .. L-2, in one pass (at least one
+    // exchange, which also orders the R reads above before any R update)
+    const int nA = max(L - 1 - tau, 0);
+    for (int i = tau; i < L - 1; ++i) {
+      const float wf = static_cast<float>(sm.w[i]);
+      double loc = 0.0;
+      for (int e = tid; e < n; e += kMdT) {
+        const float t = wf * prob(qt(set, i + 1), e) - prob(qd(set, i + 1), e);
+        if (t > 0.0f) loc += t;
+      }
+      warp_sum_to(sm, i - tau, loc);
+    }
+    __syncthreads();
+    {
+      double loc = 0.0;
+      if (tid < nA)
+        for (int w = 0; w < kMdW; ++w) loc += sm.wred[w][tid];
+      exchange(cl, sm, buf, max(nA, 1), loc);
+      buf ^= 1;
+    }
+    if (tid == 0) {
+      int best = tau;
+      double wbest = 1.0;
+      for (int i = tau; i < L; ++i) {
+        const double w = sm.w[i];
+        double h;
+        if (i < L - 1) {
+          const double A = sm.res[i - tau];
+          const double den = A + 1.0 - w;
+          h = den == 0.0 ? 1.0 : A / den;
         } else {
-          num = prob_t(i, x[i]);
-          den = prob_d(i, x[i]);
+          h = w;
         }
-        s_w = step_weight(s_w, num, den);
-      }
-      __syncthreads();
-      const double w = s_w;
-      double h;
-      if (i < L - 1) {
-        const float wf = static_cast<float>(w);
-        double loc = 0.0;
-        for (int v = tid; v < V; v += kMdThreads) {
-          const float t = wf * prob_t(i + 1, v) - prob_d(i + 1, v);
-          if (t > 0.0f) loc += t;
-        }
-        const double A = block_sum<kMdThreads>(loc, s_red);
-        const double den = A + 1.0 - w;
-        h = den == 0.0 ? 1.0 : A / den;
-      } else {
-        h = w;
-      }
-      if (tid == 0) {
         const uint4 rnd = keyed_block(p.seed, p.step, kTagMdEta, b, k, i, i);
         if (accept_uniform(rnd.x) < h) {
-          s_best = i + 1;
-          s_wbest = w;
+          best = i + 1;
+          wbest = w;
         }
       }
-      __syncthreads();
+      sm.best = best;
+      sm.wbest = wbest;
     }
-    const int best = s_best;
     __syncthreads();
+    const int best = sm.best;
+    const int rc = sm.rcur;
+    float* Rcur = Rb[rc];
+    float* Rnew = Rb[rc ^ 1];
     if (best > tau) {
       if (best < L) {
-        const float wb = static_cast<float>(s_wbest);
+        const float wb = static_cast<float>(sm.wbest);
         double loc = 0.0;
-        for (int v = tid; v < V; v += kMdThreads) {
-          const float t = wb * prob_t(best, v) - prob_d(best, v);
+        for (int e = tid; e < n; e += kMdT) {
+          const float t = wb * prob(qt(set, best), e) - prob(qd(set, best), e);
           const float rv = t > 0.0f ? t : 0.0f;
-          R[v] = rv;
+          Rnew[e] = rv;
           loc += rv;
         }
-        const double tot = block_sum<kMdThreads>(loc, s_red);
-        if (tid == 0) s_Rn = tot;
+        exch1(loc);
+        if (sm.res[0] > 0.0) {
+          if (tid == 0) sm.Rn = sm.res[0];
+        } else {
+          // the residual vanished: the correction law is P_tau itself
+          double l2 = 0.0;
+          for (int e = tid; e < n; e += kMdT) {
+            const float pv = prob(qt(set, best), e);
+            Rnew[e] = pv;
+            l2 += pv;
+          }
+          exch1(l2);
+          if (tid == 0) sm.Rn = sm.res[0];
+        }
+        if (tid == 0) sm.rcur = rc ^ 1;
       }
       if (tid == 0) {
-        s_tau = best;
-        s_a = k;
-        s_nH = 0;
-        s_qH = 0.0;
+        sm.tau = best;
+        sm.a = k;
+        sm.nH = 0;
+        sm.qH = 0.0;
       }
     } else {
-      const float inv_rn = static_cast<float>(1.0 / s_Rn);
-      const double keep = s_keep;
+      const float inv_rn = static_cast<float>(1.0 / sm.Rn);
+      const double keep = sm.keep;
       const float inv_keep = keep > 0.0 ? static_cast<float>(1.0 / keep) : 0.0f;
       double loc = 0.0;
-      for (int v = tid; v < V; v += kMdThreads) {
-        const float t = R[v] * inv_rn - prob_d(tau, v) * inv_keep;
+      for (int e = tid; e < n; e += kMdT) {
+        const float t = Rcur[e] * inv_rn - prob(qd(set, tau), e) * inv_keep;
         const float rv = t > 0.0f ? t : 0.0f;
-        R[v] = rv;
+        Rnew[e] = rv;
         loc += rv;
       }
-      const double tot = block_sum<kMdThreads>(loc, s_red);
+      exch1(loc);
       if (tid == 0) {
-        s_Rn = tot;  // tot > 0 whenever a draft is rejected at tau (its token had R < Q~)
-        s_H[s_nH++] = x[tau];
-        s_qH += static_cast<double>(prob_d(tau, x[tau]));
+        if (sm.res[0] > 0.0) {  // else R stays as it was (a vanished update changes nothing)
+          sm.Rn = sm.res[0];
+          sm.rcur = rc ^ 1;
+        }
+        sm.H[sm.nH++] = x[tau];
+        sm.qH += static_cast<double>(prob_x(qd(set, tau), sm.zg[k * L + tau].y));
       }
     }
     __syncthreads();
   }
 
-  // Correction token: race over P_L (whole block accepted) or over R at tau.
-  const int tau = s_tau;
+  // ---- 4. correction token: race over P_L of the accepted draft's rows
+  // (whole block accepted) or over R at tau
+  const int tau = sm.tau;
+  const int sa = p.per_draft && sm.a >= 0 ? sm.a : 0;
+  const float* Rf = Rb[sm.rcur];
   float bw = 0.0f, be = 1.0f;
   int bi = INT_MAX;
-  const int nblk = (V + 3) / 4;
-  for (int gi = tid; gi < nblk; gi += kMdThreads) {
-    const uint4 rnd = keyed_block(p.seed, p.step, kTagMdGumbel, b, 0, tau, gi);
+  const int g0 = v0 >> 2, g1 = (v0 + n + 3) >> 2;  // Philox blocks of the slice (v0 % 8 == 0)
+  for (int g = g0 + tid; g < g1; g += kMdT) {
+    const uint4 rnd = keyed_block(p.seed, p.step, kTagMdGumbel, b, 0, tau, static_cast<uint32_t>(g));
 #pragma unroll
     for (int w = 0; w < 4; ++w) {
-      const int v = 4 * gi + w;
-      if (v >= V) break;
-      const float wt = tau == L ? prob_t(L, v) : R[v];
+      const int v = 4 * g + w, e = v - v0;
+      if (e >= n) break;
+      const float wt = tau == L ? prob(qt(sa, L), e) : Rf[e];
       if (!(wt > 0.0f)) continue;
-      const float e = exponential_from_bits(word_of(rnd, w));
-      if (race_better(wt, e, v, bw, be, bi)) {
+      const float ev = exponential_from_bits(word_of(rnd, w));
+      if (race_better(wt, ev, v, bw, be, bi)) {
         bw = wt;
-        be = e;
+        be = ev;
         bi = v;
       }
     }
   }
-  race_reduce<kMdThreads>(bw, be, bi, s_race);
-  if (tid == 0) {
-    const int a = s_a;
-    for (int i = 0; i <= L; ++i) tok[i] = i < tau ? s_x[a * L + i] : (i == tau ? bi : -1);
+  race_reduce<kMdT>(bw, be, bi, sm.race);
+  if (tid == 0)
+    *reinterpret_cast<float4*>(cl.map_shared_rank(&sm.xb[buf][rank][0], 0)) =
+        make_float4(bw, be, __int_as_float(bi), 0.0f);
+  cl.sync();
+  if (rank == 0 && tid == 0) {
+    bw = 0.0f;
+    be = 1.0f;
+    bi = INT_MAX;
+    for (int q = 0; q < kMdC; ++q) {
+      const float4 g = *reinterpret_cast<const float4*>(&sm.xb[buf][q][0]);
+      if (race_better(g.x, g.y, __float_as_int(g.z), bw, be, bi)) {
+        bw = g.x;
+        be = g.y;
+        bi = __float_as_int(g.z);
+      }
+    }
+    const int a = sm.a;
+    for (int i = 0; i <= L; ++i) tok[i] = i < tau ? sm.tok[a * L + i] : (i == tau ? bi : -1);
     p.accept_len[b] = tau;
     if (p.out_draft_index) p.out_draft_index[b] = a;
   }
 }
 
+// ------------------------------------------------------------------ launch
+namespace {
+constexpr size_t kMaxDynSmem = 227 * 1024;
+
+struct MdShape {
+  int slice, rowstride;
+  size_t smem_local;
+};
+
+MdShape md_shape(int rows, int V, int dtype) {
+  const size_t es = dtype == SV_BF16 ? 2 : 4;
+  MdShape s{};
+  s.slice = ((V + kMdC - 1) / kMdC + 7) / 8 * 8;
+  s.rowstride = static_cast<int>((static_cast<size_t>(s.slice) * es + 16 + 15) / 16 * 16);
+  s.smem_local = kMdFixed + 2 * static_cast<size_t>(s.slice) * sizeof(float) +
+                 static_cast<size_t>(rows) * s.rowstride;
+  return s;
+}
+
+// Opt a variant into its dynamic shared memory and check that one cluster
+// of it can be resident (once per device and size); false if it cannot.
+template <typename Kernel>
+bool md_ready(Kernel kernel, size_t smem) {
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem)) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return false;
+  }
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(kMdC);
+  cfg.blockDim = dim3(kMdT);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = kMdC;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return false;
+  }
+  return n > 0;
+}
+
+template <typename Kernel>
+cudaError_t md_launch(Kernel kernel, int B, size_t smem, cudaStream_t stream, const MdcParams& p) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(B) * kMdC);
+  cfg.blockDim = dim3(kMdT);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = kMdC;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, p);
+}
+}  // namespace
+
+size_t multidraft_global_bytes(int B, int V) {  // residual laws of the global variant
+  return 2 * static_cast<size_t>(B) * static_cast<size_t>(V) * sizeof(float);
+}
+
+int multidraft_max_row_sets(int L) { return kMaxStatRows / (2 * L + 1); }
+
 int launch_multi(const void* target, const void* draft, const int32_t* tokens,
-                 const float* temps, int B, int K, int L, int V, int dtype, uint64_t seed,
-                 uint64_t step, int32_t* out_accept_len, int32_t* out_tokens,
+                 const float* temps, int B, int K, int L, int V, int dtype, int per_draft,
+                 uint64_t seed, uint64_t step, int32_t* out_accept_len, int32_t* out_tokens,
                  int32_t* out_draft_index, void* workspace, const Layout& lay,
                  cudaStream_t stream) {
   char* ws = static_cast<char*>(workspace);
-  Pass1Params p1{};
-  p1.target = target;
-  p1.draft = draft;
-  p1.tokens = tokens;
-  p1.temps = temps;
-  p1.B = B;
-  p1.gamma = L;
-  p1.V = V;
-  p1.nc = lay.nc;
-  p1.rps = 2 * L + 1;
-  p1.seed = seed;
-  p1.step = static_cast<uint32_t>(step);
-  p1.part = reinterpret_cast<RowPartial*>(ws + lay.part1);
-  p1.ticket = reinterpret_cast<unsigned*>(ws + lay.ticket1);
-  p1.rowstat = reinterpret_cast<RowPartial*>(ws + lay.rowstat);
-  const long long grid1 = static_cast<long long>(B) * p1.rps * lay.nc;
-  if (grid1 > INT_MAX)
-    return set_error(SV_ERR_INVALID_ARG, "B x (2L+1) x V too large for one launch (%lld CTAs)", grid1);
-  if (dtype == SV_BF16)
-    pass1_multi_kernel<true><<<static_cast<unsigned>(grid1), kP1Threads, 0, stream>>>(p1);
+  const int nsets = per_draft ? K : 1;
+  if (nsets * (2 * L + 1) > kMaxStatRows)
+    return set_error(SV_ERR_UNSUPPORTED,
+                     "per-draft rows: K (2L + 1) = %d row statistics per sequence, more than %d",
+                     nsets * (2 * L + 1), kMaxStatRows);
+  const MdShape sh = md_shape(nsets * (2 * L + 1), V, dtype);
+  MdcParams p{};
+  p.target = target;
+  p.draft = draft;
+  p.tokens = tokens;
+  p.temps = temps;
+  p.B = B;
+  p.K = K;
+  p.L = L;
+  p.V = V;
+  p.per_draft = per_draft ? 1 : 0;
+  p.seed = seed;
+  p.step = static_cast<uint32_t>(step);
+  p.slice = sh.slice;
+  p.rowstride = sh.rowstride;
+  p.Rws = reinterpret_cast<float*>(ws + lay.resid);
+  p.accept_len = out_accept_len;
+  p.out_tokens = out_tokens;
+  p.out_draft_index = out_draft_index;
+  if (static_cast<long long>(B) * kMdC > INT_MAX)
+    return set_error(SV_ERR_INVALID_ARG, "B too large for one launch");
+  const bool bf16 = dtype == SV_BF16;
+  // Once per device: each variant opted into its largest shared memory, and
+  // one cluster of it found residentable (1), or not (2).
+  static std::atomic<int> ready[2][2][64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+    return set_error(SV_ERR_CUDA, "no current CUDA device");
+  auto prepared = [&](bool local) {
+    std::atomic<int>& slot = ready[bf16 ? 1 : 0][local ? 1 : 0][dev];
+    int v = slot.load(std::memory_order_relaxed);
+    if (v == 0) {
+      const size_t smem = local ? kMaxDynSmem : kMdFixed;
+      bool ok;
+      if (local)
+        ok = bf16 ? md_ready(md_cluster_kernel<true, true>, smem) : md_ready(md_cluster_kernel<false, true>, smem);
+      else
+        ok = bf16 ? md_ready(md_cluster_kernel<true, false>, smem) : md_ready(md_cluster_kernel<false, false>, smem);
+      v = ok ? 1 : 2;
+      slot.store(v, std::memory_order_relaxed);
+    }
+    return v == 1;
+  };
+  const bool use_local = sh.smem_local <= kMaxDynSmem && prepared(true);
+  if (!use_local && !prepared(false))
+    return set_error(SV_ERR_CUDA, "multi-draft cluster kernel cannot be made resident");
+  cudaError_t e;
+  if (use_local)
+    e = bf16 ? md_launch(md_cluster_kernel<true, true>, B, sh.smem_local, stream, p)
+             : md_launch(md_cluster_kernel<false, true>, B, sh.smem_local, stream, p);
   else
-    pass1_multi_kernel<false><<<static_cast<unsigned>(grid1), kP1Threads, 0, stream>>>(p1);
-  if (int rc = check_launch("multidraft pass1")) return rc;
-
-  MdParams pm{};
-  pm.target = target;
-  pm.draft = draft;
-  pm.tokens = tokens;
-  pm.temps = temps;
-  pm.B = B;
-  pm.K = K;
-  pm.L = L;
-  pm.V = V;
-  pm.seed = seed;
-  pm.step = static_cast<uint32_t>(step);
-  pm.rowstat = p1.rowstat;
-  pm.R = reinterpret_cast<float*>(ws + lay.resid);
-  pm.accept_len = out_accept_len;
-  pm.out_tokens = out_tokens;
-  pm.out_draft_index = out_draft_index;
-  if (dtype == SV_BF16)
-    md_gbv_kernel<true><<<B, kMdThreads, 0, stream>>>(pm);
-  else
-    md_gbv_kernel<false><<<B, kMdThreads, 0, stream>>>(pm);
-  return check_launch("multidraft gbv");
+    e = bf16 ? md_launch(md_cluster_kernel<true, false>, B, kMdFixed, stream, p)
+             : md_launch(md_cluster_kernel<false, false>, B, kMdFixed, stream, p);
+  if (e != cudaSuccess)
+    return set_error(SV_ERR_CUDA, "multi-draft kernel launch failed: %s", cudaGetErrorString(e));
+  return check_launch("multidraft");
 }
 
 }  // namespace sv

@@ -6,6 +6,10 @@
 - a sequence whose oracle draw logged a Gumbel near-tie (top-2 gap < 1e-4)
   is excluded when only the drawn token differs;
 - gathered log-probabilities agree within 1e-5 absolute.
+
+TieLedger adds up the comparisons of a test and checks that the excluded
+sequences stay within a small multiple of the expected tie rate, so that a
+regression which shows only near ties cannot hide behind the exclusions.
 """
 from __future__ import annotations
 
@@ -76,3 +80,28 @@ def compare(gpu: dict, ora: dict, check_logprobs: bool = True) -> dict:
                 assert err <= LOGP_ATOL, f"{key}: max |gpu - oracle| = {err:.3g} > {LOGP_ATOL}"
     assert not bad, f"{len(bad)} mismatching sequences, first: {bad[:5]}"
     return stats
+
+
+class TieLedger:
+    """Counts of a test's comparisons: rows compared, ties logged by the
+    oracle and sequences excluded.  A Bernoulli tie has probability about
+    2e-6 per decision and a draw near-tie about 1e-4 per draw (more on
+    near-equality residuals, where the oracle's band widens), so the
+    excluded sequences stay far below `max_rate` of the rows."""
+
+    def __init__(self, name: str):
+        self.name = name
+        self.rows = self.excluded = self.bernoulli = self.gumbel = 0
+
+    def add(self, stats: dict) -> dict:
+        self.rows += stats["rows"]
+        self.excluded += stats["excluded"]
+        self.bernoulli += stats["bernoulli_ties"]
+        self.gumbel += stats["gumbel_ties"]
+        return stats
+
+    def check(self, max_rate: float = 2e-3, slack: int = 2):
+        print(f"{self.name}: rows {self.rows}, logged ties: bernoulli {self.bernoulli}, "
+              f"draw {self.gumbel}; excluded {self.excluded}")
+        assert self.excluded <= slack + max_rate * self.rows, (
+            f"{self.name}: {self.excluded} of {self.rows} sequences excluded as ties")

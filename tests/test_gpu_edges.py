@@ -60,3 +60,29 @@ def test_identical_drafts_accept_every_token():
 def test_many_tiny_rows():
     st = workloads.make_custom(300, 3, 5, dtype="bf16", seed=9, T=[0.0, 0.4, 1.0], device=DEV)
     compare(_gpu(st, 1, 0), run_oracle(st, 1, 0))
+
+
+def test_forced_rejection_near_equal_rows():
+    """The residual draw where it is most fragile: the draft row equals the
+    target row up to N(0, 1e-3) noise, except at the first draft token -- a
+    low-probability entry boosted by +2 in the draft row, so it is rejected
+    with probability about 0.86 -- and the correction token is drawn from
+    max(p - q, 0), a difference of nearly equal probabilities.  Many seeds
+    and steps; ties the oracle logs (its band widens with (p + q) / (p - q))
+    are excluded and counted."""
+    from tests.parity import TieLedger
+    ledger = TieLedger("near-equal residual draws")
+    B, gamma, V = 256, 2, 3001
+    residual = 0
+    for seed in (1, 2, 3):
+        s = workloads.make_custom(B, gamma, V, dtype="f32", seed=seed, T=[1.0, 0.7], device=DEV,
+                                  target_scale=2.0, noise=1e-3)
+        x = s.target[:, 0].argmin(dim=-1)
+        s.draft[torch.arange(B, device=DEV), 0, x] += 2.0
+        s.tokens[:, 0] = x.to(torch.int32)
+        for step in (0, 1):
+            g = _gpu(s, seed, step)
+            ledger.add(compare(g, run_oracle(s, seed, step)))
+            residual += int((g["accept_len"] == 0).sum())
+    assert residual > 0.7 * 6 * B  # the draws are mostly residual ones
+    ledger.check(max_rate=0.05, slack=5)

@@ -10,7 +10,7 @@ import torch
 
 import speculative_decoding_verification_85_b200 as sv
 import workloads
-from tests.parity import compare, run_oracle
+from tests.parity import TieLedger, compare, run_oracle
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda:0"
@@ -61,13 +61,15 @@ def test_small_shapes(B, gamma, V, dtype, T):
             compare(g, o)
 
 
-@pytest.mark.parametrize("cfg,steps", [(0, [0]), (1, [0, 1, 2, 50, 99]), (2, [0, 1, 49]),
-                                       (4, [0, 1, 199])])
+@pytest.mark.parametrize("cfg,steps", [(0, range(1)), (1, range(100)), (2, range(20)),
+                                       (4, range(20))])
 def test_workloads_full_size(cfg, steps):
-    """Every single-draft workload at its full shape, several steps, through
-    the same call and workspace reuse that the benchmark times."""
+    """Every single-draft workload at its full shape -- every step of C0 and
+    C1, the first 20 steps of C2 and C4 -- through the same call and workspace
+    reuse that the benchmark times."""
     c = workloads.get(cfg)
     v = sv.Verifier(DEV)
+    ledger = TieLedger(c.name)
     for step in steps:
         st = workloads.make_step(c, step, device=DEV)
         acc, tok, lp, lq = v.verify(st.target, st.draft, st.tokens, st.temps, seed=0, step=step,
@@ -75,21 +77,24 @@ def test_workloads_full_size(cfg, steps):
         torch.cuda.synchronize()
         g = {"accept_len": acc.cpu().numpy(), "tokens": tok.cpu().numpy(),
              "lp": lp.cpu().numpy(), "lq": lq.cpu().numpy()}
-        s = compare(g, run_oracle(st, 0, step))
-        print(c.name, step, s)
+        ledger.add(compare(g, run_oracle(st, 0, step)))
+    ledger.check()
 
 
 def test_multidraft_full_size():
+    """The multi-draft workload at its full shape, all 100 steps."""
     c = workloads.get(3)
     v = sv.Verifier(DEV)
-    for step in range(0, 100, 9):
+    ledger = TieLedger(c.name)
+    for step in range(100):
         st = workloads.make_step(c, step, device=DEV)
         acc, tok, idx = v.verify_multidraft(st.target, st.draft, st.tokens, st.temps, seed=0,
                                             step=step)
         torch.cuda.synchronize()
         g = {"accept_len": acc.cpu().numpy(), "tokens": tok.cpu().numpy(),
              "draft_index": idx.cpu().numpy()}
-        print(c.name, step, compare(g, run_oracle(st, 0, step)))
+        ledger.add(compare(g, run_oracle(st, 0, step)))
+    ledger.check()
 
 
 @pytest.mark.parametrize("B,K,L,V,dtype,T", [
@@ -217,3 +222,73 @@ def test_ks_gate_on_gpu_draws():
         return np.clip(below[i] + P[i] * (x - i), 0.0, 1.0)
 
     assert kstest(first, cdf).pvalue > 0.01
+
+
+def _per_draft_rows(B, K, L, V, dtype, seed, T, device):
+    """A row set per draft with prefix-consistent rows: draft k's rows at
+    position i depend only on its prefix x_k[0..i) (drafts that share a prefix
+    see equal rows, and every draft's row 0 is the same), as a
+    prefix-conditioned model gives them.  The rows of a prefix come from a
+    generator seeded by (seed, b, i, prefix); each draft's tokens from its own
+    generator, so the drafts are independent."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    base_t = torch.randn((L + 1, V), generator=g) * 2.0
+    base_d = base_t[:L] + torch.randn((L, V), generator=g) * 0.6
+    temps = torch.tensor([T[b % len(T)] for b in range(B)], dtype=torch.float32)
+    toks = torch.empty((B, K, L), dtype=torch.int32)
+    tgt = torch.empty((B, K, L + 1, V))
+    drf = torch.empty((B, K, L, V))
+    for b in range(B):
+        for k in range(K):
+            gk = torch.Generator(device="cpu")
+            gk.manual_seed((seed * 1000003 + b * 131 + k) & 0x7FFFFFFF)
+            prefix = []
+            for i in range(L + 1):
+                gi = torch.Generator(device="cpu")
+                gi.manual_seed(hash((seed, b, i) + tuple(prefix)) & 0x7FFFFFFF)
+                shift = torch.randn(V, generator=gi) * 0.8
+                tgt[b, k, i] = base_t[i] + shift
+                if i < L:
+                    drf[b, k, i] = base_d[i] + shift + torch.randn(V, generator=gi) * 0.3
+                    if float(temps[b]) > 0:
+                        q = torch.softmax(drf[b, k, i] / float(temps[b]), -1)
+                        x = int(torch.multinomial(q, 1, generator=gk))
+                    else:
+                        x = int(drf[b, k, i].argmax())
+                    toks[b, k, i] = x
+                    prefix.append(x)
+    if dtype == "bf16":
+        tgt, drf = tgt.to(torch.bfloat16), drf.to(torch.bfloat16)
+    return workloads.Step(tgt.contiguous().to(device), drf.contiguous().to(device),
+                          toks.to(device), temps.to(device), 0)
+
+
+@pytest.mark.parametrize("B,K,L,V,dtype,T", [
+    (4, 1, 1, 50, "f32", [1.0]),
+    (5, 3, 2, 7, "bf16", [0.7, 0.1]),
+    (6, 4, 5, 1000, "bf16", [0.1, 0.4, 0.7, 0.0]),
+    (8, 4, 5, 32000, "bf16", [0.1, 0.4, 0.7]),
+    (3, 8, 3, 4097, "f32", [1.0, 0.0]),
+])
+def test_multidraft_per_draft_rows(B, K, L, V, dtype, T):
+    """A row set per draft (target [B, K, L+1, V]): the CUDA path against the
+    oracle's per-draft verification."""
+    for seed in (1, 2):
+        st = _per_draft_rows(B, K, L, V, dtype, seed * 7 + V, T, DEV)
+        g = gpu_multi(st, seed=seed, step=5)
+        compare(g, run_oracle(st, seed, 5))
+
+
+def test_multidraft_per_draft_equal_copies_match_shared_rows():
+    """K equal copies of one row set give the shared-row results bit for bit."""
+    st = workloads.make_custom(6, 5, 3000, dtype="bf16", seed=77, T=[0.4, 0.7, 0.0], K=4,
+                               device=DEV, target_scale=2.0, noise=0.6)
+    K = st.tokens.shape[1]
+    rows = workloads.Step(st.target[:, None].expand(-1, K, -1, -1).contiguous(),
+                          st.draft[:, None].expand(-1, K, -1, -1).contiguous(), st.tokens,
+                          st.temps, 0)
+    a = gpu_multi(st, seed=3, step=9)
+    b = gpu_multi(rows, seed=3, step=9)
+    for key in ("accept_len", "tokens", "draft_index"):
+        assert np.array_equal(a[key], b[key]), key
