@@ -333,10 +333,9 @@ def run_ours(args, cfg):
     with torch.cuda.graph(graph, stream=stream):
         for i in range(W, W + K):
             one(i)
-    # kernels of this library per step: the row kernel plus the draw kernel
-    # (single draft), or the row pass plus the sequential verification kernel
-    # (multi-draft)
-    launches_per_replay = K * 2
+    # kernels of this library per step: two for single-draft (the row kernel,
+    # then the draw kernel), one for multi-draft (the cluster kernel)
+    launches_per_replay = K * (1 if cfg.multidraft else 2)
     with torch.cuda.stream(stream):
         graph.replay()  # warm the graph itself
     stream.synchronize()
@@ -461,8 +460,9 @@ def run_ours(args, cfg):
                        "launch": "K steps captured in one CUDA graph, replayed",
                        "parallelism": f"batch-sharded replicas x{world}"},
             "roofline": {"bound": "hbm",
-                         "kernel": ("pass1_multi_kernel + md_gbv_kernel (whole step)"
-                                    if cfg.multidraft else "rows_kernel + draw_kernel (whole step)"),
+                         "kernel": ("md_cluster_kernel (one launch per step)"
+                                    if cfg.multidraft else
+                                    "rows_kernel + draw_kernel (the whole step)"),
                          "achieved": algo_gbs, "peak": peak, "unit": "GB/s",
                          "frac": algo_gbs / peak, "traffic": traffic,
                          "peak_source": (f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)"

@@ -63,7 +63,7 @@ int check_device() {
 Layout layout_single(int B, int gamma, int V, int dtype) {
   Layout l{};
   l.nc = row_segments(V, dtype);
-  l.nc2 = draw_chunks(V, dtype);
+  l.nc2 = draw_chunks(B, V, dtype);
   l.ctl = 0;
   l.ticket1 = kHeaderCtl;
   l.ticket2 = kHeaderCtl + kSeqSlots;

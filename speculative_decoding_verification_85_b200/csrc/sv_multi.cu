@@ -42,9 +42,9 @@ namespace cg = cooperative_groups;
 namespace sv {
 
 constexpr int kMdC = 8;                          // CTAs per cluster (one sequence)
-constexpr int kMdT = 256;                        // threads per CTA
+constexpr int kMdT = 512;                        // threads per CTA
 constexpr int kMdW = kMdT / 32;
-constexpr int kXBatch = 128;                     // row statistics per exchange
+constexpr int kXBatch = 64;                      // row statistics per exchange
 constexpr int kXSlot = 2 * kXBatch;              // doubles per rank in an exchange buffer
 constexpr int kMaxStatRows = 256;                // row statistics per sequence (all row sets)
 constexpr int kMaxDraftTokens = SV_MAX_DRAFTS * SV_MAX_GAMMA;
@@ -82,12 +82,56 @@ struct alignas(16) MdSmem {
   float2 zg[kMaxDraftTokens];          // target / draft logit at each draft token
   int H[SV_MAX_DRAFTS];                // rejected tokens at tau
   float4 race[kMdW];
+  const char* rowp[kMaxStatRows];      // this slice's entry 0 of row q (shared or global memory)
   uint64_t bar;                        // staging barrier
+  uint64_t xbar[2];                    // exchange barriers (one per exchange buffer)
+  uint32_t xphase[2];                  // their current phase parity
+  int xfail;                           // an exchange wait ran out of time
   double Rn, qH, keep, wbest;
   int tau, a, nH, skip, best, rcur;
 };
 
 constexpr size_t kMdFixed = (sizeof(MdSmem) + 127) / 128 * 128;
+
+// Distributed-shared-memory stores that complete a transaction on the
+// destination CTA's mbarrier: the receiver waits on its own barrier, with no
+// cluster-wide barrier per exchange.
+__device__ __forceinline__ uint32_t mapa(const void* p, int rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_addr(p)), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void st_async_f64(uint32_t addr, double v, uint32_t bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b64 [%0], %1, [%2];"
+               ::"r"(addr), "l"(__double_as_longlong(v)), "r"(bar) : "memory");
+}
+__device__ __forceinline__ void st_async_f4(uint32_t addr, float4 v, uint32_t bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];"
+               ::"r"(addr), "r"(__float_as_uint(v.x)), "r"(__float_as_uint(v.y)),
+               "r"(__float_as_uint(v.z)), "r"(__float_as_uint(v.w)), "r"(bar)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_addr(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait (kWaitLimitNs) for a phase of an exchange barrier.
+__device__ __forceinline__ bool xbar_wait(uint64_t* bar, uint32_t parity) {
+  if (mbar_try_wait_cluster(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  for (;;) {
+    for (int k = 0; k < 64; ++k)
+      if (mbar_try_wait_cluster(bar, parity)) return true;
+    if (global_ns() - t0 > kWaitLimitNs) return false;
+  }
+}
 
 // The kMdC partials of an exchange, in rank order: thread t < nv contributes
 // `mine` as slot t of buffer `buf` to every CTA; after the cluster barrier
@@ -96,14 +140,22 @@ template <typename Cl>
 __device__ __forceinline__ void exchange(Cl& cl, MdSmem& sm, int buf, int nv, double mine) {
   const int tid = threadIdx.x;
   const int rank = static_cast<int>(cl.block_rank());
-  if (tid < nv)
-    for (int q = 0; q < kMdC; ++q) *cl.map_shared_rank(&sm.xb[buf][rank][tid], q) = mine;
-  cl.sync();
+  // every rank sends nv values to every rank: arm this CTA's barrier for them
+  if (tid == 0) mbar_arrive_expect_tx(&sm.xbar[buf], static_cast<uint32_t>(nv * kMdC * sizeof(double)));
+  if (tid < nv) {
+    // the CTA's earlier shared-memory writes (R, read remotely later) are
+    // ordered before the values that announce them (callers end with a CTA barrier)
+    asm volatile("fence.acq_rel.cluster;" ::: "memory");
+    for (int q = 0; q < kMdC; ++q) st_async_f64(mapa(&sm.xb[buf][rank][tid], q), mine, mapa(&sm.xbar[buf], q));
+  }
+  if (!xbar_wait(&sm.xbar[buf], sm.xphase[buf])) sm.xfail = 1;
   if (tid < nv) {
     double s = 0.0;
     for (int q = 0; q < kMdC; ++q) s += sm.xb[buf][q][tid];
     sm.res[tid] = s;
   }
+  __syncthreads();
+  if (tid == 0) sm.xphase[buf] ^= 1u;
   __syncthreads();
 }
 
@@ -162,27 +214,36 @@ __global__ void __launch_bounds__(kMdT) md_cluster_kernel(const __grid_constant_
     Rb[0] = p.Rws + static_cast<size_t>(b) * 2 * V + v0;
     Rb[1] = Rb[0] + V;
   }
-  // logit e (0 <= e < n) of row q of this slice
-  auto zrow = [&](int q, int e) -> float {
+  // logit e (0 <= e < n) of a row slice that starts at rp (shared memory when
+  // staged, else global memory)
+  auto zat = [&](const char* rp, int e) -> float {
     if constexpr (kLocal) {
-      const char* sp = srows + static_cast<size_t>(q) * p.rowstride +
-                       (reinterpret_cast<uintptr_t>(grow(q) + static_cast<size_t>(v0) * es) & 15u);
       if constexpr (kBf16)
-        return __uint_as_float(static_cast<uint32_t>(reinterpret_cast<const uint16_t*>(sp)[e]) << 16);
+        return __uint_as_float(static_cast<uint32_t>(reinterpret_cast<const uint16_t*>(rp)[e]) << 16);
       else
-        return reinterpret_cast<const float*>(sp)[e];
+        return reinterpret_cast<const float*>(rp)[e];
     } else {
-      return logit_at<kBf16>(grow(q), static_cast<int64_t>(v0) + e);
+      return logit_at<kBf16>(rp, e);
     }
   };
+  for (int q = tid; q < nq; q += kMdT) {
+    const char* g = grow(q) + static_cast<size_t>(v0) * es;
+    sm.rowp[q] = kLocal ? srows + static_cast<size_t>(q) * p.rowstride + (reinterpret_cast<uintptr_t>(g) & 15u)
+                        : g;
+  }
+  auto zrow = [&](int q, int e) -> float { return zat(sm.rowp[q], e); };
 
   // ---- draft tokens and their logits; staging of the slice's rows
   bool stage_ok = true;
   if (tid == 0) {
     mbar_init(&sm.bar, 1);
+    mbar_init(&sm.xbar[0], 1);
+    mbar_init(&sm.xbar[1], 1);
+    sm.xphase[0] = sm.xphase[1] = 0u;
+    sm.xfail = 0;
     mbar_init_fence();
   }
-  __syncthreads();
+  cl.sync();  // every CTA's barriers are initialised before any remote store
   for (int t = tid; t < K * L; t += kMdT) {
     const int x = __ldg(p.tokens + static_cast<size_t>(b) * K * L + t);
     const int k = t / L, i = t - k * L, set = p.per_draft ? k : 0;
@@ -247,9 +308,10 @@ __global__ void __launch_bounds__(kMdT) md_cluster_kernel(const __grid_constant_
       const int nb = min(kXBatch, nq - q0);
       for (int j = 0; j < nb; ++j) {
         RowAcc a{-INFINITY, 0.0f, 0x7fffffff, stage_ok ? 0 : 1};
+        const char* rp = sm.rowp[q0 + j];
         if (tvalid)
           for (int e = tid; e < n; e += kMdT) {
-            const float z = zrow(q0 + j, e);
+            const float z = zat(rp, e);
             if (greedy) acc_scalar<kRowArgmax>(a, z, v0 + e, c); else acc_scalar<kRowLse>(a, z, v0 + e, c);
           }
 #pragma unroll
@@ -263,6 +325,7 @@ __global__ void __launch_bounds__(kMdT) md_cluster_kernel(const __grid_constant_
         }
         if (lane == 0) sm.wpart[warp][j] = make_float4(a.m, a.s, __int_as_float(a.arg), __int_as_float(a.bad));
       }
+      if (tid == 0) mbar_arrive_expect_tx(&sm.xbar[buf], static_cast<uint32_t>(nb * kMdC * sizeof(float4)));
       __syncthreads();
       if (tid < nb) {
         RowAcc a{-INFINITY, 0.0f, 0x7fffffff, 0};
@@ -273,9 +336,9 @@ __global__ void __launch_bounds__(kMdT) md_cluster_kernel(const __grid_constant_
         }
         const float4 v = make_float4(a.m, a.s, __int_as_float(a.arg), __int_as_float(a.bad));
         for (int r = 0; r < kMdC; ++r)
-          *reinterpret_cast<float4*>(cl.map_shared_rank(&sm.xb[buf][rank][2 * tid], r)) = v;
+          st_async_f4(mapa(&sm.xb[buf][rank][2 * tid], r), v, mapa(&sm.xbar[buf], r));
       }
-      cl.sync();
+      if (!xbar_wait(&sm.xbar[buf], sm.xphase[buf])) sm.xfail = 1;
       if (tid < nb) {
         RowAcc a{-INFINITY, 0.0f, 0x7fffffff, 0};
         for (int r = 0; r < kMdC; ++r) {
@@ -291,12 +354,14 @@ __global__ void __launch_bounds__(kMdT) md_cluster_kernel(const __grid_constant_
         if (!greedy) rv = rv && isfinite(__fdiv_rn(a.m, T));
         row_ok = row_ok && rv;
       }
-      buf ^= 1;
       __syncthreads();  // wpart is reused by the next batch
+      if (tid == 0) sm.xphase[buf] ^= 1u;
+      buf ^= 1;
+      __syncthreads();
     }
   }
   // validity: temperature, rows, tokens (the same in every CTA of the cluster)
-  bool ok = tvalid && row_ok;
+  bool ok = tvalid && row_ok && !sm.xfail;
   for (int t = tid; t < K * L; t += kMdT) ok = ok && sm.tok[t] >= 0 && sm.tok[t] < V;
   ok = __syncthreads_and(ok);
   int32_t* tok = p.out_tokens + static_cast<size_t>(b) * (L + 1);
@@ -308,7 +373,8 @@ __global__ void __launch_bounds__(kMdT) md_cluster_kernel(const __grid_constant_
         if (p.out_draft_index) p.out_draft_index[b] = -1;
       }
     }
-    return;  // every CTA returns here: no one touches another CTA's memory any more
+    cl.sync();  // every CTA returns here, after every remote store has landed
+    return;
   }
   if (greedy) {
     // the accepted block is the longest draft prefix that matches the target
@@ -332,6 +398,7 @@ __global__ void __launch_bounds__(kMdT) md_cluster_kernel(const __grid_constant_
       p.accept_len[b] = tau;
       if (p.out_draft_index) p.out_draft_index[b] = a;
     }
+    cl.sync();
     return;
   }
 
@@ -340,7 +407,13 @@ __global__ void __launch_bounds__(kMdT) md_cluster_kernel(const __grid_constant_
   // within its 2^-22 relative error); one subtraction, one multiply, one ex2
   // and one multiply per value.
   const float cc = __fdiv_rn(kLog2e, T);
-  auto prob = [&](int q, int e) -> float { return ex2_approx((zrow(q, e) - sm.m[q]) * cc) * sm.is[q]; };
+  struct Law {
+    const char* rp;
+    float m, is;
+  };
+  auto law = [&](int q) { return Law{sm.rowp[q], sm.m[q], sm.is[q]}; };
+  auto at = [&](const Law& l, int e) -> float { return ex2_approx((zat(l.rp, e) - l.m) * cc) * l.is; };
+  auto prob = [&](int q, int e) -> float { return at(law(q), e); };
   auto prob_x = [&](int q, float z) -> float { return ex2_approx((z - sm.m[q]) * cc) * sm.is[q]; };
   auto exch1 = [&](double x) {  // one value: CTA sum, then cluster sum into sm.res[0]
     warp_sum_to(sm, 0, x);
@@ -427,9 +500,10 @@ __global__ void __launch_bounds__(kMdT) md_cluster_kernel(const __grid_constant_
     const int nA = max(L - 1 - tau, 0);
     for (int i = tau; i < L - 1; ++i) {
       const float wf = static_cast<float>(sm.w[i]);
+      const Law lp = law(qt(set, i + 1)), lq = law(qd(set, i + 1));
       double loc = 0.0;
       for (int e = tid; e < n; e += kMdT) {
-        const float t = wf * prob(qt(set, i + 1), e) - prob(qd(set, i + 1), e);
+        const float t = wf * at(lp, e) - at(lq, e);
         if (t > 0.0f) loc += t;
       }
       warp_sum_to(sm, i - tau, loc);
@@ -472,9 +546,10 @@ __global__ void __launch_bounds__(kMdT) md_cluster_kernel(const __grid_constant_
     if (best > tau) {
       if (best < L) {
         const float wb = static_cast<float>(sm.wbest);
+        const Law lp = law(qt(set, best)), lq = law(qd(set, best));
         double loc = 0.0;
         for (int e = tid; e < n; e += kMdT) {
-          const float t = wb * prob(qt(set, best), e) - prob(qd(set, best), e);
+          const float t = wb * at(lp, e) - at(lq, e);
           const float rv = t > 0.0f ? t : 0.0f;
           Rnew[e] = rv;
           loc += rv;
@@ -505,9 +580,10 @@ __global__ void __launch_bounds__(kMdT) md_cluster_kernel(const __grid_constant_
       const float inv_rn = static_cast<float>(1.0 / sm.Rn);
       const double keep = sm.keep;
       const float inv_keep = keep > 0.0 ? static_cast<float>(1.0 / keep) : 0.0f;
+      const Law lq = law(qd(set, tau));
       double loc = 0.0;
       for (int e = tid; e < n; e += kMdT) {
-        const float t = Rcur[e] * inv_rn - prob(qd(set, tau), e) * inv_keep;
+        const float t = Rcur[e] * inv_rn - at(lq, e) * inv_keep;
         const float rv = t > 0.0f ? t : 0.0f;
         Rnew[e] = rv;
         loc += rv;
@@ -552,19 +628,27 @@ __global__ void __launch_bounds__(kMdT) md_cluster_kernel(const __grid_constant_
   race_reduce<kMdT>(bw, be, bi, sm.race);
   if (tid == 0)
     *reinterpret_cast<float4*>(cl.map_shared_rank(&sm.xb[buf][rank][0], 0)) =
-        make_float4(bw, be, __int_as_float(bi), 0.0f);
+        make_float4(bw, be, __int_as_float(bi), __int_as_float(sm.xfail));
   cl.sync();
   if (rank == 0 && tid == 0) {
     bw = 0.0f;
     be = 1.0f;
     bi = INT_MAX;
+    int fail = 0;
     for (int q = 0; q < kMdC; ++q) {
       const float4 g = *reinterpret_cast<const float4*>(&sm.xb[buf][q][0]);
+      fail |= __float_as_int(g.w);
       if (race_better(g.x, g.y, __float_as_int(g.z), bw, be, bi)) {
         bw = g.x;
         be = g.y;
         bi = __float_as_int(g.z);
       }
+    }
+    if (fail) {  // an exchange wait of some rank ran out of time: no result
+      for (int i = 0; i <= L; ++i) tok[i] = -1;
+      p.accept_len[b] = -1;
+      if (p.out_draft_index) p.out_draft_index[b] = -1;
+      return;
     }
     const int a = sm.a;
     for (int i = 0; i <= L; ++i) tok[i] = i < tau ? sm.tok[a * L + i] : (i == tau ? bi : -1);

@@ -1,37 +1,26 @@
-// sv_single.cu -- single-draft verification: one persistent kernel per call.
+// sv_single.cu -- single-draft verification: a row kernel and a draw
+// kernel per call, chained by programmatic dependent launch.
 //
-// What it computes (per sequence b with temperature T > 0): the
-// temperature-scaled log-softmax of every needed row, the two
-// log-probabilities of each draft token, the acceptance test
-// u_i < min(1, p/q) with the first rejection j ("FlashSpec", Methodology
-// s.1; "FlexDraft", Problem definition), and the correction token at j drawn
-// from max(p_j - q_j, 0) or the bonus token from p_gamma ("Speculative
-// Speculative Decoding", s.2 Saguaro sampling), as a Gumbel-max with Philox
-// noise keyed per vocabulary entry.  T = 0 is greedy argmax matching.
-//
-// How: a grid of two CTAs per SM claims work items from a counter in the
-// workspace, in a fixed order:
-//   - row items: (sequence b, position i, vocabulary segment) -- target row i
-//     and draft row i over the segment, streamed through a ring of shared-
-//     memory stages by one-dimensional bulk copies (TMA) that a producer warp
-//     issues, and reduced by eight consumer warps to the row maximum and an
-//     integer-reference softmax sum; the CTA whose item completes a sequence
-//     (arrival ticket) combines its partials and makes the decision, then
-//     publishes it with a release flag;
-//   - draw items: (sequence b, vocabulary chunk) -- the exponential race of
-//     the correction/bonus draw over a strided part of the vocabulary.  A
-//     sequence's draw items are queued `lag` sequences after its row items, so
-//     the ALU-bound race of one sequence runs beside the HBM-bound rows of
-//     later ones.  Philox is evaluated only for 4-entry blocks that can still
-//     win: since E = -ln U > 2^-24 for every keyed uniform, a block whose
-//     largest weight w satisfies w 2^24 <= (a lower bound of the winning ratio)
-//     is skipped, exactly.  Skipped-or-not blocks are compacted per warp so
-//     that Philox runs on full warps.
-// A draw item waits (bounded) for its sequence's decision flag.  Items are
-// claimed in queue order and every row item precedes the draw items that wait
-// on it, so the item being waited on has been claimed by a running CTA, which
-// processes its items in claim order and never waits on a later item: the
-// waits always end.
+// Row kernel (FlashSpec, Methodology s.1): one CTA per (sequence, position,
+// vocabulary segment) streams the target row and the draft row of that
+// position over the segment with 16-byte loads issued up front, reduces the
+// maximum and the temperature-scaled softmax sum of both rows, picks up the
+// draft token's two logits, and publishes one partial.  The CTA that
+// completes a sequence (arrival ticket) combines its partials and makes the
+// decision: the two log-probabilities of every draft token, the Philox
+// acceptance uniforms, the first rejection by warp ballot (FlexDraft,
+// Problem definition).
+// Draw kernel (Speculative Speculative Decoding, s.2 Saguaro sampling): once
+// the row kernel has completed (griddepcontrol.wait), one CTA per (sequence,
+// vocabulary chunk) runs the exponential race for the correction token from
+// max(p_j - q_j, 0), or the bonus token from p_gamma, with Philox noise keyed
+// per vocabulary entry; the CTA that completes a sequence combines.  Philox
+// is evaluated only for 4-entry blocks that can still win: since
+// E = -ln U > 2^-24 for every keyed uniform, a block whose largest weight w
+// has 2^24 w <= (a lower bound of the winning ratio) is skipped, exactly; the
+// blocks that remain are compacted per warp so that Philox runs on full warps.
+// Neither kernel waits on another CTA: all ordering is by arrival tickets and
+// by the launch dependency.
 #include <atomic>
 #include <climits>
 
@@ -42,7 +31,6 @@
 
 namespace sv {
 
-// ------------------------------------------------------------------ decision
 // Acceptance probability min(1, p/q) from log-probabilities (fp64); q = 0
 // accepts when p > 0, 0/0 rejects.
 __device__ __forceinline__ double accept_prob(double lp, double lq) {
@@ -51,14 +39,12 @@ __device__ __forceinline__ double accept_prob(double lp, double lq) {
   return r < 1.0 ? r : 1.0;
 }
 
-// Warp 0 of the CTA that completed sequence b: validate, accept/reject, write
-// outputs, publish the draw's hand-off record and raise the sequence's
-// decision flag (1 + mode, release).  T is the sequence's temperature and
-// x[0..gamma) its draft tokens (staged in shared memory by the caller).
+// Warp 0 of the last-arriving CTA: validate, accept/reject, write outputs.
+// T is sequence b's temperature and x[0..gamma) its draft tokens (staged in
+// shared memory by the caller).
 template <bool kBf16>
 __device__ __noinline__ void decide_single(const CallParams& p, int b, float T, const int* x,
-                                           const RowAcc* rows, const float* zsel,
-                                           unsigned* ready) {
+                                           const RowAcc* rows, const float* zsel) {
   const int lane = threadIdx.x & 31;
   const int g = p.gamma;
   const bool tvalid = (T >= 0.0f) && !isinf(T);
@@ -96,7 +82,6 @@ __device__ __noinline__ void decide_single(const CallParams& p, int b, float T, 
     if (lane == 0) {
       p.accept_len[b] = -1;
       p.info[b].mode = kModeNone;
-      st_release(ready + b, 1u + kModeNone);
     }
     return;
   }
@@ -115,13 +100,20 @@ __device__ __noinline__ void decide_single(const CallParams& p, int b, float T, 
       const int i = lane + 32 * h;
       bool reject = false;
       if (i < g) {
+        constexpr size_t es = kBf16 ? 2 : 4;
+        const char* tr = static_cast<const char*>(p.target) +
+                         (static_cast<size_t>(b) * (g + 1) + i) * static_cast<size_t>(p.V) * es;
+        const char* dr = static_cast<const char*>(p.draft) +
+                         (static_cast<size_t>(b) * g + i) * static_cast<size_t>(p.V) * es;
         const RowAcc& ap = rows[i];
         const RowAcc& aq = rows[g + 1 + i];
         // d = fl32(fl32(z_x / T) - fl32(zmax / T)): the same fp32 operations
-        // as scaling the whole row and shifting by its maximum; the draft
-        // token's logits were picked up while the rows streamed
-        const float dp = __fsub_rn(__fdiv_rn(zsel[2 * i], T), __fdiv_rn(ap.m, T));
-        const float dq = __fsub_rn(__fdiv_rn(zsel[2 * i + 1], T), __fdiv_rn(aq.m, T));
+        // as scaling the whole row and shifting by its maximum.
+        // the draft token's logits were picked up while the rows streamed
+        const float zp = zsel ? zsel[2 * i] : logit_at<kBf16>(tr, xi[h]);
+        const float zq = zsel ? zsel[2 * i + 1] : logit_at<kBf16>(dr, xi[h]);
+        const float dp = __fsub_rn(__fdiv_rn(zp, T), __fdiv_rn(ap.m, T));
+        const float dq = __fsub_rn(__fdiv_rn(zq, T), __fdiv_rn(aq.m, T));
         const double lp = static_cast<double>(dp) - log(static_cast<double>(ap.s));
         const double lq = static_cast<double>(dq) - log(static_cast<double>(aq.s));
         const uint4 rnd = keyed_block(p.seed, p.step, kTagAccept, b, 0, i, i);
@@ -162,55 +154,29 @@ __device__ __noinline__ void decide_single(const CallParams& p, int b, float T, 
       }
     }
     p.info[b] = si;
-    st_release(ready + b, 1u + static_cast<unsigned>(si.mode));  // after the record
   }
 }
 
+
 // ------------------------------------------------------------------ layout
-constexpr int kCWarps = 8;                     // consumer warps of a CTA
-constexpr int kCThreads = 32 * kCWarps;        // 256 consumer threads
-constexpr int kVThreads = kCThreads + 32;      // + one producer warp
-constexpr int kStages = 3;                     // shared-memory ring stages
-constexpr int kSlotBytes = kTileVec * 16;      // one row's tile: 16 KB
-constexpr int kStageBytes = 2 * kSlotBytes;    // target tile + draft tile
-constexpr int kRingBytes = kStages * kStageBytes;
-constexpr int kQCap = 64;                      // per-warp race queue (power of two)
-constexpr int kRaceRound = kCThreads;          // Philox blocks per CTA per race round
-static_assert(kCThreads == kTileThreads, "one consumer thread per tile lane");
-
-enum ItemKind : int { kItemEnd = 0, kItemRow = 1, kItemDraw = 2 };
-constexpr int kFirstTile = 1, kLastTile = 2;
-
-// What the producer hands the consumers with each ring stage.
-struct alignas(16) TileDesc {
-  int kind;   // ItemKind
-  int b;      // sequence
-  int i;      // position (row item) or chunk (draw item)
-  int seg;    // vocabulary segment (row item)
-  int kb;     // first body vector of the tile (row item)
-  int nvA;    // 16-byte vectors of the target tile in the stage (0: not read)
-  int nvB;    // vectors of the draft tile (0: not read)
-  int flags;  // kFirstTile | kLastTile
-  float T;    // the sequence's temperature
-  int xg;     // the draft token at i (softmax rows with i < gamma), else -1
-  int pad0, pad1;
-};
+constexpr int kRowThreads = kTileThreads;  // 256
+constexpr int kDrawThreads = 256;
+constexpr int kDrawMaxBlocks = 8;          // Philox blocks per thread and draw CTA
+constexpr int kQCap = 64;                  // per-warp race queue (power of two)
+constexpr int kRaceBatch = 4;              // race rounds whose logits are loaded together
+static_assert(kRowThreads == kDrawThreads, "one thread count for both kernels");
 
 struct SingleParams {
-  CallParams p1;       // inputs, outputs, row arrivals (ticket), hand-off (info)
+  CallParams p1;       // inputs, outputs, decision state
+  RacePartial* part2;   // [B][nc2] draw partials
+  unsigned* ticket2;    // [B] draw arrivals
+  unsigned* bar;        // [B] draw bars (float bits, monotone), shared by a sequence's draw CTAs
+  int nc2;              // draw CTAs per sequence
+  int chunk2;           // vocabulary entries per draw CTA (a multiple of 4)
+  int nseg;             // row segments per row (gridDim.y of the row kernel)
+  int segvec;           // 16-byte vectors per row segment (multiple of kTileVec)
   float4* pairpart;     // [B][gamma + 1][nseg] x {target, draft} partials
   float* zx;            // [B][gamma][nseg][2] draft token's target / draft logit
-  RacePartial* part2;   // [B][nd] draw partials
-  unsigned* ticket2;    // [B] draw arrivals
-  unsigned* ready;      // [B] decision flags (1 + mode once decided)
-  unsigned* bar;        // [B] draw bars (float bits, monotone)
-  unsigned* ctl;        // control words (kCtlNext, kCtlExit, kCtlError)
-  int nseg;             // row segments per row
-  int segvec;           // 16-byte vectors per row segment (multiple of kTileVec)
-  int nd;               // draw items per sequence
-  int nr;               // row items per sequence: (gamma + 1) nseg
-  int lag;              // sequences between a sequence's rows and its draw items
-  int total;            // items in the queue: B (nr + nd)
 };
 
 template <bool kBf16>
@@ -226,179 +192,41 @@ __device__ __forceinline__ const char* draft_row(const CallParams& p, int b, int
          (static_cast<size_t>(b) * p.gamma + i) * static_cast<size_t>(p.V) * es;
 }
 
-// Item at queue position q: the row items of the first `lag` sequences, then
-// for k = 0, 1, ... the row items of sequence lag + k followed by the draw
-// items of sequence k, then the remaining draw items.
-struct Item {
-  int kind, b, idx;  // idx: row item within the sequence (i nseg + seg), or draw chunk
-};
-__device__ __forceinline__ Item decode_item(const SingleParams& f, int q) {
-  const int nr = f.nr, nd = f.nd, lag = f.lag, B = f.p1.B;
-  if (q < lag * nr) return Item{kItemRow, q / nr, q % nr};
-  q -= lag * nr;
-  const int mid = B - lag;
-  if (q < mid * (nr + nd)) {
-    const int k = q / (nr + nd), r = q % (nr + nd);
-    return r < nr ? Item{kItemRow, lag + k, r} : Item{kItemDraw, k, r - nr};
-  }
-  q -= mid * (nr + nd);
-  return Item{kItemDraw, mid + q / nd, q % nd};
+__device__ __forceinline__ void pdl_wait_and_release() {
+  // Wait for the previous grid in the stream (programmatic dependent launch),
+  // then let the next one start launching its CTAs.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;");
 }
 
-// ------------------------------------------------------------ shared memory
-struct alignas(16) VerifySmem {
-  TileDesc desc[kStages];
-  uint64_t full[kStages];
-  uint64_t empty[kStages];
-  RowAcc rows[kMaxRowsPerSeq];
-  RowAcc scratch[2 * kCWarps];
-  float2 zxw[kCWarps];
-  float zsel[2 * SV_MAX_GAMMA];
-  int tok[SV_MAX_GAMMA];
-  float4 race[kCWarps];
-  float4 qw[kCWarps][kQCap];  // race queue: weights of a pending block
-  int qg[kCWarps][kQCap];     // race queue: the pending block
-  SeqInfo info;
-  int last;
-};
-
-// ---------------------------------------------------------------- producer
-// Lane 0 of the producer warp: claim items (one ahead), describe each ring
-// stage and issue its bulk copies.  Rows are read from the first 16-byte
-// boundary on; the unaligned head and tail of a row are read by the
-// consumers as scalars.
-template <bool kBf16>
-__device__ void produce(const SingleParams& f, VerifySmem& sm, char* ring) {
-  const CallParams& p = f.p1;
-  unsigned* next = f.ctl + kCtlNext;
-  int stage = 0;
-  uint32_t phase = 1;  // a fresh barrier's preceding phase counts as complete
-  auto take = [&](TileDesc& d) -> bool {
-    if (!mbar_wait(&sm.empty[stage], phase)) {
-      atomicExch(f.ctl + kCtlError, 1u);
-      return false;
-    }
-    sm.desc[stage] = d;
-    return true;
-  };
-  auto advance = [&]() {
-    if (++stage == kStages) {
-      stage = 0;
-      phase ^= 1u;
-    }
-  };
-  int cur = static_cast<int>(atomicAdd(next, 1u));
-  for (;;) {
-    const int nxt = cur < f.total ? static_cast<int>(atomicAdd(next, 1u)) : 0;
-    if (cur >= f.total) {
-      TileDesc d{};
-      d.kind = kItemEnd;
-      if (take(d)) mbar_arrive(&sm.full[stage]);
-      return;
-    }
-    const Item it = decode_item(f, cur);
-    TileDesc d{};
-    d.b = it.b;
-    if (it.kind == kItemDraw) {
-      d.kind = kItemDraw;
-      d.i = it.idx;
-      if (!take(d)) return;
-      mbar_arrive(&sm.full[stage]);
-      advance();
-    } else {
-      const int i = it.idx / f.nseg, seg = it.idx - i * f.nseg;
-      const float T = __ldg(p.temps + it.b);
-      const int modeA = row_mode(T, true);
-      const bool loadA = modeA != kRowSkip;
-      const bool loadB = i < p.gamma && row_mode(T, false) == kRowLse;
-      int xg = -1;
-      if (modeA == kRowLse && i < p.gamma) {
-        const int xt = __ldg(p.tokens + static_cast<size_t>(it.b) * p.gamma + i);
-        if (xt >= 0 && xt < p.V) xg = xt;
-      }
-      const char* rpA = target_row<kBf16>(p, it.b, i);
-      const char* rpB = loadB ? draft_row<kBf16>(p, it.b, i) : rpA;
-      const RowGeom<kBf16> gA(rpA, p.V), gB(rpB, p.V);
-      const int k0 = seg * f.segvec;
-      const int a1 = loadA ? min(gA.nvec, k0 + f.segvec) : k0;
-      const int b1 = loadB ? min(gB.nvec, k0 + f.segvec) : k0;
-      const int kend = max(max(a1, b1), k0 + 1);  // at least one stage per item
-      d.kind = kItemRow;
-      d.i = i;
-      d.seg = seg;
-      d.T = T;
-      d.xg = xg;
-      const uint4* vA = gA.body(rpA);
-      const uint4* vB = gB.body(rpB);
-      for (int kb = k0; kb < kend; kb += kTileVec) {
-        d.kb = kb;
-        d.nvA = max(0, min(a1 - kb, kTileVec));
-        d.nvB = max(0, min(b1 - kb, kTileVec));
-        d.flags = (kb == k0 ? kFirstTile : 0) | (kb + kTileVec >= kend ? kLastTile : 0);
-        if (!take(d)) return;
-        const uint32_t bytes = static_cast<uint32_t>(d.nvA + d.nvB) * 16u;
-        char* st = ring + stage * kStageBytes;
-        if (bytes) {
-          mbar_arrive_expect_tx(&sm.full[stage], bytes);
-          if (d.nvA) bulk_g2s(st, vA + kb, static_cast<uint32_t>(d.nvA) * 16u, &sm.full[stage]);
-          if (d.nvB)
-            bulk_g2s(st + kSlotBytes, vB + kb, static_cast<uint32_t>(d.nvB) * 16u, &sm.full[stage]);
-        } else {
-          mbar_arrive(&sm.full[stage]);
-        }
-        advance();
-      }
-    }
-    cur = nxt;
-  }
-}
-
-// --------------------------------------------------------- row reductions
+// Empty partials: softmax rows carry R = -inf in the index slot.
 __device__ __forceinline__ RowAcc empty_lse_acc() {
   return RowAcc{-INFINITY, 0.0f, __float_as_int(-INFINITY), 0};
 }
 __device__ __forceinline__ RowAcc empty_argmax_acc() { return RowAcc{-INFINITY, 0.0f, 0x7fffffff, 0}; }
 
-__device__ __forceinline__ float first_number(float z) {  // any lane's non-NaN value
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) {
-    const float o = __shfl_xor_sync(0xffffffffu, z, off);
-    if (z != z) z = o;
-  }
-  return z;
-}
-
-// Consumer-wide reduction of the two rows' accumulators and of the draft
-// token's two picked-up logits: a butterfly within each warp, then warp 0
-// merges the 8 warp results of each row by a 3-step butterfly (lanes 0-7 row
-// A, lanes 8-15 row B).  One barrier; the result is valid in thread 0.
-__device__ __forceinline__ void reduce_pair(RowAcc& A, RowAcc& B, float2& z, bool argmaxA,
-                                            VerifySmem& sm) {
-  constexpr int W = kCWarps;
+// Block reduction of the two rows' accumulators: a butterfly within each
+// warp, then warp 0 merges the 8 warp results of each row by a 3-step
+// butterfly (lanes 0-7 row A, lanes 8-15 row B).  One barrier; the result is
+// valid in thread 0.
+__device__ __forceinline__ void reduce_pair(RowAcc& A, RowAcc& B, bool argmaxA, RowAcc* scratch) {
+  constexpr int W = kRowThreads / 32;  // 8 warps
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   warp_merge(A, argmaxA);
   warp_merge(B, false);
-  z.x = first_number(z.x);
-  z.y = first_number(z.y);
   if (lane == 0) {
-    sm.scratch[warp] = A;
-    sm.scratch[W + warp] = B;
-    sm.zxw[warp] = z;
+    scratch[warp] = A;
+    scratch[W + warp] = B;
   }
-  block_sync<kCThreads>();
+  block_sync<kRowThreads>();
   if (warp == 0) {
     const bool rowB = lane >= W;
-    RowAcc v = lane < 2 * W ? sm.scratch[lane] : empty_lse_acc();
+    RowAcc v = lane < 2 * W ? scratch[lane] : empty_lse_acc();
     group_merge<W>(v, rowB ? false : argmaxA);
     const RowAcc vb = shfl_xor_acc(v, W);  // lane 0 receives lane 8's row-B result
     if (lane == 0) {
       A = v;
       B = vb;
-      for (int w = 0; w < W; ++w) {
-        const float2 q = sm.zxw[w];
-        if (q.x == q.x) z.x = q.x;
-        if (q.y == q.y) z.y = q.y;
-      }
     }
   }
 }
@@ -415,13 +243,14 @@ __device__ __forceinline__ float sum_rel_max(const RowAcc& a, float c) {
 }
 
 // Combine the nseg segment partials of every position of sequence b into the
-// row table sm.rows (target rows 0..gamma, then draft rows), and pick up the
-// draft tokens' logits (sm.zsel[2i], [2i + 1]).
+// row table rows[] (target rows 0..gamma, then draft rows), and pick up the
+// draft tokens' logits (zsel[2i], zsel[2i+1]).  argmaxA and c describe the
+// sequence (greedy or softmax, c = log2(e) / T).
 __device__ __forceinline__ void combine_pairs(const SingleParams& f, int b, bool argmaxA, float c,
-                                              VerifySmem& sm) {
+                                              RowAcc* rows, float* zsel) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int g = f.p1.gamma;
-  for (int i = warp; i <= g; i += kCWarps) {
+  for (int i = warp; i <= g; i += kRowThreads / 32) {
     RowAcc A = argmaxA ? empty_argmax_acc() : empty_lse_acc(), B = empty_lse_acc();
     float zt = __int_as_float(0x7fc00000), zd = zt;
     const float4* pp = f.pairpart + (static_cast<size_t>(b) * (g + 1) + i) * f.nseg * 2;
@@ -439,78 +268,161 @@ __device__ __forceinline__ void combine_pairs(const SingleParams& f, int b, bool
     }
     warp_merge(A, argmaxA);
     warp_merge(B, false);
-    zt = first_number(zt);
-    zd = first_number(zd);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      const float a = __shfl_xor_sync(0xffffffffu, zt, off);
+      const float d = __shfl_xor_sync(0xffffffffu, zd, off);
+      if (zt != zt) zt = a;
+      if (zd != zd) zd = d;
+    }
     if (lane == 0) {
       if (!argmaxA) A.s = sum_rel_max(A, c);
       B.s = sum_rel_max(B, c);
-      sm.rows[i] = A;
+      rows[i] = A;
       if (i < g) {
-        sm.rows[g + 1 + i] = B;
-        sm.zsel[2 * i] = zt;
-        sm.zsel[2 * i + 1] = zd;
+        rows[g + 1 + i] = B;
+        zsel[2 * i] = zt;
+        zsel[2 * i + 1] = zd;
       }
     }
   }
-  block_sync<kCThreads>();
+  block_sync<kRowThreads>();
 }
 
 // Head (entries before the first 16-byte boundary) and tail (after the last)
-// of a row, read as scalars by the first / last segment's item.
+// of a row, read as scalars by the first / last segment's CTA.
 template <bool kBf16>
 __device__ __forceinline__ void row_edges(const char* rp, int V, const RowGeom<kBf16>& g, bool argmax,
-                                          float c, bool head, bool tail, int xg, float& zx,
+                                          float c, bool head, bool tail, int xg, float* zx,
                                           RunAcc& acc) {
   const int tid = threadIdx.x;
   if (head)
-    for (int v = tid; v < g.head; v += kCThreads) {
+    for (int v = tid; v < g.head; v += kRowThreads) {
       const float z = logit_at<kBf16>(rp, v);
-      if (v == xg) zx = z;
+      if (v == xg) *zx = z;
       if (argmax) argmax_scalar(acc, z, v); else lse_scalar(acc, z, c);
     }
   if (tail)
-    for (int v = g.tail0 + tid; v < V; v += kCThreads) {
+    for (int v = g.tail0 + tid; v < V; v += kRowThreads) {
       const float z = logit_at<kBf16>(rp, v);
-      if (v == xg) zx = z;
+      if (v == xg) *zx = z;
       if (argmax) argmax_scalar(acc, z, v); else lse_scalar(acc, z, c);
     }
 }
 
 // The body vector that holds entry xg of a row, if this thread loads it within
-// the segment [k0, k1); -1 otherwise.  Tiles start at k0 + t kTileVec, so the
-// thread that loads vector k is (k - k0) mod kCThreads in every tile.
+// the segment [k0, k1); -1 otherwise.
 template <bool kBf16>
 __device__ __forceinline__ int owned_vector(const RowGeom<kBf16>& g, int xg, int k0, int k1) {
   if (xg < g.head || xg >= g.tail0) return -1;
   const int k = (xg - g.head) / Vec16<kBf16>::kN;
-  if (k < k0 || k >= k1 || (k - k0) % kCThreads != static_cast<int>(threadIdx.x)) return -1;
+  if (k < k0 || k >= k1 || (k - k0) % kRowThreads != static_cast<int>(threadIdx.x)) return -1;
   return k;
 }
 
 template <bool kBf16>
 __device__ __forceinline__ void pick_logit(const uint4 (&r)[kTileRegs], int own, int kb, int xg,
-                                           const RowGeom<kBf16>& g, float& zx) {
+                                           const RowGeom<kBf16>& g, float* zx) {
   if (own < kb || own >= kb + kTileVec) return;
-  const int j = (own - kb) / kCThreads;
+  const int j = (own - kb) / kRowThreads;
   const int e = (xg - g.head) % Vec16<kBf16>::kN;
 #pragma unroll
   for (int q = 0; q < kTileRegs; ++q)  // compile-time q keeps r[] in registers
-    if (q == j) zx = Vec16<kBf16>::at(r[q], e);
+    if (q == j) *zx = Vec16<kBf16>::at(r[q], e);
 }
 
-// The thread's vectors of a staged tile (nv valid vectors); the rest read as -inf.
+// --------------------------------------------------------------- row kernel
+// Grid: x = b (gamma + 1) + i (row pair), y = segment.
 template <bool kBf16>
-__device__ __forceinline__ void stage_tile(const char* slot, int nv, uint4 (&r)[kTileRegs]) {
-  constexpr uint32_t ninf = Vec16<kBf16>::kNegInf;
-  const uint4* v = reinterpret_cast<const uint4*>(slot);
-#pragma unroll
-  for (int j = 0; j < kTileRegs; ++j) {
-    const int k = static_cast<int>(threadIdx.x) + j * kCThreads;
-    r[j] = k < nv ? lds128(v + k) : make_uint4(ninf, ninf, ninf, ninf);
+__global__ void __launch_bounds__(kRowThreads, 3) rows_kernel(const __grid_constant__ SingleParams f) {
+  __shared__ RowAcc rows[kMaxRowsPerSeq];
+  __shared__ RowAcc scratch[2 * (kRowThreads / 32)];
+  __shared__ float s_zx[2];
+  __shared__ float s_zsel[2 * SV_MAX_GAMMA];
+  __shared__ int s_tok[SV_MAX_GAMMA];
+  __shared__ int s_last;
+  pdl_wait_and_release();
+  const CallParams& p = f.p1;
+  const int tid = threadIdx.x;
+  const int pair = blockIdx.x;
+  const int b = pair / (p.gamma + 1);
+  const int i = pair - b * (p.gamma + 1);
+  const int seg = blockIdx.y;
+  const float T = __ldg(p.temps + b);
+  const int modeA = row_mode(T, true);
+  const bool argmaxA = modeA == kRowArgmax;
+  const bool loadA = modeA != kRowSkip;
+  const bool loadB = i < p.gamma && row_mode(T, false) == kRowLse;
+  const float c = modeA == kRowLse ? __fdiv_rn(kLog2e, T) : 0.0f;
+  int xg = -1;
+  if (modeA == kRowLse && i < p.gamma) {
+    const int xt = __ldg(p.tokens + static_cast<size_t>(b) * p.gamma + i);
+    if (xt >= 0 && xt < p.V) xg = xt;
   }
+  if (tid == 0) s_zx[0] = s_zx[1] = __int_as_float(0x7fc00000);  // NaN: "not in this segment"
+  // the sequence's draft tokens, for the decision if this CTA completes it
+  for (int k = tid; k < p.gamma; k += kRowThreads) s_tok[k] = __ldg(p.tokens + static_cast<size_t>(b) * p.gamma + k);
+  block_sync<kRowThreads>();
+
+  RunAcc accA, accB;
+  accA.reset();
+  accB.reset();
+  const char* rpA = target_row<kBf16>(p, b, i);
+  const char* rpB = loadB ? draft_row<kBf16>(p, b, i) : rpA;
+  const RowGeom<kBf16> gA(rpA, p.V), gB(rpB, p.V);
+  const int k0 = seg * f.segvec;
+  const int a1 = min(gA.nvec, k0 + f.segvec), b1 = min(gB.nvec, k0 + f.segvec);
+  const uint4* vA = gA.body(rpA);
+  const uint4* vB = gB.body(rpB);
+  const int ownA = owned_vector<kBf16>(gA, xg, k0, a1);
+  const int ownB = owned_vector<kBf16>(gB, xg, k0, b1);
+  const int kend = max(loadA ? a1 : k0, loadB ? b1 : k0);
+  for (int kb = k0; kb < kend; kb += kTileVec) {
+    uint4 ra[kTileRegs], rb[kTileRegs];
+    if (loadA) load_tile<kBf16>(vA, kb, a1, ra);
+    if (loadB) load_tile<kBf16>(vB, kb, b1, rb);
+    if (loadA) {
+      pick_logit<kBf16>(ra, ownA, kb, xg, gA, &s_zx[0]);
+      if (argmaxA)
+        argmax_tile<kBf16>(accA, ra, gA.head + (kb + tid) * Vec16<kBf16>::kN);
+      else
+        lse_tile<kBf16>(accA, ra, c);
+    }
+    if (loadB) {
+      pick_logit<kBf16>(rb, ownB, kb, xg, gB, &s_zx[1]);
+      lse_tile<kBf16>(accB, rb, c);
+    }
+  }
+  const bool first = seg == 0, last = seg == f.nseg - 1;
+  if (loadA && (first || last))
+    row_edges<kBf16>(rpA, p.V, gA, argmaxA, c, first, last, xg, &s_zx[0], accA);
+  if (loadB && (first || last))
+    row_edges<kBf16>(rpB, p.V, gB, false, c, first, last, xg, &s_zx[1], accB);
+
+  RowAcc A = argmaxA ? accA.argmax_row() : accA.lse_row(), B = accB.lse_row();
+  reduce_pair(A, B, argmaxA, scratch);
+  if (tid == 0) {
+    float4* pp = f.pairpart + ((static_cast<size_t>(b) * (p.gamma + 1) + i) * f.nseg + seg) * 2;
+    pp[0] = make_float4(A.m, A.s, __int_as_float(A.arg), __int_as_float(A.bad));
+    pp[1] = make_float4(B.m, B.s, __int_as_float(B.arg), __int_as_float(B.bad));
+    if (i < p.gamma) {
+      float* z = f.zx + ((static_cast<size_t>(b) * p.gamma + i) * f.nseg + seg) * 2;
+      z[0] = s_zx[0];
+      z[1] = s_zx[1];
+    }
+    // release this CTA's partial; the last arriver also acquires the others'
+    const unsigned tk = ticket_acq_rel(p.ticket + b);
+    const unsigned arrivals = static_cast<unsigned>((p.gamma + 1) * f.nseg);
+    s_last = (tk == arrivals - 1);
+    if (s_last) p.ticket[b] = 0;  // leave the counter at zero for the next call
+  }
+  block_sync<kRowThreads>();  // orders the other threads after thread 0's acquire
+  if (!s_last) return;
+  combine_pairs(f, b, argmaxA, c, rows, s_zsel);
+  if (tid < 32) decide_single<kBf16>(p, b, T, s_tok, rows, s_zsel);
 }
 
-// ------------------------------------------------------------------- races
+// -------------------------------------------------------------- draw kernel
 // The 4 logits of Philox block g of a row, kept packed until used; entries
 // at or beyond V read as -inf.
 template <bool kBf16>
@@ -622,18 +534,48 @@ __device__ __forceinline__ float warp_max(float v) {
   return v;
 }
 
+// Philox stream of one draw race: blocks (c0 = g) of the keyed counter
+// (g, b, step, tag 2 << 24 | j) under key (lo32 seed, hi32 seed).
+struct RaceKey {
+  uint32_t k0, k1, b, step, c3;
+  __device__ __forceinline__ uint4 block(int g) const {
+    return philox4x32_10(make_uint4(static_cast<uint32_t>(g), b, step, c3), k0, k1);
+  }
+};
+
+// Philox and the exact test for up to 32 queued blocks, one per lane (lanes
+// at or beyond `count` take none).
+__device__ __forceinline__ void flush_queue(Race& race, const float4* qw, const int* qg, int head,
+                                            int count, const RaceKey& key) {
+  const int lane = threadIdx.x & 31;
+  const int e = (head + lane) & (kQCap - 1);
+  const bool mine = lane < count;
+  const float4 ww = mine ? qw[e] : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+  const int gg = mine ? qg[e] : 0;
+  __syncwarp();  // entries read before later rounds overwrite them
+  if (mine) race_block(race, ww, key.block(gg), 4 * gg);
+}
+
 // Exponential race of sequence b's draw over the Philox blocks of chunk
-// `chunk` of nchunk (round r covers blocks [(r nchunk + chunk) 256, + 256);
-// warp w takes 32 of them): the winner of w_v / E_v (E_v = -ln U_v) with
+// `chunk` of nchunk, by one CTA: round r covers blocks
+// [(r nchunk + chunk) 256, + 256), warp w 32 of them, one per lane, so every
+// chunk meets the low vocabulary indices first; each warp keeps its own
+// winner.  The winner is that of w_v / E_v (E_v = -ln U_v) with
 // w = max(p - q, 0) (residual) or w = p (bonus), p_v = 2^{(z_v - zmp) c - lsp}.
-// A block is queued for Philox only if 2^24 max_k w_k exceeds the warp's bar
-// (exact: E > 2^-24, so a skipped entry's ratio stays below the bar, which is
-// below the winning ratio); the queue is flushed 32 blocks at a time, so
-// Philox runs on full warps.  `gbar` (or NULL) is the sequence's shared bar:
-// read every few rounds, raised when this warp's bar grows.
+// Rounds are taken kRaceBatch at a time, their logits loaded together.  The
+// warp's bar (a lower bound of the winning ratio, lowered for rounding) starts
+// from the sequence's shared bar and from max w / 17 (an entry's E is below
+// 17 for every keyed uniform), and grows with every candidate tested.  A block
+// is queued for Philox only if 2^24 max_k w_k exceeds the bar (exact: E > 2^-24,
+// so a skipped entry's ratio stays below the bar, which is below the winning
+// ratio); the queue is flushed 32 blocks at a time, so Philox runs on full
+// warps, and a batch in which every block needs Philox bypasses the queue.
+// `gbar` (or NULL) is the sequence's shared bar: read every batch, raised when
+// this warp's bar grows.
 template <bool kBf16>
-__device__ void race_chunk(const SingleParams& f, const SeqInfo& si, int b, int chunk, int nchunk,
-                           unsigned* gbar, Race& race, VerifySmem& sm) {
+__device__ __forceinline__ void race_span(const SingleParams& f, const SeqInfo& si, int b, int chunk,
+                                          int nchunk, unsigned* gbar, Race& race, float4* qw, int* qg) {
+  constexpr int U = kRaceBatch;
   constexpr uintptr_t kVecAlign = kBf16 ? 8 : 16;
   const CallParams& p = f.p1;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -644,59 +586,88 @@ __device__ void race_chunk(const SingleParams& f, const SeqInfo& si, int b, int 
   const bool dvec = (reinterpret_cast<uintptr_t>(drow) % kVecAlign) == 0;
   const float2 nm = make_float2(-si.zmp, -si.zmq), cc = make_float2(si.c, si.c),
                nl = make_float2(-si.lsp, -si.lsq);
-  const PhiloxStream ps(p.seed, p.step, kTagGumbel, b, 0, si.j);
+  const RaceKey key{static_cast<uint32_t>(p.seed), static_cast<uint32_t>(p.seed >> 32),
+                    static_cast<uint32_t>(b), p.step, (kTagGumbel << 24) | static_cast<uint32_t>(si.j)};
   const int nblocks = (p.V + 3) / 4;
-  float4* qw = sm.qw[warp];
-  int* qg = sm.qg[warp];
   int qh = 0, qn = 0;  // queue head and length (warp-uniform)
   float published = 0.0f;
   unsigned gnext = 0;
   const unsigned lt_mask = (1u << lane) - 1u;
   if (gbar && lane == 0) gnext = ld_relaxed(gbar);
-  for (int r = 0;; ++r) {
-    const int base = (r * nchunk + chunk) * kRaceRound;
-    if (base >= nblocks) break;  // uniform over the CTA
-    const int g = base + warp * 32 + lane;
-    float w[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-    if (g < nblocks) {
-      Block4<kBf16> t, d;
-      t.load(trow, tvec, p.V, g);
-      if (resid) d.load(drow, dvec, p.V, g); else d.set_neg_inf();
+  for (int r0 = 0;; r0 += U) {
+    if ((r0 * nchunk + chunk) * kDrawThreads >= nblocks) break;  // uniform over the CTA
+    int g[U];
+    float4 w[U];
+    {
+      Block4<kBf16> tb[U], db[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        g[u] = ((r0 + u) * nchunk + chunk) * kDrawThreads + warp * 32 + lane;
+        tb[u].set_neg_inf();
+        db[u].set_neg_inf();
+        if (g[u] < nblocks) {
+          tb[u].load(trow, tvec, p.V, g[u]);
+          if (resid) db[u].load(drow, dvec, p.V, g[u]);
+        }
+      }
       // p_v = 2^{(z_v - zmp) c - lsp}, q_v likewise: the target and draft
       // value of an entry travel as one packed pair
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const float2 e = __ffma2_rn(__fadd2_rn(make_float2(t.at(k), d.at(k)), nm), cc, nl);
-        w[k] = ex2_approx(e.x);
-        if (resid) w[k] -= ex2_approx(e.y);
+      for (int u = 0; u < U; ++u) {
+        float ww[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float2 e = __ffma2_rn(__fadd2_rn(make_float2(tb[u].at(k), db[u].at(k)), nm), cc, nl);
+          ww[k] = ex2_approx(e.x);
+          if (resid) ww[k] -= ex2_approx(e.y);
+        }
+        w[u] = make_float4(ww[0], ww[1], ww[2], ww[3]);
       }
     }
-    if (gbar) {  // the shared bar read one round earlier
+    {
+      // bar from the heaviest entry of the batch: its E is below 17
+      float wmx = 0.0f;
+#pragma unroll
+      for (int u = 0; u < U; ++u) wmx = fmaxf(wmx, fmaxf(fmaxf(w[u].x, w[u].y), fmaxf(w[u].z, w[u].w)));
+      race.lo = fmaxf(race.lo, warp_max(wmx) * (1.0f / 17.0f));
+    }
+    if (gbar) {  // the shared bar read one batch earlier
       const float gv = __uint_as_float(__shfl_sync(0xffffffffu, gnext, 0));
       race.lo = fmaxf(race.lo, gv);
-      if (lane == 0 && (r & 3) == 3) gnext = ld_relaxed(gbar);
+      if (lane == 0) gnext = ld_relaxed(gbar);
     }
-    const float wm = fmaxf(fmaxf(w[0], w[1]), fmaxf(w[2], w[3]));
-    const bool need = wm * 16777216.0f > race.lo;
-    const unsigned bal = __ballot_sync(0xffffffffu, need);
-    if (bal == 0xffffffffu && qn == 0) {
-      race_block(race, make_float4(w[0], w[1], w[2], w[3]), ps.block(g), 4 * g);
-    } else if (bal) {
-      const int pos = (qh + qn + __popc(bal & lt_mask)) & (kQCap - 1);
-      if (need) {
-        qw[pos] = make_float4(w[0], w[1], w[2], w[3]);
-        qg[pos] = g;
-      }
-      qn += __popc(bal);
-      __syncwarp();
-      if (qn >= 32) {
-        const int e = (qh + lane) & (kQCap - 1);
-        const float4 ww = qw[e];
-        const int gg = qg[e];
-        qh = (qh + 32) & (kQCap - 1);
-        qn -= 32;
-        __syncwarp();  // entries read before later rounds overwrite them
-        race_block(race, ww, ps.block(gg), 4 * gg);
+    bool need[U];
+    unsigned bal[U];
+    bool dense = qn == 0;
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const float wm = fmaxf(fmaxf(w[u].x, w[u].y), fmaxf(w[u].z, w[u].w));
+      need[u] = wm * 16777216.0f > race.lo;
+      bal[u] = __ballot_sync(0xffffffffu, need[u]);
+      dense = dense && bal[u] == 0xffffffffu;
+    }
+    if (dense) {
+      uint4 rnd[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) rnd[u] = key.block(g[u]);  // independent chains
+#pragma unroll
+      for (int u = 0; u < U; ++u) race_block(race, w[u], rnd[u], 4 * g[u]);
+    } else {
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        if (!bal[u]) continue;  // uniform over the warp
+        const int pos = (qh + qn + __popc(bal[u] & lt_mask)) & (kQCap - 1);
+        if (need[u]) {
+          qw[pos] = w[u];
+          qg[pos] = g[u];
+        }
+        qn += __popc(bal[u]);
+        __syncwarp();
+        if (qn >= 32) {
+          flush_queue(race, qw, qg, qh, 32, key);
+          qh = (qh + 32) & (kQCap - 1);
+          qn -= 32;
+        }
       }
     }
     race.lo = warp_max(race.lo);
@@ -705,266 +676,80 @@ __device__ void race_chunk(const SingleParams& f, const SeqInfo& si, int b, int 
       published = race.lo;
     }
   }
-  if (qn > 0) {  // the rest of the queue
-    const int e = (qh + lane) & (kQCap - 1);
-    const float4 ww = lane < qn ? qw[e] : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-    const int gg = lane < qn ? qg[e] : 0;
-    __syncwarp();
-    if (lane < qn) race_block(race, ww, ps.block(gg), 4 * gg);
-  }
+  if (qn > 0) flush_queue(race, qw, qg, qh, qn, key);  // the rest of the queue
 }
 
-// --------------------------------------------------------------- consumers
-// Bounded wait for sequence b's decision flag (thread 0).  Returns the flag,
-// or 0 when the wait ran out of time (then the kernel's error word is set).
-__device__ __forceinline__ unsigned wait_decision(const SingleParams& f, int b) {
-  unsigned v = ld_acquire(f.ready + b);
-  if (v) return v;
-  const uint64_t t0 = global_ns();
-  for (uint32_t it = 0;; ++it) {
-    __nanosleep(it < 64 ? 32 : 128);
-    v = ld_acquire(f.ready + b);
-    if (v) return v;
-    if (global_ns() - t0 > kWaitLimitNs) break;
-  }
-  atomicExch(f.ctl + kCtlError, 2u);
-  return 0;
-}
-
-// A draw item: chunk `chunk` of sequence b's race, and, in the CTA that
-// completes the sequence's draw items, the combined winner (the token) and
-// the reset of the sequence's flags for the next call.
 template <bool kBf16>
-__device__ void draw_item(const SingleParams& f, int b, int chunk, VerifySmem& sm) {
+__global__ void __launch_bounds__(kDrawThreads, 4) draw_kernel(const __grid_constant__ SingleParams f) {
+  __shared__ float4 scratch[kDrawThreads / 32];
+  __shared__ float4 qw[kDrawThreads / 32][kQCap];  // per-warp race queues
+  __shared__ int qg[kDrawThreads / 32][kQCap];
+  __shared__ int s_last;
+  pdl_wait_and_release();  // the row kernel has completed: every decision is visible
+  const int b = blockIdx.x / f.nc2;
+  const int chunk = blockIdx.x - b * f.nc2;
+  const int warp = threadIdx.x >> 5;
   const CallParams& p = f.p1;
-  const int tid = threadIdx.x;
-  if (tid == 0) {
-    const unsigned flag = wait_decision(f, b);
-    SeqInfo si{};
-    if (flag) {
-      const float4* ip = reinterpret_cast<const float4*>(p.info + b);
-      const float4 w0 = __ldcg(ip), w1 = __ldcg(ip + 1);
-      si.mode = __float_as_int(w0.x);
-      si.j = __float_as_int(w0.y);
-      si.zmp = w0.z;
-      si.zmq = w0.w;
-      si.c = w1.x;
-      si.lsp = w1.y;
-      si.lsq = w1.z;
-    } else {
-      si.mode = kModeNone;  // the decision never came: mark the sequence invalid
-      p.accept_len[b] = -1;
-      for (int i = 0; i <= p.gamma; ++i) p.out_tokens[static_cast<size_t>(b) * (p.gamma + 1) + i] = -1;
-    }
-    sm.info = si;
-  }
-  block_sync<kCThreads>();
-  const SeqInfo si = sm.info;
+  const float4* ip = reinterpret_cast<const float4*>(p.info + b);
+  const float4 w0 = __ldcg(ip), w1 = __ldcg(ip + 1);
+  SeqInfo si{};
+  si.mode = __float_as_int(w0.x);
+  si.j = __float_as_int(w0.y);
+  si.zmp = w0.z;
+  si.zmq = w0.w;
+  si.c = w1.x;
+  si.lsp = w1.y;
+  si.lsq = w1.z;
   const bool draw = (si.mode == kModeResidual && si.j >= 0 && si.j < p.gamma) ||
                     (si.mode == kModeBonus && si.j == p.gamma);
+  if (!draw) return;  // uniform: greedy or invalid sequence
   Race race;
   race.reset();
-  if (draw) {
-    // bonus draw: the entry at the row maximum has weight 2^-lsp and E < 17,
-    // so its ratio -- and the winner's -- exceeds 2^-lsp / 17
-    if (si.mode == kModeBonus) race.lo = ex2_approx(-si.lsp) * (1.0f / 17.0f);
-    race_chunk<kBf16>(f, si, b, chunk, f.nd, f.bar + b, race, sm);
-  }
+  // bonus draw: the entry at the row maximum has weight 2^-lsp and E < 17, so
+  // its ratio -- and the winner's -- exceeds 2^-lsp / 17
+  if (si.mode == kModeBonus) race.lo = ex2_approx(-si.lsp) * (1.0f / 17.0f);
+  race_span<kBf16>(f, si, b, chunk, f.nc2, f.bar + b, race, qw[warp], qg[warp]);
   float bw = race.bw, be = race.be;
   int bi = race.bi;
-  race_reduce<kCThreads>(bw, be, bi, sm.race);
-  if (tid == 0) {
-    RacePartial* pp = f.part2 + static_cast<size_t>(b) * f.nd + chunk;
+  race_reduce<kDrawThreads>(bw, be, bi, scratch);
+  if (threadIdx.x == 0) {
+    RacePartial* pp = f.part2 + static_cast<size_t>(b) * f.nc2 + chunk;
     *reinterpret_cast<float4*>(pp) = make_float4(bw, be, __int_as_float(bi), 0.0f);
     const unsigned t = ticket_acq_rel(f.ticket2 + b);
-    sm.last = (t == static_cast<unsigned>(f.nd - 1));
-  }
-  block_sync<kCThreads>();  // orders the other threads after thread 0's acquire
-  if (!sm.last) return;
-  if (draw) {
-    bw = 0.0f;
-    be = 1.0f;
-    bi = INT_MAX;
-    for (int q = tid; q < f.nd; q += kCThreads) {
-      const float4 g = __ldcg(reinterpret_cast<const float4*>(f.part2 + static_cast<size_t>(b) * f.nd + q));
-      if (race_better(g.x, g.y, __float_as_int(g.z), bw, be, bi)) {
-        bw = g.x;
-        be = g.y;
-        bi = __float_as_int(g.z);
-      }
-    }
-    race_reduce<kCThreads>(bw, be, bi, sm.race);
-    if (!(bw > 0.0f)) {  // uniform: race_reduce returns the winner to every thread
-      // the residual vanished (p_j == q_j to rounding): draw from p_j instead,
-      // over the whole row in this CTA (without the residual race's bar)
-      SeqInfo sb = si;
-      sb.mode = kModeBonus;
-      race.reset();
-      race.lo = ex2_approx(-sb.lsp) * (1.0f / 17.0f);
-      race_chunk<kBf16>(f, sb, b, 0, 1, nullptr, race, sm);
-      bw = race.bw;
-      be = race.be;
-      bi = race.bi;
-      race_reduce<kCThreads>(bw, be, bi, sm.race);
-    }
-    if (tid == 0) p.out_tokens[static_cast<size_t>(b) * (p.gamma + 1) + si.j] = bi;
-  }
-  if (tid == 0) {  // every chunk of b is past its wait and its race
-    f.ready[b] = 0u;
-    f.bar[b] = 0u;
-    f.ticket2[b] = 0u;
-  }
-}
-
-// Per-item state of a row item, set up at its first tile.
-template <bool kBf16>
-struct RowItem {
-  int b, i, seg;
-  float T, c;
-  bool argmaxA, loadA, loadB;
-  int xg, ownA, ownB;
-  const char* rpA;
-  const char* rpB;
-  RowGeom<kBf16> gA, gB;
-  __device__ __forceinline__ RowItem(const SingleParams& f, const TileDesc& d)
-      : b(d.b), i(d.i), seg(d.seg), T(d.T), xg(d.xg),
-        rpA(target_row<kBf16>(f.p1, d.b, d.i)),
-        rpB(d.i < f.p1.gamma ? draft_row<kBf16>(f.p1, d.b, d.i) : rpA),
-        gA(rpA, f.p1.V), gB(rpB, f.p1.V) {
-    const int modeA = row_mode(T, true);
-    argmaxA = modeA == kRowArgmax;
-    loadA = modeA != kRowSkip;
-    loadB = i < f.p1.gamma && row_mode(T, false) == kRowLse;
-    c = modeA == kRowLse ? __fdiv_rn(kLog2e, T) : 0.0f;
-    const int k0 = seg * f.segvec;
-    ownA = owned_vector<kBf16>(gA, xg, k0, min(gA.nvec, k0 + f.segvec));
-    ownB = owned_vector<kBf16>(gB, xg, k0, min(gB.nvec, k0 + f.segvec));
-  }
-};
-
-// The end of a row item: row edges, the consumer-wide reduction, the partial
-// and the arrival ticket; the CTA that completes the sequence decides.
-template <bool kBf16>
-__device__ void row_item_end(const SingleParams& f, const RowItem<kBf16>& it, RunAcc& accA, RunAcc& accB,
-                             float2 z, VerifySmem& sm) {
-  const CallParams& p = f.p1;
-  const int tid = threadIdx.x;
-  const bool first = it.seg == 0, last = it.seg == f.nseg - 1;
-  if (it.loadA && (first || last))
-    row_edges<kBf16>(it.rpA, p.V, it.gA, it.argmaxA, it.c, first, last, it.xg, z.x, accA);
-  if (it.loadB && (first || last))
-    row_edges<kBf16>(it.rpB, p.V, it.gB, false, it.c, first, last, it.xg, z.y, accB);
-  RowAcc A = it.argmaxA ? accA.argmax_row() : accA.lse_row(), B = accB.lse_row();
-  reduce_pair(A, B, z, it.argmaxA, sm);
-  if (tid == 0) {
-    float4* pp = f.pairpart + ((static_cast<size_t>(it.b) * (p.gamma + 1) + it.i) * f.nseg + it.seg) * 2;
-    pp[0] = make_float4(A.m, A.s, __int_as_float(A.arg), __int_as_float(A.bad));
-    pp[1] = make_float4(B.m, B.s, __int_as_float(B.arg), __int_as_float(B.bad));
-    if (it.i < p.gamma) {
-      float* zz = f.zx + ((static_cast<size_t>(it.b) * p.gamma + it.i) * f.nseg + it.seg) * 2;
-      zz[0] = z.x;
-      zz[1] = z.y;
-    }
-    // release this item's partial; the last arriver also acquires the others'
-    const unsigned tk = ticket_acq_rel(p.ticket + it.b);
-    const unsigned arrivals = static_cast<unsigned>(f.nr);
-    sm.last = (tk == arrivals - 1);
-    if (sm.last) p.ticket[it.b] = 0;  // leave the counter at zero for the next call
-  }
-  block_sync<kCThreads>();  // orders the other threads after thread 0's acquire
-  if (!sm.last) return;
-  for (int k = tid; k < p.gamma; k += kCThreads)
-    sm.tok[k] = __ldg(p.tokens + static_cast<size_t>(it.b) * p.gamma + k);
-  combine_pairs(f, it.b, it.argmaxA, it.c, sm);  // ends with a consumer barrier
-  if (tid < 32) decide_single<kBf16>(p, it.b, it.T, sm.tok, sm.rows, sm.zsel, f.ready);
-  block_sync<kCThreads>();  // sm.rows / sm.tok are reused by the next decision
-}
-
-template <bool kBf16>
-__device__ void consume(const SingleParams& f, VerifySmem& sm, const char* ring) {
-  const int tid = threadIdx.x;
-  int stage = 0;
-  uint32_t phase = 0;
-  RunAcc accA, accB;
-  accA.reset();
-  accB.reset();
-  float2 z = make_float2(__int_as_float(0x7fc00000), __int_as_float(0x7fc00000));
-  // the current row item (rebuilt at each item's first tile)
-  RowItem<kBf16> it(f, TileDesc{kItemRow, 0, 0, 0, 0, 0, 0, 0, 0.0f, -1, 0, 0});
-  for (;;) {
-    if (!mbar_wait(&sm.full[stage], phase)) {
-      if (tid == 0) atomicExch(f.ctl + kCtlError, 3u);
-      return;
-    }
-    const TileDesc d = sm.desc[stage];
-    if (d.kind == kItemEnd) return;
-    const char* st = ring + stage * kStageBytes;
-    if (d.kind == kItemDraw) {
-      __syncwarp();
-      if ((tid & 31) == 0) mbar_arrive(&sm.empty[stage]);
-      if (++stage == kStages) { stage = 0; phase ^= 1u; }
-      draw_item<kBf16>(f, d.b, d.i, sm);
-      continue;
-    }
-    if (d.flags & kFirstTile) {
-      it = RowItem<kBf16>(f, d);
-      accA.reset();
-      accB.reset();
-      z = make_float2(__int_as_float(0x7fc00000), __int_as_float(0x7fc00000));
-    }
-    uint4 ra[kTileRegs], rb[kTileRegs];
-    stage_tile<kBf16>(st, d.nvA, ra);
-    stage_tile<kBf16>(st + kSlotBytes, d.nvB, rb);
-    __syncwarp();
-    if ((tid & 31) == 0) mbar_arrive(&sm.empty[stage]);  // the stage may be refilled
-    if (++stage == kStages) { stage = 0; phase ^= 1u; }
-    if (d.nvA) {
-      pick_logit<kBf16>(ra, it.ownA, d.kb, it.xg, it.gA, z.x);
-      if (it.argmaxA)
-        argmax_tile<kBf16>(accA, ra, it.gA.head + (d.kb + tid) * Vec16<kBf16>::kN);
-      else
-        lse_tile<kBf16>(accA, ra, it.c);
-    }
-    if (d.nvB) {
-      pick_logit<kBf16>(rb, it.ownB, d.kb, it.xg, it.gB, z.y);
-      lse_tile<kBf16>(accB, rb, it.c);
-    }
-    if (d.flags & kLastTile) row_item_end<kBf16>(f, it, accA, accB, z, sm);
-  }
-}
-
-// --------------------------------------------------------------- the kernel
-template <bool kBf16>
-__global__ void __launch_bounds__(kVThreads, 2) verify_kernel(const __grid_constant__ SingleParams f) {
-  extern __shared__ __align__(128) char ring[];
-  __shared__ VerifySmem sm;
-  const int tid = threadIdx.x;
-  if (tid == 0) {
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(&sm.full[s], 1);
-      mbar_init(&sm.empty[s], kCWarps);
-    }
-    mbar_init_fence();
-  }
-  __syncthreads();
-  // the previous grid in the stream has completed (programmatic dependent
-  // launch); the next may start launching its CTAs
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  asm volatile("griddepcontrol.launch_dependents;");
-  if (tid >= kCThreads) {
-    if (tid == kCThreads) produce<kBf16>(f, sm, ring);
-    return;
-  }
-  consume<kBf16>(f, sm, ring);
-  block_sync<kCThreads>();
-  if (tid == 0) {
-    // the last CTA to leave returns the work counter to zero for the next call
-    const unsigned t = ticket_acq_rel(f.ctl + kCtlExit);
-    if (t == gridDim.x - 1) {
-      f.ctl[kCtlNext] = 0u;
-      f.ctl[kCtlExit] = 0u;
+    s_last = (t == static_cast<unsigned>(f.nc2 - 1));
+    if (s_last) {
+      f.ticket2[b] = 0;
+      f.bar[b] = 0;  // every CTA of the sequence is past its race
     }
   }
+  block_sync<kDrawThreads>();  // orders the other threads after thread 0's acquire
+  if (!s_last) return;
+  bw = 0.0f;
+  be = 1.0f;
+  bi = INT_MAX;
+  for (int q = threadIdx.x; q < f.nc2; q += kDrawThreads) {
+    const float4 g = __ldcg(reinterpret_cast<const float4*>(f.part2 + static_cast<size_t>(b) * f.nc2 + q));
+    if (race_better(g.x, g.y, __float_as_int(g.z), bw, be, bi)) {
+      bw = g.x;
+      be = g.y;
+      bi = __float_as_int(g.z);
+    }
+  }
+  race_reduce<kDrawThreads>(bw, be, bi, scratch);
+  if (!(bw > 0.0f)) {  // uniform: race_reduce returns the winner to every thread
+    // the residual vanished (p_j == q_j to rounding): draw from p_j instead,
+    // over the whole row in this CTA (without the residual race's bar)
+    SeqInfo sb = si;
+    sb.mode = kModeBonus;
+    race.reset();
+    race.lo = ex2_approx(-sb.lsp) * (1.0f / 17.0f);
+    race_span<kBf16>(f, sb, b, 0, 1, nullptr, race, qw[warp], qg[warp]);
+    bw = race.bw;
+    be = race.be;
+    bi = race.bi;
+    race_reduce<kDrawThreads>(bw, be, bi, scratch);
+  }
+  if (threadIdx.x == 0) p.out_tokens[static_cast<size_t>(b) * (p.gamma + 1) + si.j] = bi;
 }
 
 // ------------------------------------------------------------------ launch
@@ -978,10 +763,10 @@ int body_tiles(int V, int dtype) {  // tiles of kTileVec vectors covering a row'
 
 int row_segments(int V, int dtype) { return body_tiles(V, dtype); }  // bound on segments per row
 
-int draw_chunks(int V, int dtype) {  // upper bound on draw items per sequence
+int draw_chunks(int B, int V, int dtype) {  // upper bound on draw CTAs per sequence
+  (void)B;
   (void)dtype;
-  const int nb = (V + 3) / 4;
-  return (nb + kRaceRound - 1) / kRaceRound;
+  return (V + 255) / 256;
 }
 
 namespace {
@@ -1013,35 +798,36 @@ int sm_count() {
   });
 }
 
-// Opt the kernel into its dynamic shared memory (once per device) and return
-// its resident CTAs per SM (0 if the attribute could not be set).
 template <typename Kernel>
-int prepare(Kernel kernel) {
-  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kRingBytes) !=
-      cudaSuccess) {
-    (void)cudaGetLastError();
-    return 0;
-  }
+int occupancy(Kernel kernel, int threads) {
   int n = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, kVThreads, kRingBytes) != cudaSuccess) {
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, threads, 0) != cudaSuccess) {
     (void)cudaGetLastError();
     return 0;
   }
   return n;
 }
 
-int ctas_per_sm(bool bf16) {
+// Resident row-kernel CTAs per SM.
+int row_ctas_per_sm(bool bf16) {
   static std::atomic<int> slots[2][64];
-  return bf16 ? per_device(slots[1], -1, [](int) { return prepare(verify_kernel<true>); })
-              : per_device(slots[0], -1, [](int) { return prepare(verify_kernel<false>); });
+  return bf16 ? per_device(slots[1], 3, [](int) { return occupancy(rows_kernel<true>, kRowThreads); })
+              : per_device(slots[0], 3, [](int) { return occupancy(rows_kernel<false>, kRowThreads); });
+}
+
+// Resident draw-kernel CTAs per SM.
+int draw_ctas_per_sm(bool bf16) {
+  static std::atomic<int> slots[2][64];
+  return bf16 ? per_device(slots[1], 4, [](int) { return occupancy(draw_kernel<true>, kDrawThreads); })
+              : per_device(slots[0], 4, [](int) { return occupancy(draw_kernel<false>, kDrawThreads); });
 }
 
 template <typename K>
-cudaError_t launch_pdl(K kernel, unsigned grid, cudaStream_t stream, const SingleParams& f) {
+cudaError_t launch_pdl(K kernel, dim3 grid, unsigned block, cudaStream_t stream,
+                       const SingleParams& f) {
   cudaLaunchConfig_t cfg{};
-  cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(kVThreads);
-  cfg.dynamicSmemBytes = kRingBytes;
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(block);
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -1063,11 +849,6 @@ int launch_single(const void* target, const void* draft, const int32_t* tokens,
                   uint64_t step, int32_t* out_accept_len, int32_t* out_tokens, float* out_lp,
                   float* out_lq, void* workspace, const Layout& lay, cudaStream_t stream) {
   char* ws = static_cast<char*>(workspace);
-  const bool bf16 = dtype == SV_BF16;
-  const int per_sm = ctas_per_sm(bf16);
-  if (per_sm <= 0)
-    return set_error(SV_ERR_CUDA, "verification kernel cannot be made resident (%d CTAs per SM)",
-                     per_sm);
   SingleParams f{};
   CallParams& p1 = f.p1;
   p1.target = target;
@@ -1086,59 +867,61 @@ int launch_single(const void* target, const void* draft, const int32_t* tokens,
   p1.out_tokens = out_tokens;
   p1.out_lp = out_lp;
   p1.out_lq = out_lq;
-  f.pairpart = reinterpret_cast<float4*>(ws + lay.part1);
-  f.zx = reinterpret_cast<float*>(ws + lay.resid);
-  f.part2 = reinterpret_cast<RacePartial*>(ws + lay.part2);
-  f.ticket2 = reinterpret_cast<unsigned*>(ws + lay.ticket2);
-  f.ready = reinterpret_cast<unsigned*>(ws + lay.ready);
-  f.bar = reinterpret_cast<unsigned*>(ws + lay.bar);
-  f.ctl = reinterpret_cast<unsigned*>(ws + lay.ctl);
-  const long long ctas = static_cast<long long>(sm_count()) * per_sm;
-
-  // Row segments: whole tiles, at most kMaxSegTiles per item, about
-  // kItemsPerCta row items per CTA for balance; balanced so that segments
-  // differ by at most one tile.
+  // Row segments: whole tiles, about kRowWaves waves of CTAs over the GPU but
+  // at most kMaxSegTiles tiles per CTA; balanced so segments differ by at
+  // most one tile.  Long segments spread each CTA's fixed cost (launch, block
+  // reduce, ticket) over more streaming; about three waves keep the last one
+  // mostly full.
+  const bool bf16 = dtype == SV_BF16;
   {
-    constexpr int kMaxSegTiles = 4, kItemsPerCta = 4;
+    constexpr int kRowWaves = 3, kMaxSegTiles = 10;
     const int tiles = body_tiles(V, dtype);
     const long long pairs = static_cast<long long>(B) * (gamma + 1);
-    long long st = pairs * tiles / (kItemsPerCta * ctas);
+    const long long slots = static_cast<long long>(sm_count()) * row_ctas_per_sm(bf16);
+    long long st = pairs * tiles / (kRowWaves * slots);
     st = st < 1 ? 1 : (st > kMaxSegTiles ? kMaxSegTiles : st);
     int nseg = static_cast<int>((tiles + st - 1) / st);
     if (nseg > lay.nc) nseg = lay.nc;
+    if (nseg > 65535) nseg = 65535;  // gridDim.y
     st = (tiles + nseg - 1) / nseg;
     f.nseg = nseg;
     f.segvec = static_cast<int>(st) * kTileVec;
   }
-  // Draw items: about kDrawBlocks Philox blocks per consumer thread each.
+  f.pairpart = reinterpret_cast<float4*>(ws + lay.part1);
+  f.zx = reinterpret_cast<float*>(ws + lay.resid);
+  f.part2 = reinterpret_cast<RacePartial*>(ws + lay.part2);
+  f.ticket2 = reinterpret_cast<unsigned*>(ws + lay.ticket2);
+  f.bar = reinterpret_cast<unsigned*>(ws + lay.bar);
+  // Draw chunks: a whole number of waves of the draw kernel over the GPU,
+  // with at most about kDrawMaxBlocks Philox blocks per thread; chunks are
+  // balanced within a sequence (in Philox blocks of 4 entries).
   {
-    constexpr int kDrawBlocks = 16;
-    const long long nb = (V + 3) / 4;
-    long long nd = (nb + static_cast<long long>(kDrawBlocks) * kRaceRound - 1) /
-                   (static_cast<long long>(kDrawBlocks) * kRaceRound);
-    const long long rounds = (nb + kRaceRound - 1) / kRaceRound;  // every chunk has a round
-    if (nd > rounds) nd = rounds;
-    if (nd < 1) nd = 1;
-    if (nd > lay.nc2) nd = lay.nc2;
-    f.nd = static_cast<int>(nd);
+    const long long nb = (V + 3) / 4;  // Philox blocks per row
+    const long long slots2 = static_cast<long long>(sm_count()) * draw_ctas_per_sm(bf16);
+    const long long per_cta = static_cast<long long>(kDrawMaxBlocks) * kDrawThreads;
+    const long long waves = (static_cast<long long>(B) * nb + per_cta * slots2 - 1) / (per_cta * slots2);
+    long long nc2 = waves * slots2 / B;
+    if (nc2 < 1) nc2 = 1;
+    if (nc2 > lay.nc2) nc2 = lay.nc2;
+    if (nc2 > nb) nc2 = nb;
+    const long long cb = (nb + nc2 - 1) / nc2;  // blocks per draw CTA
+    f.chunk2 = static_cast<int>(4 * cb);
+    f.nc2 = static_cast<int>((nb + cb - 1) / cb);
   }
-  f.nr = (gamma + 1) * f.nseg;
-  // Lag: two CTA-loads of row items between a sequence's rows and its draws.
-  {
-    long long lag = (2 * ctas + f.nr - 1) / f.nr;
-    if (lag > B) lag = B;
-    if (lag < 1) lag = 1;
-    f.lag = static_cast<int>(lag);
-  }
-  const long long total = static_cast<long long>(B) * (f.nr + f.nd);
-  if (total > INT_MAX / 2)
-    return set_error(SV_ERR_INVALID_ARG, "B x V too large for one launch (%lld work items)", total);
-  f.total = static_cast<int>(total);
-  const unsigned grid = static_cast<unsigned>(total < ctas ? total : ctas);
-  const cudaError_t e = bf16 ? launch_pdl(verify_kernel<true>, grid, stream, f)
-                             : launch_pdl(verify_kernel<false>, grid, stream, f);
+
+  if (static_cast<long long>(B) * f.nc2 > INT_MAX)
+    return set_error(SV_ERR_INVALID_ARG, "B x V too large for one launch (draw grid %lld CTAs)",
+                     static_cast<long long>(B) * f.nc2);
+  const dim3 grid1(static_cast<unsigned>(B * (gamma + 1)), static_cast<unsigned>(f.nseg));
+  cudaError_t e = bf16 ? launch_pdl(rows_kernel<true>, grid1, kRowThreads, stream, f)
+                       : launch_pdl(rows_kernel<false>, grid1, kRowThreads, stream, f);
   if (e != cudaSuccess)
-    return set_error(SV_ERR_CUDA, "verification kernel launch failed: %s", cudaGetErrorString(e));
+    return set_error(SV_ERR_CUDA, "row kernel launch failed: %s", cudaGetErrorString(e));
+  const dim3 grid2(static_cast<unsigned>(static_cast<long long>(B) * f.nc2));
+  e = bf16 ? launch_pdl(draw_kernel<true>, grid2, kDrawThreads, stream, f)
+           : launch_pdl(draw_kernel<false>, grid2, kDrawThreads, stream, f);
+  if (e != cudaSuccess)
+    return set_error(SV_ERR_CUDA, "draw kernel launch failed: %s", cudaGetErrorString(e));
   return check_launch("verify");
 }
 

@@ -1,10 +1,10 @@
-// sv_stream.cuh -- per-thread row reductions of the single-draft row kernel.
+// sv_stream.cuh -- per-thread row reductions of the single-draft row items.
 //
-// A row-kernel CTA covers (sequence b, position i, vocabulary segment): target
-// row i and draft row i over the same segment (position gamma: the target row
-// alone).  The segment is walked in tiles of kTileVec 16-byte vectors; each
-// thread loads its kTileRegs vectors of a tile into registers, then folds
-// them into a running accumulator.
+// A row item covers (sequence b, position i, vocabulary segment): target row i
+// and draft row i over the same segment (position gamma: the target row
+// alone).  The segment arrives in tiles of kTileVec 16-byte vectors per row;
+// each thread copies its kTileRegs vectors of a tile into registers, then
+// folds them into a running accumulator.
 //
 // Softmax sums use an integer reference exponent.  With c = log2(e) / T and
 // R(m) = ceil(fl(m c)) for the running maximum m, a thread accumulates
