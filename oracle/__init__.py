@@ -27,6 +27,8 @@ _LIB_PATH = os.path.join(_HERE, "libsvoracle.so")
 
 F32, BF16 = 0, 1
 TAG_ACCEPT, TAG_GUMBEL, TAG_MD_ETA, TAG_MD_GUMBEL = 1, 2, 3, 4
+TAG_GROUP = 7
+RACE_GROUP = 1024  # vocabulary entries per group of the single-draft two-level race
 TIE_BERNOULLI, TIE_GUMBEL = 1, 2
 
 _lock = threading.Lock()
@@ -81,6 +83,8 @@ def lib():
             L.svo_residual_logw.restype = i64
             L.svo_gumbel_argmax.argtypes = [vp, i64, u64, u64, u32, u32, u32, vp]
             L.svo_gumbel_argmax.restype = i64
+            L.svo_group_race.argtypes = [vp, i64, u64, u64, u32, u32, u32, vp]
+            L.svo_group_race.restype = i64
             L.svo_verify.argtypes = [vp, vp, vp, vp, i64, C.c_int, i64, C.c_int, u64, u64,
                                      i64, i64, vp, vp, vp, vp, vp, C.POINTER(Rng)]
             L.svo_verify.restype = C.c_int
@@ -169,6 +173,14 @@ def gumbel_argmax(logw: np.ndarray, seed, step, tag, b, pos):
     logw = np.ascontiguousarray(logw, dtype=np.float64)
     gap = np.zeros(1, dtype=np.float64)
     y = lib().svo_gumbel_argmax(_ptr(logw), logw.size, seed, step, tag, b, pos, _ptr(gap))
+    return int(y), float(gap[0])
+
+
+def group_race(logw: np.ndarray, seed, step, tag, b, pos):
+    """The single-draft draw: two-level exponential race (groups of RACE_GROUP)."""
+    logw = np.ascontiguousarray(logw, dtype=np.float64)
+    gap = np.zeros(1, dtype=np.float64)
+    y = lib().svo_group_race(_ptr(logw), logw.size, seed, step, tag, b, pos, _ptr(gap))
     return int(y), float(gap[0])
 
 

@@ -192,6 +192,74 @@ int64_t svo_gumbel_argmax(const double* logw, int64_t V, uint64_t seed, uint64_t
   return arg;
 }
 
+/* Reading of the draw "from r(.)" ([SSD] s.2): any exact sampler of the
+ * normalised weights qualifies; the single-draft draw takes a two-level
+ * exponential race.  With W_g the summed weight of group g and E_g, E_v
+ * independent unit exponentials, the group g* maximising W_g / E_g is g with
+ * probability W_g / W (the minimum of independent exponential clocks of
+ * rates W_g), and the entry maximising w_v / E_v within g* is v with
+ * probability w_v / W_g* (the same property within the group), so v is drawn
+ * with probability w_v / W.  The group noise uses its own tag, so the two
+ * levels are independent.  In log space: ln W_g - ln E_g and logw_v - ln E_v. */
+static double group_exponential(uint64_t seed, uint64_t step, uint32_t b, uint32_t pos,
+                                int64_t g) {
+  const uint32_t x = svo_stream_word(seed, step, SVO_TAG_GROUP, b, 0, pos, (uint32_t)g, 0);
+  return -log1p(-(1.0 - svo_u01_gumbel(x)));
+}
+
+static double entry_exponential(uint64_t seed, uint64_t step, uint32_t tag, uint32_t b,
+                                uint32_t pos, int64_t v) {
+  const uint32_t x =
+      svo_stream_word(seed, step, tag, b, 0, pos, (uint32_t)(v >> 2), (uint32_t)(v & 3));
+  return -log1p(-(1.0 - svo_u01_gumbel(x)));
+}
+
+int64_t svo_group_race(const double* logw, int64_t V, uint64_t seed, uint64_t step,
+                       uint32_t tag, uint32_t b, uint32_t pos, double* gap) {
+  const int64_t G = SVO_RACE_GROUP;
+  const int64_t ng = (V + G - 1) / G;
+  /* level 1: the groups */
+  double best = -INFINITY, second = -INFINITY;
+  int64_t gbest = -1;
+  for (int64_t g = 0; g < ng; ++g) {
+    double W = 0.0;
+    for (int64_t v = g * G; v < V && v < (g + 1) * G; ++v)
+      if (logw[v] != -INFINITY) W += exp(logw[v]);
+    if (!(W > 0.0)) continue;
+    const double score = log(W) - log(group_exponential(seed, step, b, pos, g));
+    if (gbest < 0 || score > best) {
+      second = best;
+      best = score;
+      gbest = g;
+    } else if (score > second) {
+      second = score;
+    }
+  }
+  if (gbest < 0) {
+    if (gap) *gap = INFINITY;
+    return -1;
+  }
+  const double ggap = second > -INFINITY ? best - second : INFINITY;
+  /* level 2: the entries of the winning group */
+  best = -INFINITY;
+  second = -INFINITY;
+  int64_t arg = -1;
+  for (int64_t v = gbest * G; v < V && v < (gbest + 1) * G; ++v) {
+    if (logw[v] == -INFINITY) continue;
+    const double score = logw[v] - log(entry_exponential(seed, step, tag, b, pos, v));
+    if (arg < 0 || score > best) {
+      second = best;
+      best = score;
+      arg = v;
+    } else if (score > second) {
+      second = score;
+    }
+  }
+  const double egap = second > -INFINITY ? best - second : INFINITY;
+  if (gap) *gap = ggap < egap ? ggap : egap;
+  return arg;
+}
+
 /* ------------------------------------------------------------------------
  * Default randomness: Philox uniforms.
  * ---------------------------------------------------------------------- */
@@ -212,15 +280,47 @@ typedef struct {
  * its band widens by (p + q) / (p - q).  lq == NULL: bonus draw. */
 static double prob_eta(double lp) { return 2e-6 + 2e-7 * fabs(lp); }
 
+/* Group level of the same rule: an fp32 group sum lies within
+ * [W_g^-, W_g^+], where each weight is moved by its evaluation error
+ * d_v = eta_p p_v + eta_q q_v (and clipped at zero, so entries with p <= q
+ * that rounding could make positive are counted) and the sum by its own
+ * rounding (relative GROUP_SUM_ETA: a sum of non-negative fp32 terms of
+ * depth at most 64).  The draw is logged when another group's score
+ * ln W^+ - ln E could reach the winning group's ln W^- - ln E, each also
+ * moved by half the fixed band. */
+#define GROUP_SUM_ETA (64.0 * 0x1p-24)
+
 static int draw_fragile(const double* lw, const double* lp, const double* lq, int64_t V,
                         const philox_ctx* pc, uint32_t b, uint32_t pos, int64_t y) {
   if (y < 0) return 0;
+  const int64_t G = SVO_RACE_GROUP;
+  const int64_t ng = (V + G - 1) / G;
+  const int64_t gy = y / G;
+  double lo_y = -INFINITY, hi_other = -INFINITY;
+  for (int64_t g = 0; g < ng; ++g) {
+    double Wlo = 0.0, Whi = 0.0;
+    for (int64_t v = g * G; v < V && v < (g + 1) * G; ++v) {
+      const double p = exp(lp[v]);
+      const double q = lq ? exp(lq[v]) : 0.0;
+      const double d = prob_eta(lp[v]) * p + (lq ? prob_eta(lq[v]) * q : 0.0);
+      const double w = p - q;
+      if (w - d > 0.0) Wlo += w - d;
+      if (w + d > 0.0) Whi += w + d;
+    }
+    const double lnE = log(group_exponential(pc->seed, pc->step, b, pos, g));
+    if (g == gy) {
+      lo_y = Wlo > 0.0 ? log(Wlo * (1.0 - GROUP_SUM_ETA)) - lnE - 0.5 * GUMBEL_TIE_BAND : -INFINITY;
+    } else if (Whi > 0.0) {
+      const double hi = log(Whi * (1.0 + GROUP_SUM_ETA)) - lnE + 0.5 * GUMBEL_TIE_BAND;
+      if (hi > hi_other) hi_other = hi;
+    }
+  }
+  if (hi_other > -INFINITY && hi_other >= lo_y) return 1; /* no competitor: no group flip */
+  /* entry level, within the winning group */
   double sy = -INFINITY, uy = 0.0, other = -INFINITY;
-  for (int64_t v = 0; v < V; ++v) {
+  for (int64_t v = gy * G; v < V && v < (gy + 1) * G; ++v) {
     if (lw[v] == -INFINITY) continue;
-    const uint32_t x = svo_stream_word(pc->seed, pc->step, SVO_TAG_GUMBEL, b, 0, pos,
-                                       (uint32_t)(v >> 2), (uint32_t)(v & 3));
-    const double E = -log1p(-(1.0 - svo_u01_gumbel(x)));
+    const double E = entry_exponential(pc->seed, pc->step, SVO_TAG_GUMBEL, b, pos, v);
     const double score = lw[v] - log(E);
     const double p = exp(lp[v]);
     const double q = lq ? exp(lq[v]) : 0.0;
@@ -248,6 +348,8 @@ static int philox_coin(void* ctx, double h, uint32_t tag, uint32_t b, uint32_t k
 static int64_t philox_categorical(void* ctx, const double* logw, int64_t V, uint32_t tag,
                                   uint32_t b, uint32_t pos, double* gap) {
   const philox_ctx* c = (const philox_ctx*)ctx;
+  /* single-draft draws: the two-level race; multi-draft draws: the plain race */
+  if (tag == SVO_TAG_GUMBEL) return svo_group_race(logw, V, c->seed, c->step, tag, b, pos, gap);
   return svo_gumbel_argmax(logw, V, c->seed, c->step, tag, b, pos, gap);
 }
 

@@ -45,8 +45,13 @@ enum {
   SVO_TAG_ACCEPT = 1,      /* single-draft acceptance uniform             */
   SVO_TAG_GUMBEL = 2,      /* single-draft residual / bonus Gumbel noise   */
   SVO_TAG_MD_ETA = 3,      /* multi-draft sub-block acceptance uniform     */
-  SVO_TAG_MD_GUMBEL = 4    /* multi-draft correction Gumbel noise          */
+  SVO_TAG_MD_GUMBEL = 4,   /* multi-draft correction Gumbel noise          */
+  SVO_TAG_GROUP = 7        /* single-draft group-level race noise          */
 };
+
+/* Vocabulary entries per group of the single-draft two-level race (group g
+ * holds entries [g * SVO_RACE_GROUP, (g + 1) * SVO_RACE_GROUP) of the row). */
+enum { SVO_RACE_GROUP = 1024 };
 
 /* Per-sequence tie flags written to out_tie[b]. */
 enum {
@@ -94,6 +99,16 @@ int64_t svo_residual_logw(const double* lp, const double* lq, int64_t V, double*
 /* Default Gumbel-max draw over logw with the keyed Philox stream. */
 int64_t svo_gumbel_argmax(const double* logw, int64_t V, uint64_t seed, uint64_t step,
                           uint32_t tag, uint32_t b, uint32_t pos, double* gap);
+
+/* Two-level exponential race over logw: group g (SVO_RACE_GROUP entries)
+ * has weight W_g = sum of exp(logw) over its entries and exponential
+ * E_g = -ln U_g, U_g from word 0 of the keyed block (c0 = g) with tag
+ * SVO_TAG_GROUP; the winning group is argmax ln W_g - ln E_g (ties: lowest g);
+ * within it the entry is argmax logw_v - ln E_v with the entry noise of
+ * svo_gumbel_argmax (tag `tag`).  Returns -1 when every weight is zero.
+ * gap = the smaller of the two top-2 score gaps. */
+int64_t svo_group_race(const double* logw, int64_t V, uint64_t seed, uint64_t step,
+                       uint32_t tag, uint32_t b, uint32_t pos, double* gap);
 
 /* ---- single-draft verification ---------------------------------------
  * target [B, gamma+1, V], draft [B, gamma, V] (dtype), tokens [B, gamma],

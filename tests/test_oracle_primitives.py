@@ -137,3 +137,72 @@ def test_gumbel_argmax_deterministic_and_keyed():
     assert a == oracle.gumbel_argmax(logw, 0, 0, oracle.TAG_GUMBEL, 0, 0)[0]
     draws = {oracle.gumbel_argmax(logw, 0, s, oracle.TAG_GUMBEL, 0, 0)[0] for s in range(200)}
     assert len(draws) > 40  # different steps give different keys
+
+
+def test_group_race_law():
+    """The two-level race draws from the normalised weights: entry
+    frequencies over three groups (the last one ragged) against w / W,
+    chi-square over heavy entries at group edges and the rest of each group."""
+    from scipy.stats import chisquare
+    G = oracle.RACE_GROUP
+    V = 2 * G + 300
+    rng = np.random.default_rng(5)
+    w = rng.uniform(0.0, 1.0, V) * 1e-3
+    w[rng.random(V) < 0.3] = 0.0
+    heavy = [0, 5, G - 1, G, 2 * G - 1, 2 * G, V - 1]
+    w[heavy] = [0.4, 0.2, 0.3, 0.25, 0.1, 0.05, 0.15]
+    logw = np.full(V, -np.inf)
+    logw[w > 0] = np.log(w[w > 0])
+    cat = np.full(V, -1)
+    for i, v in enumerate(heavy):
+        cat[v] = i
+    for g in range(3):
+        rest = np.arange(g * G, min(V, (g + 1) * G))
+        rest = rest[cat[rest] < 0]
+        cat[rest] = len(heavy) + g
+    ncat = len(heavy) + 3
+    p = np.bincount(cat, weights=w, minlength=ncat) / w.sum()
+    n = 40_000
+    counts = np.zeros(ncat)
+    for b in range(n):
+        y, _ = oracle.group_race(logw, 3, 9, oracle.TAG_GUMBEL, b, 1)
+        assert w[y] > 0
+        counts[cat[y]] += 1
+    assert chisquare(counts, n * p).pvalue > 1e-3
+
+
+def test_group_race_with_one_group_is_the_plain_race():
+    """Support inside one group (or V <= RACE_GROUP): the group level has one
+    candidate and the entry level uses the plain race's noise, so the draw
+    equals svo_gumbel_argmax under every key."""
+    G = oracle.RACE_GROUP
+    rng = np.random.default_rng(6)
+    V = 3 * G
+    logw = np.full(V, -np.inf)
+    logw[G + 17:2 * G - 3] = rng.normal(0.0, 1.5, G - 20)
+    small = rng.normal(0.0, 1.0, 700)
+    for s in range(300):
+        assert (oracle.group_race(logw, 11, s, oracle.TAG_GUMBEL, 2, 3)[0]
+                == oracle.gumbel_argmax(logw, 11, s, oracle.TAG_GUMBEL, 2, 3)[0])
+        assert (oracle.group_race(small, 11, s, oracle.TAG_GUMBEL, 2, 3)[0]
+                == oracle.gumbel_argmax(small, 11, s, oracle.TAG_GUMBEL, 2, 3)[0])
+
+
+def test_group_race_levels_are_independent():
+    """Two groups of equal total weight, one entry of each heavy: the chosen
+    group must be a fair coin whatever entry the entry noise favours, i.e.
+    the group choice is independent of the entry level (a shared noise
+    source would tie them)."""
+    G = oracle.RACE_GROUP
+    V = 2 * G
+    logw = np.full(V, -np.inf)
+    logw[3] = 0.0
+    logw[G + 3] = 0.0  # same offset within its group: same entry counter word layout
+    n = 20_000
+    g1 = sum(oracle.group_race(logw, 1, 2, oracle.TAG_GUMBEL, b, 0)[0] >= G for b in range(n))
+    assert abs(g1 / n - 0.5) < 4.0 * math.sqrt(0.25 / n)
+
+
+def test_group_race_empty_support():
+    logw = np.full(3000, -np.inf)
+    assert oracle.group_race(logw, 0, 0, oracle.TAG_GUMBEL, 0, 0)[0] == -1
