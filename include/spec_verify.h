@@ -216,7 +216,7 @@ int spec_verify_host_async(const void* target_logits, const void* draft_logits,
  * loaded) instead of a caller workspace.  The call allocates nothing.
  *   - Size limit: shapes whose spec_verify_workspace_size exceeds
  *     SV_NOALLOC_MAX_WORKSPACE (8 MiB; for example B = 256, gamma = 4,
- *     V = 151936 bf16 needs about 3.9 MB) return SV_ERR_WORKSPACE and launch
+ *     V = 151936 bf16 needs about 1.5 MB) return SV_ERR_WORKSPACE and launch
  *     nothing; use spec_verify with a caller workspace for those.
  *   - First call per device: it looks up the array's device address
  *     (cudaGetSymbolAddress, with that device current) and clears its counter

@@ -63,12 +63,9 @@ int check_device() {
 Layout layout_single(int B, int gamma, int V, int dtype) {
   Layout l{};
   l.nc = row_segments(V, dtype);
-  l.nc2 = draw_chunks(B, V, dtype);
-  l.ctl = 0;
-  l.ticket1 = kHeaderCtl;
-  l.ticket2 = kHeaderCtl + kSeqSlots;
-  l.ready = kHeaderCtl + 2 * kSeqSlots;
-  l.bar = kHeaderCtl + 3 * kSeqSlots;
+  l.nc2 = draw_chunks(V);
+  l.ticket1 = 0;
+  l.ticket2 = kSeqSlots;
   size_t off = kHeaderBytes;
   l.part1 = off;  // row-pair partials: [B][gamma + 1][nseg] x 2 x 16 bytes
   off += up(static_cast<size_t>(B) * (gamma + 1) * l.nc * 2 * sizeof(float4));
@@ -89,11 +86,8 @@ Layout layout_multi(int B, int K, int L, int V, int dtype) {
   Layout l{};
   l.nc = 0;
   l.nc2 = 0;
-  l.ctl = 0;
-  l.ticket1 = kHeaderCtl;
-  l.ticket2 = kHeaderCtl + kSeqSlots;
-  l.ready = kHeaderCtl + 2 * kSeqSlots;
-  l.bar = kHeaderCtl + 3 * kSeqSlots;
+  l.ticket1 = 0;
+  l.ticket2 = kSeqSlots;
   size_t off = kHeaderBytes;
   l.resid = off;  // residual laws R (two per sequence) when they do not fit on chip
   off += up(multidraft_global_bytes(B, V));

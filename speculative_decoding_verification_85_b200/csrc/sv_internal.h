@@ -49,27 +49,20 @@ struct CallParams {
 };
 
 // Workspace layout of one call.  A header of fixed size at offset 0 holds the
-// control words and the per-sequence counters and flags (one slot per
-// sequence, up to SV_MAX_BATCH), so their positions do not depend on the
-// shape: every call leaves them at zero and a later call of any shape finds
-// them zeroed.
-// Header: 256 bytes of control words (kCtlNext / kCtlDraw: row-item and
-// draw-item counters of the verification kernel; kCtlExit: its CTA exit
-// counter; kCtlError: sticky word, non-zero once a bounded wait ran out),
-// then four per-sequence u32 arrays: row arrivals, draw arrivals,
-// decision-ready flags, draw bars.
-constexpr size_t kHeaderCtl = 256;
-constexpr int kCtlNext = 0, kCtlExit = 1, kCtlError = 2, kCtlDraw = 3;
+// per-sequence arrival counters (one slot per sequence, up to SV_MAX_BATCH),
+// so their positions do not depend on the shape: every call leaves them at
+// zero and a later call of any shape finds them zeroed.  Header: two u32
+// arrays, the row kernel's arrivals and the draw kernel's arrivals.
 constexpr size_t kSeqSlots = static_cast<size_t>(SV_MAX_BATCH) * sizeof(unsigned);
-constexpr size_t kHeaderBytes = kHeaderCtl + 4 * kSeqSlots;
+constexpr size_t kHeaderBytes = 2 * kSeqSlots;
 
 struct Layout {
-  size_t ctl, part1, ticket1, info, part2, ticket2, ready, bar, resid, total;
+  size_t part1, ticket1, info, part2, ticket2, resid, total;
   int nc, nc2;
 };
 
 Layout layout_single(int B, int gamma, int V, int dtype);
-int draw_chunks(int B, int V, int dtype);  // bound on draw items per sequence (sv_single.cu)
+int draw_chunks(int V);  // bound on draw CTAs per sequence (sv_single.cu)
 int row_segments(int V, int dtype);  // bound on row segments per row (sv_single.cu)
 Layout layout_multi(int B, int K, int L, int V, int dtype);
 size_t multidraft_global_bytes(int B, int V);  // residual laws of the multi-draft kernel (sv_multi.cu)

@@ -11,14 +11,13 @@
 // acceptance uniforms, the first rejection by warp ballot (FlexDraft,
 // Problem definition).
 // Draw kernel (Speculative Speculative Decoding, s.2 Saguaro sampling): once
-// the row kernel has completed (griddepcontrol.wait), one CTA per (sequence,
-// vocabulary chunk) runs the exponential race for the correction token from
-// max(p_j - q_j, 0), or the bonus token from p_gamma, with Philox noise keyed
-// per vocabulary entry; the CTA that completes a sequence combines.  Philox
-// is evaluated only for 4-entry blocks that can still win: since
-// E = -ln U > 2^-24 for every keyed uniform, a block whose largest weight w
-// has 2^24 w <= (a lower bound of the winning ratio) is skipped, exactly; the
-// blocks that remain are compacted per warp so that Philox runs on full warps.
+// the row kernel has completed (griddepcontrol.wait), the correction token is
+// drawn from max(p_j - q_j, 0), or the bonus token from p_gamma, by a
+// two-level exponential race: vocabulary groups of 1024 entries race with
+// their summed weights and one Philox exponential each, then the entries of
+// the winning group race with per-entry Philox noise.  Several CTAs per
+// sequence sum the groups; the CTA that completes a sequence runs the second
+// level.
 // Neither kernel waits on another CTA: all ordering is by arrival tickets and
 // by the launch dependency.
 #include <atomic>
@@ -161,18 +160,17 @@ __device__ __noinline__ void decide_single(const CallParams& p, int b, float T, 
 // ------------------------------------------------------------------ layout
 constexpr int kRowThreads = kTileThreads;  // 256
 constexpr int kDrawThreads = 256;
-constexpr int kDrawMaxBlocks = 8;          // Philox blocks per thread and draw CTA
-constexpr int kQCap = 64;                  // per-warp race queue (power of two)
-constexpr int kRaceBatch = 4;              // race rounds whose logits are loaded together
+constexpr int kRaceGroup = 1024;           // vocabulary entries per group of the draw race
+constexpr uint32_t kTagGroup = 7;          // Philox tag of the group-level noise
+constexpr int kDrawWaves = 4;              // about this many waves of draw CTAs per call
 static_assert(kRowThreads == kDrawThreads, "one thread count for both kernels");
 
 struct SingleParams {
   CallParams p1;       // inputs, outputs, decision state
   RacePartial* part2;   // [B][nc2] draw partials
   unsigned* ticket2;    // [B] draw arrivals
-  unsigned* bar;        // [B] draw bars (float bits, monotone), shared by a sequence's draw CTAs
   int nc2;              // draw CTAs per sequence
-  int chunk2;           // vocabulary entries per draw CTA (a multiple of 4)
+  int gpc;              // race groups per draw CTA
   int nseg;             // row segments per row (gridDim.y of the row kernel)
   int segvec;           // 16-byte vectors per row segment (multiple of kTileVec)
   float4* pairpart;     // [B][gamma + 1][nseg] x {target, draft} partials
@@ -472,70 +470,8 @@ struct Block4<false> {
   __device__ __forceinline__ void set_neg_inf() { r = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY); }
 };
 
-// Running winner of an exponential race: best weight / exponential pair and
-// index, and a slightly lowered lower bound of the winning ratio for the
-// cheap pre-tests.
-struct Race {
-  float bw, be;
-  int bi;
-  float lo;  // at most (winning ratio) (1 - 2^-20)
-  __device__ __forceinline__ void reset() {
-    bw = 0.0f;
-    be = 1.0f;
-    bi = INT_MAX;
-    lo = 0.0f;
-  }
-  // Exact test of candidate v (weight w > 0, Philox word x).
-  __device__ __forceinline__ void offer(float w, uint32_t x, int v) {
-    const float e = exponential_from_bits(x);
-    if (race_better(w, e, v, bw, be, bi)) {
-      bw = w;
-      be = e;
-      bi = v;
-      lo = fmaxf(lo, __fdiv_rn(bw, be) * (1.0f - 0x1p-20f));
-    }
-  }
-};
-
-// Candidates of one Philox block (entries v0 .. v0 + 3).  First a bound
-// without logarithms: since -ln U <= (1 - U) / U, every candidate's ratio
-// w / E is at least w U / t (t = 1 - U), so the block's largest such bound
-// (lowered for rounding) is a valid bar.  Then every entry runs the cheap
-// test w > lo t: since E >= t, w / t must beat the bar (lowered, so the test
-// never drops a possible winner; with lo >= 0 it also rejects w <= 0).  Only
-// entries that pass take the logarithm.
-__device__ __forceinline__ void race_block(Race& race, const float4& wv, const uint4& rnd, int v0) {
-  const float w[4] = {wv.x, wv.y, wv.z, wv.w};
-  float t[4];
-  float lb = 0.0f;
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    t[k] = gumbel_one_minus_u(word_of(rnd, k));
-    lb = fmaxf(lb, __fdividef(w[k] * (1.0f - t[k]), t[k]));
-  }
-  race.lo = fmaxf(race.lo, lb * (1.0f - 0x1p-20f));
-  bool pass[4];
-  bool any = false;
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    pass[k] = w[k] > race.lo * t[k];
-    any |= pass[k];
-  }
-  if (any) {
-#pragma unroll
-    for (int k = 0; k < 4; ++k)
-      if (pass[k] && w[k] > 0.0f) race.offer(w[k], word_of(rnd, k), v0 + k);
-  }
-}
-
-__device__ __forceinline__ float warp_max(float v) {
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
-  return v;
-}
-
-// Philox stream of one draw race: blocks (c0 = g) of the keyed counter
-// (g, b, step, tag 2 << 24 | j) under key (lo32 seed, hi32 seed).
+// Philox stream of one draw: blocks (c0 = g) of the keyed counter
+// (g, b, step, tag << 24 | j) under key (lo32 seed, hi32 seed).
 struct RaceKey {
   uint32_t k0, k1, b, step, c3;
   __device__ __forceinline__ uint4 block(int g) const {
@@ -543,147 +479,156 @@ struct RaceKey {
   }
 };
 
-// Philox and the exact test for up to 32 queued blocks, one per lane (lanes
-// at or beyond `count` take none).
-__device__ __forceinline__ void flush_queue(Race& race, const float4* qw, const int* qg, int head,
-                                            int count, const RaceKey& key) {
-  const int lane = threadIdx.x & 31;
-  const int e = (head + lane) & (kQCap - 1);
-  const bool mine = lane < count;
-  const float4 ww = mine ? qw[e] : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-  const int gg = mine ? qg[e] : 0;
-  __syncwarp();  // entries read before later rounds overwrite them
-  if (mine) race_block(race, ww, key.block(gg), 4 * gg);
-}
-
-// Exponential race of sequence b's draw over the Philox blocks of chunk
-// `chunk` of nchunk, by one CTA: round r covers blocks
-// [(r nchunk + chunk) 256, + 256), warp w 32 of them, one per lane, so every
-// chunk meets the low vocabulary indices first; each warp keeps its own
-// winner.  The winner is that of w_v / E_v (E_v = -ln U_v) with
-// w = max(p - q, 0) (residual) or w = p (bonus), p_v = 2^{(z_v - zmp) c - lsp}.
-// Rounds are taken kRaceBatch at a time, their logits loaded together.  The
-// warp's bar (a lower bound of the winning ratio, lowered for rounding) starts
-// from the sequence's shared bar and from max w / 17 (an entry's E is below
-// 17 for every keyed uniform), and grows with every candidate tested.  A block
-// is queued for Philox only if 2^24 max_k w_k exceeds the bar (exact: E > 2^-24,
-// so a skipped entry's ratio stays below the bar, which is below the winning
-// ratio); the queue is flushed 32 blocks at a time, so Philox runs on full
-// warps, and a batch in which every block needs Philox bypasses the queue.
-// `gbar` (or NULL) is the sequence's shared bar: read every batch, raised when
-// this warp's bar grows.
+// Sequence b's draw: the row(s) it reads and the constants of its weights
+// w_v = max(p_v - q_v, 0) (residual) or p_v (bonus), with
+// p_v = 2^{(z_v - zmp) c - lsp} and q_v = 2^{(y_v - zmq) c - lsq}.
 template <bool kBf16>
-__device__ __forceinline__ void race_span(const SingleParams& f, const SeqInfo& si, int b, int chunk,
-                                          int nchunk, unsigned* gbar, Race& race, float4* qw, int* qg) {
-  constexpr int U = kRaceBatch;
-  constexpr uintptr_t kVecAlign = kBf16 ? 8 : 16;
-  const CallParams& p = f.p1;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const char* trow = target_row<kBf16>(p, b, si.j);
-  const bool resid = si.mode == kModeResidual;
-  const char* drow = resid ? draft_row<kBf16>(p, b, si.j) : trow;
-  const bool tvec = (reinterpret_cast<uintptr_t>(trow) % kVecAlign) == 0;
-  const bool dvec = (reinterpret_cast<uintptr_t>(drow) % kVecAlign) == 0;
-  const float2 nm = make_float2(-si.zmp, -si.zmq), cc = make_float2(si.c, si.c),
-               nl = make_float2(-si.lsp, -si.lsq);
-  const RaceKey key{static_cast<uint32_t>(p.seed), static_cast<uint32_t>(p.seed >> 32),
-                    static_cast<uint32_t>(b), p.step, (kTagGumbel << 24) | static_cast<uint32_t>(si.j)};
-  const int nblocks = (p.V + 3) / 4;
-  int qh = 0, qn = 0;  // queue head and length (warp-uniform)
-  float published = 0.0f;
-  unsigned gnext = 0;
-  const unsigned lt_mask = (1u << lane) - 1u;
-  if (gbar && lane == 0) gnext = ld_relaxed(gbar);
-  for (int r0 = 0;; r0 += U) {
-    if ((r0 * nchunk + chunk) * kDrawThreads >= nblocks) break;  // uniform over the CTA
-    int g[U];
-    float4 w[U];
-    {
-      Block4<kBf16> tb[U], db[U];
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        g[u] = ((r0 + u) * nchunk + chunk) * kDrawThreads + warp * 32 + lane;
-        tb[u].set_neg_inf();
-        db[u].set_neg_inf();
-        if (g[u] < nblocks) {
-          tb[u].load(trow, tvec, p.V, g[u]);
-          if (resid) db[u].load(drow, dvec, p.V, g[u]);
-        }
-      }
-      // p_v = 2^{(z_v - zmp) c - lsp}, q_v likewise: the target and draft
-      // value of an entry travel as one packed pair
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        float ww[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const float2 e = __ffma2_rn(__fadd2_rn(make_float2(tb[u].at(k), db[u].at(k)), nm), cc, nl);
-          ww[k] = ex2_approx(e.x);
-          if (resid) ww[k] -= ex2_approx(e.y);
-        }
-        w[u] = make_float4(ww[0], ww[1], ww[2], ww[3]);
-      }
-    }
-    {
-      // bar from the heaviest entry of the batch: its E is below 17
-      float wmx = 0.0f;
-#pragma unroll
-      for (int u = 0; u < U; ++u) wmx = fmaxf(wmx, fmaxf(fmaxf(w[u].x, w[u].y), fmaxf(w[u].z, w[u].w)));
-      race.lo = fmaxf(race.lo, warp_max(wmx) * (1.0f / 17.0f));
-    }
-    if (gbar) {  // the shared bar read one batch earlier
-      const float gv = __uint_as_float(__shfl_sync(0xffffffffu, gnext, 0));
-      race.lo = fmaxf(race.lo, gv);
-      if (lane == 0) gnext = ld_relaxed(gbar);
-    }
-    bool need[U];
-    unsigned bal[U];
-    bool dense = qn == 0;
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const float wm = fmaxf(fmaxf(w[u].x, w[u].y), fmaxf(w[u].z, w[u].w));
-      need[u] = wm * 16777216.0f > race.lo;
-      bal[u] = __ballot_sync(0xffffffffu, need[u]);
-      dense = dense && bal[u] == 0xffffffffu;
-    }
-    if (dense) {
-      uint4 rnd[U];
-#pragma unroll
-      for (int u = 0; u < U; ++u) rnd[u] = key.block(g[u]);  // independent chains
-#pragma unroll
-      for (int u = 0; u < U; ++u) race_block(race, w[u], rnd[u], 4 * g[u]);
-    } else {
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        if (!bal[u]) continue;  // uniform over the warp
-        const int pos = (qh + qn + __popc(bal[u] & lt_mask)) & (kQCap - 1);
-        if (need[u]) {
-          qw[pos] = w[u];
-          qg[pos] = g[u];
-        }
-        qn += __popc(bal[u]);
-        __syncwarp();
-        if (qn >= 32) {
-          flush_queue(race, qw, qg, qh, 32, key);
-          qh = (qh + 32) & (kQCap - 1);
-          qn -= 32;
-        }
-      }
-    }
-    race.lo = warp_max(race.lo);
-    if (gbar && lane == 0 && race.lo > 2.0f * published) {
-      atomicMax(gbar, __float_as_uint(race.lo));  // non-negative floats order as their bits
-      published = race.lo;
+struct DrawRow {
+  const char* trow;
+  const char* drow;
+  bool tvec, dvec, resid;
+  int V, nblocks;
+  float2 nm, cc, nl;
+  __device__ __forceinline__ DrawRow(const CallParams& p, const SeqInfo& si, int b, bool resid_) {
+    constexpr uintptr_t kVecAlign = kBf16 ? 8 : 16;
+    resid = resid_;
+    trow = target_row<kBf16>(p, b, si.j);
+    drow = resid ? draft_row<kBf16>(p, b, si.j) : trow;
+    tvec = (reinterpret_cast<uintptr_t>(trow) % kVecAlign) == 0;
+    dvec = (reinterpret_cast<uintptr_t>(drow) % kVecAlign) == 0;
+    V = p.V;
+    nblocks = (p.V + 3) / 4;
+    nm = make_float2(-si.zmp, -si.zmq);
+    cc = make_float2(si.c, si.c);
+    nl = make_float2(-si.lsp, -si.lsq);
+  }
+  // Logits of Philox block g (entries 4g .. 4g + 3; -inf past the row).
+  __device__ __forceinline__ void load(int g, Block4<kBf16>& tb, Block4<kBf16>& db) const {
+    tb.set_neg_inf();
+    db.set_neg_inf();
+    if (g < nblocks) {
+      tb.load(trow, tvec, V, g);
+      if (resid) db.load(drow, dvec, V, g);
     }
   }
-  if (qn > 0) flush_queue(race, qw, qg, qh, qn, key);  // the rest of the queue
+  // The four weights: the target and draft value of an entry travel as one
+  // packed pair through the shift and the scale.
+  __device__ __forceinline__ float4 weights(const Block4<kBf16>& tb, const Block4<kBf16>& db) const {
+    float w[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float2 e = __ffma2_rn(__fadd2_rn(make_float2(tb.at(k), db.at(k)), nm), cc, nl);
+      w[k] = ex2_approx(e.x);
+      if (resid) w[k] = fmaxf(w[k] - ex2_approx(e.y), 0.0f);
+    }
+    return make_float4(w[0], w[1], w[2], w[3]);
+  }
+};
+
+// Level 1 of the draw, by one warp: the groups gid = g0, g0 + gstride, ...
+// below g1.  A group's 1024 entries are 8 passes of 32 lanes x 4 entries
+// (lane l of pass t holds Philox block 256 gid + 32 t + l), loaded 8 (bf16) or
+// 4 (fp32) passes at a time before any is used; each lane sums its 32 weights in order, then a butterfly over
+// the lanes gives every lane the same W_g.  The k-th group's W_g stays with
+// lane k % 32; every 32 groups (and at the end) those lanes draw their
+// groups' exponentials in parallel and enter the race.  Returns the warp's
+// winner in (bw, be, bi) (bi: the group index).
+template <bool kBf16>
+__device__ __forceinline__ void race_groups(const DrawRow<kBf16>& r, const RaceKey& gkey, int g0,
+                                            int gstride, int g1, float& bw, float& be, int& bi) {
+  constexpr int kPasses = kRaceGroup / 128;
+  constexpr int kBatch = kBf16 ? 8 : 4;  // passes loaded together (32 registers of logits)
+  const int lane = threadIdx.x & 31;
+  float myW = 0.0f;
+  int myG = -1;
+  int k = 0;
+  auto enter = [&]() {
+    if (myG >= 0) {
+      const float e = exponential_from_bits(gkey.block(myG).x);
+      if (race_better(myW, e, myG, bw, be, bi)) {
+        bw = myW;
+        be = e;
+        bi = myG;
+      }
+    }
+    myG = -1;
+  };
+  for (int gid = g0; gid < g1; gid += gstride, ++k) {
+    float s = 0.0f;
+#pragma unroll
+    for (int t0 = 0; t0 < kPasses; t0 += kBatch) {
+      Block4<kBf16> tb[kBatch], db[kBatch];
+#pragma unroll
+      for (int t = 0; t < kBatch; ++t) r.load(gid * (kRaceGroup / 4) + (t0 + t) * 32 + lane, tb[t], db[t]);
+#pragma unroll
+      for (int t = 0; t < kBatch; ++t) {
+        const float4 w = r.weights(tb[t], db[t]);
+        s = (((s + w.x) + w.y) + w.z) + w.w;
+      }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+    if (lane == (k & 31)) {
+      myW = s;
+      myG = gid;
+    }
+    if ((k & 31) == 31) enter();
+  }
+  enter();
 }
 
+// Level 2, by the whole CTA: the entries of group gid, one Philox block per
+// thread (block 256 gid + t), in the race of w_v / E_v with the per-entry
+// noise.  Returns the CTA's winner in every thread.
+template <bool kBf16>
+__device__ __forceinline__ int race_entries(const DrawRow<kBf16>& r, const RaceKey& ekey, int gid,
+                                            float4* scratch) {
+  static_assert(kDrawThreads * 4 == kRaceGroup, "one Philox block per thread");
+  const int g = gid * (kRaceGroup / 4) + static_cast<int>(threadIdx.x);
+  Block4<kBf16> tb, db;
+  r.load(g, tb, db);
+  const float4 w4 = r.weights(tb, db);
+  const float w[4] = {w4.x, w4.y, w4.z, w4.w};
+  const uint4 rnd = ekey.block(g);
+  float bw = 0.0f, be = 1.0f;
+  int bi = INT_MAX;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    if (!(w[k] > 0.0f)) continue;
+    const float e = exponential_from_bits(word_of(rnd, k));
+    if (race_better(w[k], e, 4 * g + k, bw, be, bi)) {
+      bw = w[k];
+      be = e;
+      bi = 4 * g + k;
+    }
+  }
+  race_reduce<kDrawThreads>(bw, be, bi, scratch);
+  return bi;
+}
+
+// Both levels over the whole target row j in one CTA: the draw from p_j
+// when the residual max(p_j - q_j, 0) vanished (p_j == q_j to rounding).
+template <bool kBf16>
+__device__ __noinline__ int draw_from_target(const CallParams& p, const SeqInfo& si, int b,
+                                             const RaceKey& gkey, const RaceKey& ekey, float4* scratch) {
+  const DrawRow<kBf16> prow(p, si, b, false);
+  const int ng = (p.V + kRaceGroup - 1) / kRaceGroup;
+  float bw = 0.0f, be = 1.0f;
+  int bi = INT_MAX;
+  race_groups<kBf16>(prow, gkey, static_cast<int>(threadIdx.x >> 5), kDrawThreads / 32, ng, bw, be, bi);
+  race_reduce<kDrawThreads>(bw, be, bi, scratch);
+  return race_entries<kBf16>(prow, ekey, bi, scratch);
+}
+
+// Draw kernel.  Grid: nc2 CTAs per sequence; CTA c of sequence b runs level
+// 1 over groups [c gpc, (c + 1) gpc) (warp w: groups c gpc + w, + 8, ...),
+// publishes its winning group, and the CTA that completes the sequence
+// (arrival ticket) combines the nc2 winners and runs level 2 in the winning
+// group.  If every residual weight is zero (p_j == q_j to rounding), that CTA
+// draws from p_j instead, both levels over the whole row.
 template <bool kBf16>
 __global__ void __launch_bounds__(kDrawThreads, 4) draw_kernel(const __grid_constant__ SingleParams f) {
   __shared__ float4 scratch[kDrawThreads / 32];
-  __shared__ float4 qw[kDrawThreads / 32][kQCap];  // per-warp race queues
-  __shared__ int qg[kDrawThreads / 32][kQCap];
   __shared__ int s_last;
   pdl_wait_and_release();  // the row kernel has completed: every decision is visible
   const int b = blockIdx.x / f.nc2;
@@ -703,24 +648,22 @@ __global__ void __launch_bounds__(kDrawThreads, 4) draw_kernel(const __grid_cons
   const bool draw = (si.mode == kModeResidual && si.j >= 0 && si.j < p.gamma) ||
                     (si.mode == kModeBonus && si.j == p.gamma);
   if (!draw) return;  // uniform: greedy or invalid sequence
-  Race race;
-  race.reset();
-  // bonus draw: the entry at the row maximum has weight 2^-lsp and E < 17, so
-  // its ratio -- and the winner's -- exceeds 2^-lsp / 17
-  if (si.mode == kModeBonus) race.lo = ex2_approx(-si.lsp) * (1.0f / 17.0f);
-  race_span<kBf16>(f, si, b, chunk, f.nc2, f.bar + b, race, qw[warp], qg[warp]);
-  float bw = race.bw, be = race.be;
-  int bi = race.bi;
+  const uint32_t k0 = static_cast<uint32_t>(p.seed), k1 = static_cast<uint32_t>(p.seed >> 32);
+  const RaceKey gkey{k0, k1, static_cast<uint32_t>(b), p.step, (kTagGroup << 24) | static_cast<uint32_t>(si.j)};
+  const RaceKey ekey{k0, k1, static_cast<uint32_t>(b), p.step, (kTagGumbel << 24) | static_cast<uint32_t>(si.j)};
+  const int ng = (p.V + kRaceGroup - 1) / kRaceGroup;
+  const DrawRow<kBf16> row(p, si, b, si.mode == kModeResidual);
+  float bw = 0.0f, be = 1.0f;
+  int bi = INT_MAX;
+  const int gc0 = chunk * f.gpc;
+  race_groups<kBf16>(row, gkey, gc0 + warp, kDrawThreads / 32, min(ng, gc0 + f.gpc), bw, be, bi);
   race_reduce<kDrawThreads>(bw, be, bi, scratch);
   if (threadIdx.x == 0) {
     RacePartial* pp = f.part2 + static_cast<size_t>(b) * f.nc2 + chunk;
     *reinterpret_cast<float4*>(pp) = make_float4(bw, be, __int_as_float(bi), 0.0f);
     const unsigned t = ticket_acq_rel(f.ticket2 + b);
     s_last = (t == static_cast<unsigned>(f.nc2 - 1));
-    if (s_last) {
-      f.ticket2[b] = 0;
-      f.bar[b] = 0;  // every CTA of the sequence is past its race
-    }
+    if (s_last) f.ticket2[b] = 0;  // leave the counter at zero for the next call
   }
   block_sync<kDrawThreads>();  // orders the other threads after thread 0's acquire
   if (!s_last) return;
@@ -736,20 +679,13 @@ __global__ void __launch_bounds__(kDrawThreads, 4) draw_kernel(const __grid_cons
     }
   }
   race_reduce<kDrawThreads>(bw, be, bi, scratch);
-  if (!(bw > 0.0f)) {  // uniform: race_reduce returns the winner to every thread
-    // the residual vanished (p_j == q_j to rounding): draw from p_j instead,
-    // over the whole row in this CTA (without the residual race's bar)
-    SeqInfo sb = si;
-    sb.mode = kModeBonus;
-    race.reset();
-    race.lo = ex2_approx(-sb.lsp) * (1.0f / 17.0f);
-    race_span<kBf16>(f, sb, b, 0, 1, nullptr, race, qw[warp], qg[warp]);
-    bw = race.bw;
-    be = race.be;
-    bi = race.bi;
-    race_reduce<kDrawThreads>(bw, be, bi, scratch);
+  int y;
+  if (bw > 0.0f) {  // uniform: race_reduce returns the winner to every thread
+    y = race_entries<kBf16>(row, ekey, bi, scratch);
+  } else {
+    y = draw_from_target<kBf16>(p, si, b, gkey, ekey, scratch);  // the residual vanished
   }
-  if (threadIdx.x == 0) p.out_tokens[static_cast<size_t>(b) * (p.gamma + 1) + si.j] = bi;
+  if (threadIdx.x == 0) p.out_tokens[static_cast<size_t>(b) * (p.gamma + 1) + si.j] = y;
 }
 
 // ------------------------------------------------------------------ launch
@@ -763,10 +699,9 @@ int body_tiles(int V, int dtype) {  // tiles of kTileVec vectors covering a row'
 
 int row_segments(int V, int dtype) { return body_tiles(V, dtype); }  // bound on segments per row
 
-int draw_chunks(int B, int V, int dtype) {  // upper bound on draw CTAs per sequence
-  (void)B;
-  (void)dtype;
-  return (V + 255) / 256;
+int draw_chunks(int V) {  // upper bound on draw CTAs per sequence: one group per warp
+  const int ng = (V + kRaceGroup - 1) / kRaceGroup;
+  return (ng + kDrawThreads / 32 - 1) / (kDrawThreads / 32);
 }
 
 namespace {
@@ -891,22 +826,18 @@ int launch_single(const void* target, const void* draft, const int32_t* tokens,
   f.zx = reinterpret_cast<float*>(ws + lay.resid);
   f.part2 = reinterpret_cast<RacePartial*>(ws + lay.part2);
   f.ticket2 = reinterpret_cast<unsigned*>(ws + lay.ticket2);
-  f.bar = reinterpret_cast<unsigned*>(ws + lay.bar);
-  // Draw chunks: a whole number of waves of the draw kernel over the GPU,
-  // with at most about kDrawMaxBlocks Philox blocks per thread; chunks are
-  // balanced within a sequence (in Philox blocks of 4 entries).
+  // Draw CTAs: race groups per warp chosen so that the B sequences' groups
+  // fill about kDrawWaves waves of CTAs (at least one group per warp, so a
+  // small batch still spreads each row over several CTAs); a CTA covers
+  // 8 warps' groups.
   {
-    const long long nb = (V + 3) / 4;  // Philox blocks per row
-    const long long slots2 = static_cast<long long>(sm_count()) * draw_ctas_per_sm(bf16);
-    const long long per_cta = static_cast<long long>(kDrawMaxBlocks) * kDrawThreads;
-    const long long waves = (static_cast<long long>(B) * nb + per_cta * slots2 - 1) / (per_cta * slots2);
-    long long nc2 = waves * slots2 / B;
-    if (nc2 < 1) nc2 = 1;
-    if (nc2 > lay.nc2) nc2 = lay.nc2;
-    if (nc2 > nb) nc2 = nb;
-    const long long cb = (nb + nc2 - 1) / nc2;  // blocks per draw CTA
-    f.chunk2 = static_cast<int>(4 * cb);
-    f.nc2 = static_cast<int>((nb + cb - 1) / cb);
+    const long long ng = (V + kRaceGroup - 1) / kRaceGroup;
+    const long long warps = static_cast<long long>(sm_count()) * draw_ctas_per_sm(bf16) * (kDrawThreads / 32);
+    long long gpw = (static_cast<long long>(B) * ng + warps * kDrawWaves - 1) / (warps * kDrawWaves);
+    if (gpw < 1) gpw = 1;
+    const long long gpc = gpw * (kDrawThreads / 32);
+    f.gpc = static_cast<int>(gpc < ng ? gpc : ng);
+    f.nc2 = static_cast<int>((ng + f.gpc - 1) / f.gpc);  // <= lay.nc2: gpc >= 8 or nc2 == 1
   }
 
   if (static_cast<long long>(B) * f.nc2 > INT_MAX)
