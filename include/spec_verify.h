@@ -38,8 +38,8 @@
  *   - Workspace: caller-owned device memory of at least the size returned by
  *     the matching *_workspace_size function, 256-byte aligned, zero-filled
  *     before its first use (spec_verify_workspace_init or cudaMemset).  The
- *     workspace starts with a fixed 512 KB header of per-sequence arrival
- *     counters (their offsets do not depend on the shape), followed by
+ *     workspace starts with a fixed 768 KB header of per-sequence arrival
+ *     counters and flags (their offsets do not depend on the shape), followed by
  *     per-call partial results.  Every call returns the counters to zero, so
  *     the workspace can be reused by later calls on the same stream, of any
  *     shape that fits, without clearing.  Two calls that may run concurrently

@@ -66,6 +66,7 @@ Layout layout_single(int B, int gamma, int V, int dtype) {
   l.nc2 = draw_chunks(V);
   l.ticket1 = 0;
   l.ticket2 = kSeqSlots;
+  l.ready = 2 * kSeqSlots;
   size_t off = kHeaderBytes;
   l.part1 = off;  // row-pair partials: [B][gamma + 1][nseg] x 2 x 16 bytes
   off += up(static_cast<size_t>(B) * (gamma + 1) * l.nc * 2 * sizeof(float4));
@@ -88,6 +89,7 @@ Layout layout_multi(int B, int K, int L, int V, int dtype) {
   l.nc2 = 0;
   l.ticket1 = 0;
   l.ticket2 = kSeqSlots;
+  l.ready = 2 * kSeqSlots;
   size_t off = kHeaderBytes;
   l.resid = off;  // residual laws R (two per sequence) when they do not fit on chip
   off += up(multidraft_global_bytes(B, V));

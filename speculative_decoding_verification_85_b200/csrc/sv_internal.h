@@ -51,13 +51,14 @@ struct CallParams {
 // Workspace layout of one call.  A header of fixed size at offset 0 holds the
 // per-sequence arrival counters (one slot per sequence, up to SV_MAX_BATCH),
 // so their positions do not depend on the shape: every call leaves them at
-// zero and a later call of any shape finds them zeroed.  Header: two u32
-// arrays, the row kernel's arrivals and the draw kernel's arrivals.
+// zero and a later call of any shape finds them zeroed.  Header: three u32
+// arrays, the row kernel's arrivals, the draw kernel's arrivals and the
+// decision-published flags.
 constexpr size_t kSeqSlots = static_cast<size_t>(SV_MAX_BATCH) * sizeof(unsigned);
-constexpr size_t kHeaderBytes = 2 * kSeqSlots;
+constexpr size_t kHeaderBytes = 3 * kSeqSlots;
 
 struct Layout {
-  size_t part1, ticket1, info, part2, ticket2, resid, total;
+  size_t part1, ticket1, info, part2, ticket2, ready, resid, total;
   int nc, nc2;
 };
 

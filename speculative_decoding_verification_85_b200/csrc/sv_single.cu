@@ -11,15 +11,17 @@
 // acceptance uniforms, the first rejection by warp ballot (FlexDraft,
 // Problem definition).
 // Draw kernel (Speculative Speculative Decoding, s.2 Saguaro sampling): once
-// the row kernel has completed (griddepcontrol.wait), the correction token is
+// its sequence's decision is published (a flag the row kernel sets; the draw
+// grid may start while the row kernel's last CTAs run), the correction token is
 // drawn from max(p_j - q_j, 0), or the bonus token from p_gamma, by a
 // two-level exponential race: vocabulary groups of 1024 entries race with
 // their summed weights and one Philox exponential each, then the entries of
 // the winning group race with per-entry Philox noise.  Several CTAs per
 // sequence sum the groups; the CTA that completes a sequence runs the second
 // level.
-// Neither kernel waits on another CTA: all ordering is by arrival tickets and
-// by the launch dependency.
+// The row kernel waits on no other CTA (arrival tickets only); a draw CTA
+// waits, with a time limit, for one flag that a row-kernel CTA already
+// running sets.
 #include <atomic>
 #include <climits>
 
@@ -169,9 +171,10 @@ struct SingleParams {
   CallParams p1;       // inputs, outputs, decision state
   RacePartial* part2;   // [B][nc2] draw partials
   unsigned* ticket2;    // [B] draw arrivals
+  unsigned* ready;      // [B] decision published (set by the row kernel, cleared by the draw kernel)
   int nc2;              // draw CTAs per sequence
   int gpc;              // race groups per draw CTA
-  int nseg;             // row segments per row (gridDim.y of the row kernel)
+  int nseg;             // row segments per row
   int segvec;           // 16-byte vectors per row segment (multiple of kTileVec)
   float4* pairpart;     // [B][gamma + 1][nseg] x {target, draft} partials
   float* zx;            // [B][gamma][nseg][2] draft token's target / draft logit
@@ -330,7 +333,9 @@ __device__ __forceinline__ void pick_logit(const uint4 (&r)[kTileRegs], int own,
 }
 
 // --------------------------------------------------------------- row kernel
-// Grid: x = b (gamma + 1) + i (row pair), y = segment.
+// Grid: one CTA per (row pair, segment), blockIdx.x = (b (gamma + 1) + i)
+// nseg + seg: a sequence's CTAs are consecutive, so sequences complete in
+// order of b while the kernel runs.
 template <bool kBf16>
 __global__ void __launch_bounds__(kRowThreads, 3) rows_kernel(const __grid_constant__ SingleParams f) {
   __shared__ RowAcc rows[kMaxRowsPerSeq];
@@ -342,10 +347,10 @@ __global__ void __launch_bounds__(kRowThreads, 3) rows_kernel(const __grid_const
   pdl_wait_and_release();
   const CallParams& p = f.p1;
   const int tid = threadIdx.x;
-  const int pair = blockIdx.x;
+  const int pair = static_cast<int>(blockIdx.x) / f.nseg;
+  const int seg = static_cast<int>(blockIdx.x) - pair * f.nseg;
   const int b = pair / (p.gamma + 1);
   const int i = pair - b * (p.gamma + 1);
-  const int seg = blockIdx.y;
   const float T = __ldg(p.temps + b);
   const int modeA = row_mode(T, true);
   const bool argmaxA = modeA == kRowArgmax;
@@ -417,7 +422,13 @@ __global__ void __launch_bounds__(kRowThreads, 3) rows_kernel(const __grid_const
   block_sync<kRowThreads>();  // orders the other threads after thread 0's acquire
   if (!s_last) return;
   combine_pairs(f, b, argmaxA, c, rows, s_zsel);
-  if (tid < 32) decide_single<kBf16>(p, b, T, s_tok, rows, s_zsel);
+  if (tid < 32) {
+    decide_single<kBf16>(p, b, T, s_tok, rows, s_zsel);
+    // publish the decision: every lane's writes, then the flag (release)
+    __threadfence();
+    __syncwarp();
+    if (tid == 0) st_release(f.ready + b, 1u);
+  }
 }
 
 // -------------------------------------------------------------- draw kernel
@@ -442,6 +453,9 @@ struct Block4<true> {
       r = make_uint2(h[0] | (h[1] << 16), h[2] | (h[3] << 16));
     }
   }
+  __device__ __forceinline__ void load_vec(const char* row, int g) {
+    r = __ldg(reinterpret_cast<const uint2*>(row) + g);
+  }
   __device__ __forceinline__ float at(int w) const {
     const uint32_t x = w < 2 ? r.x : r.y;
     return (w & 1) ? bf16_hi(x) : bf16_lo(x);
@@ -463,6 +477,9 @@ struct Block4<false> {
       r.z = v0 + 2 < V ? __ldg(q + v0 + 2) : -INFINITY;
       r.w = v0 + 3 < V ? __ldg(q + v0 + 3) : -INFINITY;
     }
+  }
+  __device__ __forceinline__ void load_vec(const char* row, int g) {
+    r = __ldg(reinterpret_cast<const float4*>(row) + g);
   }
   __device__ __forceinline__ float at(int w) const {
     return w == 0 ? r.x : (w == 1 ? r.y : (w == 2 ? r.z : r.w));
@@ -511,6 +528,15 @@ struct DrawRow {
       if (resid) db.load(drow, dvec, V, g);
     }
   }
+  // The same for a block known to lie inside the row, rows vector-aligned.
+  __device__ __forceinline__ void load_fast(int g, Block4<kBf16>& tb, Block4<kBf16>& db) const {
+    tb.load_vec(trow, g);
+    if (resid) db.load_vec(drow, g); else db.set_neg_inf();
+  }
+  // Group gid lies inside the row and both rows take vector loads.
+  __device__ __forceinline__ bool fast(int gid) const {
+    return tvec && (dvec || !resid) && (gid + 1) * kRaceGroup <= V;
+  }
   // The four weights: the target and draft value of an entry travel as one
   // packed pair through the shift and the scale.
   __device__ __forceinline__ float4 weights(const Block4<kBf16>& tb, const Block4<kBf16>& db) const {
@@ -558,8 +584,13 @@ __device__ __forceinline__ void race_groups(const DrawRow<kBf16>& r, const RaceK
 #pragma unroll
     for (int t0 = 0; t0 < kPasses; t0 += kBatch) {
       Block4<kBf16> tb[kBatch], db[kBatch];
+      if (r.fast(gid)) {  // uniform over the warp
 #pragma unroll
-      for (int t = 0; t < kBatch; ++t) r.load(gid * (kRaceGroup / 4) + (t0 + t) * 32 + lane, tb[t], db[t]);
+        for (int t = 0; t < kBatch; ++t) r.load_fast(gid * (kRaceGroup / 4) + (t0 + t) * 32 + lane, tb[t], db[t]);
+      } else {
+#pragma unroll
+        for (int t = 0; t < kBatch; ++t) r.load(gid * (kRaceGroup / 4) + (t0 + t) * 32 + lane, tb[t], db[t]);
+      }
 #pragma unroll
       for (int t = 0; t < kBatch; ++t) {
         const float4 w = r.weights(tb[t], db[t]);
@@ -626,47 +657,78 @@ __device__ __noinline__ int draw_from_target(const CallParams& p, const SeqInfo&
 // (arrival ticket) combines the nc2 winners and runs level 2 in the winning
 // group.  If every residual weight is zero (p_j == q_j to rounding), that CTA
 // draws from p_j instead, both levels over the whole row.
+// Bounded wait (kWaitLimitNs) for sequence b's decision flag, by one thread.
+__device__ __forceinline__ bool wait_ready(const unsigned* flag) {
+  if (ld_acquire(flag) != 0u) return true;
+  const uint64_t t0 = global_ns();
+  for (;;) {
+    __nanosleep(256);
+    if (ld_acquire(flag) != 0u) return true;
+    if (global_ns() - t0 > kWaitLimitNs) return false;
+  }
+}
+
 template <bool kBf16>
 __global__ void __launch_bounds__(kDrawThreads, 4) draw_kernel(const __grid_constant__ SingleParams f) {
   __shared__ float4 scratch[kDrawThreads / 32];
-  __shared__ int s_last;
-  pdl_wait_and_release();  // the row kernel has completed: every decision is visible
+  __shared__ int s_last, s_ready;
+  // No griddepcontrol.wait: this grid may start while the row kernel's last
+  // CTAs still run, and each CTA waits for its own sequence's decision flag
+  // instead.  (It starts only once every row-kernel CTA has started, so the
+  // row kernel never waits for SM room held by this grid.)
+  asm volatile("griddepcontrol.launch_dependents;");
   const int b = blockIdx.x / f.nc2;
   const int chunk = blockIdx.x - b * f.nc2;
   const int warp = threadIdx.x >> 5;
   const CallParams& p = f.p1;
-  const float4* ip = reinterpret_cast<const float4*>(p.info + b);
-  const float4 w0 = __ldcg(ip), w1 = __ldcg(ip + 1);
+  if (threadIdx.x == 0) s_ready = wait_ready(f.ready + b) ? 1 : 0;
+  block_sync<kDrawThreads>();  // orders the other threads after thread 0's acquire
   SeqInfo si{};
-  si.mode = __float_as_int(w0.x);
-  si.j = __float_as_int(w0.y);
-  si.zmp = w0.z;
-  si.zmq = w0.w;
-  si.c = w1.x;
-  si.lsp = w1.y;
-  si.lsq = w1.z;
+  si.mode = kModeNone;
+  if (s_ready) {
+    const float4* ip = reinterpret_cast<const float4*>(p.info + b);
+    const float4 w0 = __ldcg(ip), w1 = __ldcg(ip + 1);
+    si.mode = __float_as_int(w0.x);
+    si.j = __float_as_int(w0.y);
+    si.zmp = w0.z;
+    si.zmq = w0.w;
+    si.c = w1.x;
+    si.lsp = w1.y;
+    si.lsq = w1.z;
+  } else if (chunk == 0) {
+    // the decision never came (a wait ran out of time): no result
+    for (int i = threadIdx.x; i <= p.gamma; i += kDrawThreads)
+      p.out_tokens[static_cast<size_t>(b) * (p.gamma + 1) + i] = -1;
+    if (threadIdx.x == 0) p.accept_len[b] = -1;
+  }
   const bool draw = (si.mode == kModeResidual && si.j >= 0 && si.j < p.gamma) ||
                     (si.mode == kModeBonus && si.j == p.gamma);
-  if (!draw) return;  // uniform: greedy or invalid sequence
   const uint32_t k0 = static_cast<uint32_t>(p.seed), k1 = static_cast<uint32_t>(p.seed >> 32);
   const RaceKey gkey{k0, k1, static_cast<uint32_t>(b), p.step, (kTagGroup << 24) | static_cast<uint32_t>(si.j)};
   const RaceKey ekey{k0, k1, static_cast<uint32_t>(b), p.step, (kTagGumbel << 24) | static_cast<uint32_t>(si.j)};
   const int ng = (p.V + kRaceGroup - 1) / kRaceGroup;
-  const DrawRow<kBf16> row(p, si, b, si.mode == kModeResidual);
   float bw = 0.0f, be = 1.0f;
   int bi = INT_MAX;
-  const int gc0 = chunk * f.gpc;
-  race_groups<kBf16>(row, gkey, gc0 + warp, kDrawThreads / 32, min(ng, gc0 + f.gpc), bw, be, bi);
-  race_reduce<kDrawThreads>(bw, be, bi, scratch);
+  if (draw) {  // uniform
+    const DrawRow<kBf16> row(p, si, b, si.mode == kModeResidual);
+    const int gc0 = chunk * f.gpc;
+    race_groups<kBf16>(row, gkey, gc0 + warp, kDrawThreads / 32, min(ng, gc0 + f.gpc), bw, be, bi);
+    race_reduce<kDrawThreads>(bw, be, bi, scratch);
+  }
+  // Every CTA of the sequence arrives (drawing or not), so the last one can
+  // clear the flag and the counter for the next call.
   if (threadIdx.x == 0) {
     RacePartial* pp = f.part2 + static_cast<size_t>(b) * f.nc2 + chunk;
-    *reinterpret_cast<float4*>(pp) = make_float4(bw, be, __int_as_float(bi), 0.0f);
+    if (draw) *reinterpret_cast<float4*>(pp) = make_float4(bw, be, __int_as_float(bi), 0.0f);
     const unsigned t = ticket_acq_rel(f.ticket2 + b);
     s_last = (t == static_cast<unsigned>(f.nc2 - 1));
-    if (s_last) f.ticket2[b] = 0;  // leave the counter at zero for the next call
+    if (s_last) {
+      f.ticket2[b] = 0;
+      f.ready[b] = 0;  // every CTA of the sequence is past its wait
+    }
   }
   block_sync<kDrawThreads>();  // orders the other threads after thread 0's acquire
-  if (!s_last) return;
+  if (!s_last || !draw) return;
   bw = 0.0f;
   be = 1.0f;
   bi = INT_MAX;
@@ -681,6 +743,7 @@ __global__ void __launch_bounds__(kDrawThreads, 4) draw_kernel(const __grid_cons
   race_reduce<kDrawThreads>(bw, be, bi, scratch);
   int y;
   if (bw > 0.0f) {  // uniform: race_reduce returns the winner to every thread
+    const DrawRow<kBf16> row(p, si, b, si.mode == kModeResidual);
     y = race_entries<kBf16>(row, ekey, bi, scratch);
   } else {
     y = draw_from_target<kBf16>(p, si, b, gkey, ekey, scratch);  // the residual vanished
@@ -817,7 +880,6 @@ int launch_single(const void* target, const void* draft, const int32_t* tokens,
     st = st < 1 ? 1 : (st > kMaxSegTiles ? kMaxSegTiles : st);
     int nseg = static_cast<int>((tiles + st - 1) / st);
     if (nseg > lay.nc) nseg = lay.nc;
-    if (nseg > 65535) nseg = 65535;  // gridDim.y
     st = (tiles + nseg - 1) / nseg;
     f.nseg = nseg;
     f.segvec = static_cast<int>(st) * kTileVec;
@@ -826,6 +888,7 @@ int launch_single(const void* target, const void* draft, const int32_t* tokens,
   f.zx = reinterpret_cast<float*>(ws + lay.resid);
   f.part2 = reinterpret_cast<RacePartial*>(ws + lay.part2);
   f.ticket2 = reinterpret_cast<unsigned*>(ws + lay.ticket2);
+  f.ready = reinterpret_cast<unsigned*>(ws + lay.ready);
   // Draw CTAs: race groups per warp chosen so that the B sequences' groups
   // fill about kDrawWaves waves of CTAs (at least one group per warp, so a
   // small batch still spreads each row over several CTAs); a CTA covers
@@ -843,7 +906,10 @@ int launch_single(const void* target, const void* draft, const int32_t* tokens,
   if (static_cast<long long>(B) * f.nc2 > INT_MAX)
     return set_error(SV_ERR_INVALID_ARG, "B x V too large for one launch (draw grid %lld CTAs)",
                      static_cast<long long>(B) * f.nc2);
-  const dim3 grid1(static_cast<unsigned>(B * (gamma + 1)), static_cast<unsigned>(f.nseg));
+  const long long ctas1 = static_cast<long long>(B) * (gamma + 1) * f.nseg;
+  if (ctas1 > INT_MAX)
+    return set_error(SV_ERR_INVALID_ARG, "B x V too large for one launch (row grid %lld CTAs)", ctas1);
+  const dim3 grid1(static_cast<unsigned>(ctas1));
   cudaError_t e = bf16 ? launch_pdl(rows_kernel<true>, grid1, kRowThreads, stream, f)
                        : launch_pdl(rows_kernel<false>, grid1, kRowThreads, stream, f);
   if (e != cudaSuccess)
