@@ -195,6 +195,12 @@ __device__ __forceinline__ bool race_better(float w, float e, int idx, float bw,
 
 
 // ------------------------------------------------ async copies and flags
+// Bulk prefetch of [p, p + bytes) into L2 (p and bytes multiples of 16); no
+// destination, no completion to wait for.
+__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
 // Shared-memory address of a generic pointer to this CTA's shared memory.
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

@@ -165,6 +165,7 @@ constexpr int kDrawThreads = 256;
 constexpr int kRaceGroup = 1024;           // vocabulary entries per group of the draw race
 constexpr uint32_t kTagGroup = 7;          // Philox tag of the group-level noise
 constexpr int kDrawWaves = 4;              // about this many waves of draw CTAs per call
+constexpr int kPrefetchTiles = 1;          // row tiles requested into L2 ahead of the loads
 static_assert(kRowThreads == kDrawThreads, "one thread count for both kernels");
 
 struct SingleParams {
@@ -380,7 +381,17 @@ __global__ void __launch_bounds__(kRowThreads, 3) rows_kernel(const __grid_const
   const int ownA = owned_vector<kBf16>(gA, xg, k0, a1);
   const int ownB = owned_vector<kBf16>(gB, xg, k0, b1);
   const int kend = max(loadA ? a1 : k0, loadB ? b1 : k0);
+  // L2 prefetch kPrefetchTiles tiles ahead of the loads (one bulk request
+  // per row and tile, issued by lane 0 of warps 0 and 1), so DRAM keeps
+  // streaming while the registers wait on the current tile.
+  auto prefetch = [&](int kp) {
+    if (tid == 0 && loadA && kp < a1) prefetch_l2(vA + kp, static_cast<uint32_t>(min(kTileVec, a1 - kp)) * 16u);
+    if (tid == 32 && loadB && kp < b1) prefetch_l2(vB + kp, static_cast<uint32_t>(min(kTileVec, b1 - kp)) * 16u);
+  };
+#pragma unroll
+  for (int d = 1; d < kPrefetchTiles; ++d) prefetch(k0 + d * kTileVec);
   for (int kb = k0; kb < kend; kb += kTileVec) {
+    if (kPrefetchTiles > 0) prefetch(kb + kPrefetchTiles * kTileVec);
     uint4 ra[kTileRegs], rb[kTileRegs];
     if (loadA) load_tile<kBf16>(vA, kb, a1, ra);
     if (loadB) load_tile<kBf16>(vB, kb, b1, rb);

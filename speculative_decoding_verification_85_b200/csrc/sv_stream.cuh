@@ -159,14 +159,18 @@ __device__ __forceinline__ void lse_tile(RunAcc& a, const uint4 (&r)[kTileRegs],
   }
   if (tm > a.m) lift_ref(a, tm, c);
   const float2 nr = make_float2(-a.R, -a.R), cc = make_float2(c, c);
-  float2 acc = make_float2(0.0f, 0.0f);
+  // one partial sum per vector, so the adds form kTileRegs independent chains
+  float2 acc[kTileRegs];
 #pragma unroll
   for (int j = 0; j < kTileRegs; ++j) {
+    acc[j] = ex2_pair(__ffma2_rn(V::pair(r[j], 0), cc, nr));
 #pragma unroll
-    for (int k = 0; k < V::kN / 2; ++k)
-      acc = __fadd2_rn(acc, ex2_pair(__ffma2_rn(V::pair(r[j], k), cc, nr)));
+    for (int k = 1; k < V::kN / 2; ++k)
+      acc[j] = __fadd2_rn(acc[j], ex2_pair(__ffma2_rn(V::pair(r[j], k), cc, nr)));
   }
-  a.s = __fadd2_rn(a.s, acc);
+#pragma unroll
+  for (int j = 1; j < kTileRegs; ++j) acc[0] = __fadd2_rn(acc[0], acc[j]);
+  a.s = __fadd2_rn(a.s, acc[0]);
 }
 
 // Fold a tile into a first-argmax accumulator; v0 is the row index of the
