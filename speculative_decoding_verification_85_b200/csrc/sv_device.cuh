@@ -20,6 +20,8 @@ constexpr uint32_t kTagAccept = 1;
 constexpr uint32_t kTagGumbel = 2;
 constexpr uint32_t kTagMdEta = 3;
 constexpr uint32_t kTagMdGumbel = 4;
+constexpr uint32_t kTagGroup = 7;   // group-level noise of the single-draft draw
+constexpr int kRaceGroup = 1024;    // vocabulary entries per group of the single-draft draw
 
 // Pass-2 modes of a sequence.
 constexpr int kModeNone = 0;      // nothing to draw (greedy or invalid)

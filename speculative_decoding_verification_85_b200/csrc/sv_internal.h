@@ -66,6 +66,10 @@ Layout layout_single(int B, int gamma, int V, int dtype);
 int draw_chunks(int V);  // bound on draw CTAs per sequence (sv_single.cu)
 int row_segments(int V, int dtype);  // bound on row segments per row (sv_single.cu)
 Layout layout_multi(int B, int K, int L, int V, int dtype);
+// Small batches (sv_small.cu): whether a shape takes the one-cluster-per-
+// sequence kernel, and its launch.
+bool small_path(int B, int gamma, int V, int dtype);
+int launch_small(const CallParams& p1, int dtype, cudaStream_t stream);
 size_t multidraft_global_bytes(int B, int V);  // residual laws of the multi-draft kernel (sv_multi.cu)
 
 // Host helpers (sv_api.cu).

@@ -33,6 +33,7 @@
 #include <atomic>
 #include <climits>
 
+#include "sv_cluster.cuh"
 #include "sv_device.cuh"
 #include "sv_internal.h"
 #include "sv_rows.cuh"
@@ -92,46 +93,6 @@ struct alignas(16) MdSmem {
 };
 
 constexpr size_t kMdFixed = (sizeof(MdSmem) + 127) / 128 * 128;
-
-// Distributed-shared-memory stores that complete a transaction on the
-// destination CTA's mbarrier: the receiver waits on its own barrier, with no
-// cluster-wide barrier per exchange.
-__device__ __forceinline__ uint32_t mapa(const void* p, int rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_addr(p)), "r"(rank));
-  return r;
-}
-__device__ __forceinline__ void st_async_f64(uint32_t addr, double v, uint32_t bar) {
-  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b64 [%0], %1, [%2];"
-               ::"r"(addr), "l"(__double_as_longlong(v)), "r"(bar) : "memory");
-}
-__device__ __forceinline__ void st_async_f4(uint32_t addr, float4 v, uint32_t bar) {
-  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];"
-               ::"r"(addr), "r"(__float_as_uint(v.x)), "r"(__float_as_uint(v.y)),
-               "r"(__float_as_uint(v.z)), "r"(__float_as_uint(v.w)), "r"(bar)
-               : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_addr(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-// Bounded wait (kWaitLimitNs) for a phase of an exchange barrier.
-__device__ __forceinline__ bool xbar_wait(uint64_t* bar, uint32_t parity) {
-  if (mbar_try_wait_cluster(bar, parity)) return true;
-  const uint64_t t0 = global_ns();
-  for (;;) {
-    for (int k = 0; k < 64; ++k)
-      if (mbar_try_wait_cluster(bar, parity)) return true;
-    if (global_ns() - t0 > kWaitLimitNs) return false;
-  }
-}
 
 // The kMdC partials of an exchange, in rank order: thread t < nv contributes
 // `mine` as slot t of buffer `buf` to every CTA; after the cluster barrier
@@ -257,43 +218,11 @@ __global__ void __launch_bounds__(kMdT) md_cluster_kernel(const __grid_constant_
   }
   if constexpr (kLocal) {
     if (tvalid) {
-      // rows start at the same offset modulo 16 in shared and in global memory,
-      // so the aligned body of each row slice is one bulk copy
-      if (tid == 0) {
-        uint32_t total = 0;
-        for (int q = 0; q < nq; ++q) {
-          const uintptr_t ga = reinterpret_cast<uintptr_t>(grow(q) + static_cast<size_t>(v0) * es);
-          const uint32_t hb = min(static_cast<uint32_t>((16u - (ga & 15u)) & 15u), static_cast<uint32_t>(n * es));
-          total += (static_cast<uint32_t>(n * es) - hb) / 16u * 16u;
-        }
-        if (total) {
-          mbar_arrive_expect_tx(&sm.bar, total);
-          for (int q = 0; q < nq; ++q) {
-            const char* g = grow(q) + static_cast<size_t>(v0) * es;
-            const uintptr_t ga = reinterpret_cast<uintptr_t>(g);
-            const uint32_t hb = min(static_cast<uint32_t>((16u - (ga & 15u)) & 15u), static_cast<uint32_t>(n * es));
-            const uint32_t body = (static_cast<uint32_t>(n * es) - hb) / 16u * 16u;
-            char* sdst = srows + static_cast<size_t>(q) * p.rowstride + (ga & 15u);
-            if (body) bulk_g2s(sdst + hb, g + hb, body, &sm.bar);
-          }
-        } else {
-          mbar_arrive(&sm.bar);
-        }
-      }
-      // the unaligned head and tail of each row slice, as scalars
-      for (int q = 0; q < nq; ++q) {
-        const char* g = grow(q) + static_cast<size_t>(v0) * es;
-        const uintptr_t ga = reinterpret_cast<uintptr_t>(g);
-        const int hb = min(static_cast<int>((16u - (ga & 15u)) & 15u), static_cast<int>(n * es));
-        const int body = (static_cast<int>(n * es) - hb) / 16 * 16;
-        char* sdst = srows + static_cast<size_t>(q) * p.rowstride + (ga & 15u);
-        const int h = hb / static_cast<int>(es), t0 = (hb + body) / static_cast<int>(es);
-        for (int e = tid; e < h; e += kMdT) memcpy(sdst + e * es, g + e * es, es);
-        for (int e = t0 + tid; e < n; e += kMdT) memcpy(sdst + e * es, g + e * es, es);
-      }
-      // if the copies never completed, the slice's rows count as bad (NaN)
-      // and the whole sequence is reported invalid
-      stage_ok = mbar_wait(&sm.bar, 0);
+      // rows start at the same offset modulo 16 in shared and in global
+      // memory, so the aligned body of each row slice is one bulk copy; if
+      // the copies never completed, the slice's rows count as bad (NaN) and
+      // the whole sequence is reported invalid
+      stage_ok = stage_slices<es, kMdT>(grow, nq, v0, n, srows, p.rowstride, &sm.bar);
     }
   }
   __syncthreads();

@@ -25,6 +25,7 @@
 #include <atomic>
 #include <climits>
 
+#include "sv_decide.cuh"
 #include "sv_device.cuh"
 #include "sv_internal.h"
 #include "sv_rows.cuh"
@@ -32,138 +33,9 @@
 
 namespace sv {
 
-// Acceptance probability min(1, p/q) from log-probabilities (fp64); q = 0
-// accepts when p > 0, 0/0 rejects.
-__device__ __forceinline__ double accept_prob(double lp, double lq) {
-  if (lq == -INFINITY) return lp == -INFINITY ? 0.0 : 1.0;
-  const double r = exp(lp - lq);
-  return r < 1.0 ? r : 1.0;
-}
-
-// Warp 0 of the last-arriving CTA: validate, accept/reject, write outputs.
-// T is sequence b's temperature and x[0..gamma) its draft tokens (staged in
-// shared memory by the caller).
-template <bool kBf16>
-__device__ __noinline__ void decide_single(const CallParams& p, int b, float T, const int* x,
-                                           const RowAcc* rows, const float* zsel) {
-  const int lane = threadIdx.x & 31;
-  const int g = p.gamma;
-  const bool tvalid = (T >= 0.0f) && !isinf(T);
-  int32_t* tok = p.out_tokens + static_cast<size_t>(b) * (g + 1);
-
-  bool ok = tvalid;
-  int xi[2] = {0, 0};
-#pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    const int i = lane + 32 * h;
-    if (i < g) {
-      xi[h] = x[i];
-      ok = ok && xi[h] >= 0 && xi[h] < p.V;
-    }
-  }
-  if (tvalid) {
-    const bool greedy = (T == 0.0f);
-    for (int r = lane; r < p.rps; r += 32) {
-      const bool needed = !greedy || r <= g;
-      if (needed) {
-        const RowAcc& a = rows[r];
-        bool rv = !a.bad && isfinite(a.m);
-        if (!greedy) rv = rv && isfinite(__fdiv_rn(a.m, T));
-        ok = ok && rv;
-      }
-    }
-  }
-  ok = __all_sync(0xffffffffu, ok);
-  if (!ok) {
-    for (int i = lane; i <= g; i += 32) tok[i] = -1;
-    for (int i = lane; i < g; i += 32) {
-      if (p.out_lp) p.out_lp[static_cast<size_t>(b) * g + i] = __int_as_float(0x7fc00000);
-      if (p.out_lq) p.out_lq[static_cast<size_t>(b) * g + i] = __int_as_float(0x7fc00000);
-    }
-    if (lane == 0) {
-      p.accept_len[b] = -1;
-      p.info[b].mode = kModeNone;
-    }
-    return;
-  }
-
-  unsigned rej[2];
-  if (T == 0.0f) {
-    // Greedy: accept while the draft token is the first argmax of the raw row.
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int i = lane + 32 * h;
-      rej[h] = __ballot_sync(0xffffffffu, i < g && xi[h] != rows[i].arg);
-    }
-  } else {
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int i = lane + 32 * h;
-      bool reject = false;
-      if (i < g) {
-        constexpr size_t es = kBf16 ? 2 : 4;
-        const char* tr = static_cast<const char*>(p.target) +
-                         (static_cast<size_t>(b) * (g + 1) + i) * static_cast<size_t>(p.V) * es;
-        const char* dr = static_cast<const char*>(p.draft) +
-                         (static_cast<size_t>(b) * g + i) * static_cast<size_t>(p.V) * es;
-        const RowAcc& ap = rows[i];
-        const RowAcc& aq = rows[g + 1 + i];
-        // d = fl32(fl32(z_x / T) - fl32(zmax / T)): the same fp32 operations
-        // as scaling the whole row and shifting by its maximum.
-        // the draft token's logits were picked up while the rows streamed
-        const float zp = zsel ? zsel[2 * i] : logit_at<kBf16>(tr, xi[h]);
-        const float zq = zsel ? zsel[2 * i + 1] : logit_at<kBf16>(dr, xi[h]);
-        const float dp = __fsub_rn(__fdiv_rn(zp, T), __fdiv_rn(ap.m, T));
-        const float dq = __fsub_rn(__fdiv_rn(zq, T), __fdiv_rn(aq.m, T));
-        const double lp = static_cast<double>(dp) - log(static_cast<double>(ap.s));
-        const double lq = static_cast<double>(dq) - log(static_cast<double>(aq.s));
-        const uint4 rnd = keyed_block(p.seed, p.step, kTagAccept, b, 0, i, i);
-        const double u = accept_uniform(rnd.x);
-        reject = !(u < accept_prob(lp, lq));
-        if (p.out_lp) p.out_lp[static_cast<size_t>(b) * g + i] = static_cast<float>(lp);
-        if (p.out_lq) p.out_lq[static_cast<size_t>(b) * g + i] = static_cast<float>(lq);
-      }
-      rej[h] = __ballot_sync(0xffffffffu, reject);
-    }
-  }
-  const int j = rej[0] ? __ffs(rej[0]) - 1 : (rej[1] ? 32 + __ffs(rej[1]) - 1 : g);
-
-  for (int i = lane; i <= g; i += 32) tok[i] = i < j ? x[i] : -1;
-  if (T == 0.0f) {
-    for (int i = lane; i < g; i += 32) {
-      if (p.out_lp) p.out_lp[static_cast<size_t>(b) * g + i] = __int_as_float(0x7fc00000);
-      if (p.out_lq) p.out_lq[static_cast<size_t>(b) * g + i] = __int_as_float(0x7fc00000);
-    }
-  }
-  __syncwarp();
-  if (lane == 0) {
-    p.accept_len[b] = j;
-    SeqInfo si{};
-    if (T == 0.0f) {
-      tok[j] = rows[j].arg;
-      si.mode = kModeNone;
-    } else {
-      const float c = __fdiv_rn(kLog2e, T);
-      si.mode = j < g ? kModeResidual : kModeBonus;
-      si.j = j;
-      si.c = c;
-      si.zmp = rows[j].m;
-      si.lsp = log2f(rows[j].s);
-      if (j < g) {
-        si.zmq = rows[g + 1 + j].m;
-        si.lsq = log2f(rows[g + 1 + j].s);
-      }
-    }
-    p.info[b] = si;
-  }
-}
-
-
 // ------------------------------------------------------------------ layout
 constexpr int kRowThreads = kTileThreads;  // 256
 constexpr int kDrawThreads = 256;
-constexpr int kRaceGroup = 1024;           // vocabulary entries per group of the draw race
-constexpr uint32_t kTagGroup = 7;          // Philox tag of the group-level noise
 constexpr int kDrawWaves = 4;              // about this many waves of draw CTAs per call
 constexpr int kPrefetchTiles = 1;          // row tiles requested into L2 ahead of the loads
 static_assert(kRowThreads == kDrawThreads, "one thread count for both kernels");
@@ -434,7 +306,7 @@ __global__ void __launch_bounds__(kRowThreads, 3) rows_kernel(const __grid_const
   if (!s_last) return;
   combine_pairs(f, b, argmaxA, c, rows, s_zsel);
   if (tid < 32) {
-    decide_single<kBf16>(p, b, T, s_tok, rows, s_zsel);
+    decide_single<kBf16>(p, b, T, s_tok, rows, s_zsel, p.info + b, true);
     // publish the decision: every lane's writes, then the flag (release)
     __threadfence();
     __syncwarp();
@@ -876,6 +748,9 @@ int launch_single(const void* target, const void* draft, const int32_t* tokens,
   p1.out_tokens = out_tokens;
   p1.out_lp = out_lp;
   p1.out_lq = out_lq;
+  // a batch whose sequences fit one cluster each, in one wave, with every
+  // row slice in shared memory: the latency-bound case, one cluster kernel
+  if (small_path(B, gamma, V, dtype)) return launch_small(p1, dtype, stream);
   // Row segments: whole tiles, about kRowWaves waves of CTAs over the GPU but
   // at most kMaxSegTiles tiles per CTA; balanced so segments differ by at
   // most one tile.  Long segments spread each CTA's fixed cost (launch, block
