@@ -99,14 +99,16 @@ __device__ __forceinline__ bool stage_slices(RowFn grow, int nq, int v0, int n, 
 
 // The same staging with one barrier per row (bars[q], initialised, phase
 // 0), issued without waiting: thread 0 issues the bulk copies in row order
-// and all kThreads threads copy the unaligned heads and tails.  After a CTA
-// barrier (which orders those scalar copies) a thread may use row q once
-// mbar_wait(&bars[q], 0) returns true, so a row is processed while later
-// rows are still in flight.
+// and all kThreads threads copy the unaligned heads and tails.  Returns
+// whether there were any (the same answer in every thread); if so, a CTA
+// barrier must order those scalar copies before use.  A thread may use row q
+// once mbar_wait(&bars[q], 0) returns true, so a row is processed while
+// later rows are still in flight.
 template <size_t es, int kThreads, typename RowFn>
-__device__ __forceinline__ void stage_rows_issue(RowFn grow, int nq, int v0, int n, char* srows,
+__device__ __forceinline__ bool stage_rows_issue(RowFn grow, int nq, int v0, int n, char* srows,
                                                  int rowstride, uint64_t* bars) {
   const int tid = threadIdx.x;
+  bool scalar = false;  // some row slice has an unaligned head or tail
   for (int q = 0; q < nq; ++q) {
     const char* g = grow(q) + static_cast<size_t>(v0) * es;
     const uintptr_t ga = reinterpret_cast<uintptr_t>(g);
@@ -122,9 +124,11 @@ __device__ __forceinline__ void stage_rows_issue(RowFn grow, int nq, int v0, int
       }
     }
     const int h = static_cast<int>(hb / es), t0 = static_cast<int>((hb + body) / es);
+    scalar = scalar || h > 0 || t0 < n;
     for (int e = tid; e < h; e += kThreads) memcpy(sdst + e * es, g + e * es, es);
     for (int e = t0 + tid; e < n; e += kThreads) memcpy(sdst + e * es, g + e * es, es);
   }
+  return scalar;
 }
 
 }  // namespace sv

@@ -84,7 +84,8 @@ struct alignas(16) MdSmem {
   int H[SV_MAX_DRAFTS];                // rejected tokens at tau
   float4 race[kMdW];
   const char* rowp[kMaxStatRows];      // this slice's entry 0 of row q (shared or global memory)
-  uint64_t bar;                        // staging barrier
+  uint64_t rbar[kMaxStatRows];         // staging barriers, one per row
+  float eta[kMaxDraftTokens];          // sub-block acceptance uniforms [K][L]
   uint64_t xbar[2];                    // exchange barriers (one per exchange buffer)
   uint32_t xphase[2];                  // their current phase parity
   int xfail;                           // an exchange wait ran out of time
@@ -194,76 +195,117 @@ __global__ void __launch_bounds__(kMdT) md_cluster_kernel(const __grid_constant_
   }
   auto zrow = [&](int q, int e) -> float { return zat(sm.rowp[q], e); };
 
-  // ---- draft tokens and their logits; staging of the slice's rows
-  bool stage_ok = true;
+  // ---- staging of the slice's rows (a bulk copy and a barrier per row;
+  // rows start at the same offset modulo 16 in shared and in global memory,
+  // so the aligned body of each row slice is one bulk copy), then the draft
+  // tokens, their logits and the sub-block acceptance uniforms while the
+  // rows are in flight
   if (tid == 0) {
-    mbar_init(&sm.bar, 1);
+    if (kLocal && tvalid)
+      for (int q = 0; q < nq; ++q) mbar_init(&sm.rbar[q], 1);
     mbar_init(&sm.xbar[0], 1);
     mbar_init(&sm.xbar[1], 1);
     sm.xphase[0] = sm.xphase[1] = 0u;
     sm.xfail = 0;
     mbar_init_fence();
   }
-  cl.sync();  // every CTA's barriers are initialised before any remote store
-  for (int t = tid; t < K * L; t += kMdT) {
-    const int x = __ldg(p.tokens + static_cast<size_t>(b) * K * L + t);
+  __syncthreads();  // the barriers are initialised before any thread waits on them
+  bool scalar_copies = false;
+  if constexpr (kLocal) {
+    if (tvalid) scalar_copies = stage_rows_issue<es, kMdT>(grow, nq, v0, n, srows, p.rowstride, sm.rbar);
+  }
+  // every CTA's barriers are initialised before any remote store: arrive
+  // now, wait just before the first exchange
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+  // draft token t of the sequence ([K][L] order): the token, its two logits
+  // and its sub-block acceptance uniform ((x >> 8) 2^-24, exact in fp32)
+  auto token_info = [&](int t, int& x, float2& z, float& u) {
+    x = __ldg(p.tokens + static_cast<size_t>(b) * K * L + t);
     const int k = t / L, i = t - k * L, set = p.per_draft ? k : 0;
-    sm.tok[t] = x;
-    float2 z = make_float2(__int_as_float(0x7fc00000), __int_as_float(0x7fc00000));
+    z = make_float2(__int_as_float(0x7fc00000), __int_as_float(0x7fc00000));
     if (tvalid && !greedy && x >= 0 && x < V) {
       z.x = logit_at<kBf16>(grow(qt(set, i)), x);
       z.y = logit_at<kBf16>(grow(qd(set, i)), x);
     }
-    sm.zg[t] = z;
-  }
-  if constexpr (kLocal) {
-    if (tvalid) {
-      // rows start at the same offset modulo 16 in shared and in global
-      // memory, so the aligned body of each row slice is one bulk copy; if
-      // the copies never completed, the slice's rows count as bad (NaN) and
-      // the whole sequence is reported invalid
-      stage_ok = stage_slices<es, kMdT>(grow, nq, v0, n, srows, p.rowstride, &sm.bar);
-    }
-  }
-  __syncthreads();
+    u = static_cast<float>(accept_uniform(keyed_block(p.seed, p.step, kTagMdEta, b, k, i, i).x));
+  };
+  // the first kMdT tokens, by the highest threads (whose warps have no row
+  // when the rows are fewer than the warps): loaded now, stored after the
+  // row statistics
+  const int tt = kMdT - 1 - tid;
+  int x0 = 0;
+  float2 z0 = make_float2(0.0f, 0.0f);
+  float u0 = 0.0f;
+  if (tt < K * L) token_info(tt, x0, z0, u0);
+  if (scalar_copies) __syncthreads();  // the scalar head and tail copies
 
-  // ---- 1. row statistics: slice partials, one exchange per batch of rows,
+  // ---- 1. row statistics of the slice: a warp per row (q = warp, warp +
+  // kMdW, ...; lane l takes entries l, l + 32, ...) as soon as the row has
+  // landed: the maximum (NaN-propagating; for greedy rows with its first
+  // index), then the scaled sum s = sum_v 2^{(z_v - m) c} against it, each
+  // with four independent chains; then one exchange per batch of rows,
   // merged in rank order
   int buf = 0;
   bool row_ok = true;
   {
     const float c = tvalid && !greedy ? __fdiv_rn(kLog2e, T) : 0.0f;
-    for (int q0 = 0; q0 < nq; q0 += kXBatch) {
-      const int nb = min(kXBatch, nq - q0);
-      for (int j = 0; j < nb; ++j) {
-        RowAcc a{-INFINITY, 0.0f, 0x7fffffff, stage_ok ? 0 : 1};
-        const char* rp = sm.rowp[q0 + j];
-        if (tvalid)
-          for (int e = tid; e < n; e += kMdT) {
+    float4* part = &sm.wpart[0][0];  // [nq] this slice's row statistics
+    for (int q = warp; q < nq; q += kMdW) {
+      bool landed = true;
+      if constexpr (kLocal) landed = !tvalid || mbar_wait(&sm.rbar[q], 0);
+      const char* gq = grow(q) + static_cast<size_t>(v0) * es;
+      const char* rp = kLocal ? srows + static_cast<size_t>(q) * p.rowstride + (reinterpret_cast<uintptr_t>(gq) & 15u) : gq;
+      float m = -INFINITY, sum = 0.0f;
+      int arg = 0x7fffffff, bad = landed ? 0 : 1;
+      if (tvalid && landed) {
+        if (greedy) {
+          for (int e = lane; e < n; e += 32) {
             const float z = zat(rp, e);
-            if (greedy) acc_scalar<kRowArgmax>(a, z, v0 + e, c); else acc_scalar<kRowLse>(a, z, v0 + e, c);
+            if (z != z) bad = 1;
+            else if (z > m) {
+              m = z;
+              arg = v0 + e;
+            }
           }
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) {
-          RowAcc o;
-          o.m = __shfl_down_sync(0xffffffffu, a.m, off);
-          o.s = __shfl_down_sync(0xffffffffu, a.s, off);
-          o.arg = __shfl_down_sync(0xffffffffu, a.arg, off);
-          o.bad = __shfl_down_sync(0xffffffffu, a.bad, off);
-          if (greedy) acc_merge<kRowArgmax>(a, o, c); else acc_merge<kRowLse>(a, o, c);
+          for (int off = 16; off > 0; off >>= 1) {
+            const float m2 = __shfl_xor_sync(0xffffffffu, m, off);
+            const int a2 = __shfl_xor_sync(0xffffffffu, arg, off);
+            argmax_merge(m, arg, m2, a2);
+          }
+        } else {
+          float mk[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+          for (int e0 = lane; e0 < n; e0 += 128)
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              if (e0 + 32 * k < n) mk[k] = max_nan(mk[k], zat(rp, e0 + 32 * k));
+          m = max_nan(max_nan(mk[0], mk[1]), max_nan(mk[2], mk[3]));
+#pragma unroll
+          for (int off = 16; off > 0; off >>= 1) m = max_nan(m, __shfl_xor_sync(0xffffffffu, m, off));
+          if (m != m) {
+            bad = 1;
+          } else if (m != -INFINITY) {
+            float sk[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+            for (int e0 = lane; e0 < n; e0 += 128)
+#pragma unroll
+              for (int k = 0; k < 4; ++k)
+                if (e0 + 32 * k < n) sk[k] += ex2_approx((zat(rp, e0 + 32 * k) - m) * c);
+            sum = (sk[0] + sk[1]) + (sk[2] + sk[3]);
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+          }
         }
-        if (lane == 0) sm.wpart[warp][j] = make_float4(a.m, a.s, __int_as_float(a.arg), __int_as_float(a.bad));
+        bad = __any_sync(0xffffffffu, bad) ? 1 : 0;
       }
+      if (lane == 0) part[q] = make_float4(m, sum, __int_as_float(arg), __int_as_float(bad));
+    }
+    __syncthreads();
+    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+    for (int q0 = 0; q0 < nq; q0 += kXBatch) {
+      const int nb = min(kXBatch, nq - q0);
       if (tid == 0) mbar_arrive_expect_tx(&sm.xbar[buf], static_cast<uint32_t>(nb * kMdC * sizeof(float4)));
-      __syncthreads();
       if (tid < nb) {
-        RowAcc a{-INFINITY, 0.0f, 0x7fffffff, 0};
-        for (int w = 0; w < kMdW; ++w) {
-          const float4 x = sm.wpart[w][tid];
-          const RowAcc o{x.x, x.y, __float_as_int(x.z), __float_as_int(x.w)};
-          if (greedy) acc_merge<kRowArgmax>(a, o, c); else acc_merge<kRowLse>(a, o, c);
-        }
-        const float4 v = make_float4(a.m, a.s, __int_as_float(a.arg), __int_as_float(a.bad));
+        const float4 v = part[q0 + tid];
         for (int r = 0; r < kMdC; ++r)
           st_async_f4(mapa(&sm.xb[buf][rank][2 * tid], r), v, mapa(&sm.xbar[buf], r));
       }
@@ -283,12 +325,27 @@ __global__ void __launch_bounds__(kMdT) md_cluster_kernel(const __grid_constant_
         if (!greedy) rv = rv && isfinite(__fdiv_rn(a.m, T));
         row_ok = row_ok && rv;
       }
-      __syncthreads();  // wpart is reused by the next batch
+      __syncthreads();  // every thread has read the buffer
       if (tid == 0) sm.xphase[buf] ^= 1u;
       buf ^= 1;
       __syncthreads();
     }
   }
+  if (tt < K * L) {
+    sm.tok[tt] = x0;
+    sm.zg[tt] = z0;
+    sm.eta[tt] = u0;
+  }
+  for (int t = kMdT + tid; t < K * L; t += kMdT) {  // more than kMdT draft tokens
+    int x;
+    float2 z;
+    float u;
+    token_info(t, x, z, u);
+    sm.tok[t] = x;
+    sm.zg[t] = z;
+    sm.eta[t] = u;
+  }
+  __syncthreads();
   // validity: temperature, rows, tokens (the same in every CTA of the cluster)
   bool ok = tvalid && row_ok && !sm.xfail;
   for (int t = tid; t < K * L; t += kMdT) ok = ok && sm.tok[t] >= 0 && sm.tok[t] < V;
@@ -458,8 +515,7 @@ __global__ void __launch_bounds__(kMdT) md_cluster_kernel(const __grid_constant_
         } else {
           h = w;
         }
-        const uint4 rnd = keyed_block(p.seed, p.step, kTagMdEta, b, k, i, i);
-        if (accept_uniform(rnd.x) < h) {
+        if (static_cast<double>(sm.eta[k * L + i]) < h) {
           best = i + 1;
           wbest = w;
         }

@@ -38,6 +38,7 @@ constexpr int kSdC = 8;      // CTAs per cluster (one sequence)
 constexpr int kSdT = 512;    // threads per CTA
 constexpr int kSdW = kSdT / 32;
 constexpr int kSdBatch = 32; // row statistics per exchange
+static_assert(SV_MAX_GAMMA <= kSdT, "one thread per draft token");
 constexpr int kSdMaxUnits = 64;               // level-1 work units (group parts) per slice
 
 struct SdParams {
@@ -129,18 +130,19 @@ __global__ void __launch_bounds__(kSdT) sd_cluster_kernel(const __grid_constant_
     sm.xfail = 0;
     mbar_init_fence();
   }
-  stage_rows_issue<es, kSdT>(grow, nall, v0, n, srows, f.rowstride, sm.rbar);
+  __syncthreads();  // the barriers are initialised before any thread waits on them
+  const bool scalar_copies = stage_rows_issue<es, kSdT>(grow, nall, v0, n, srows, f.rowstride, sm.rbar);
   // every CTA's barriers are initialised before any remote store: arrive
   // now, wait just before the first exchange
   asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
-  // the temperature and the draft tokens (thread i < gamma), then the draft
-  // tokens' two logits: loads issued now, stored to shared memory before the
-  // decision
+  // the temperature and the draft tokens (draft token i by thread
+  // kSdT - 1 - i, a warp without a row when the rows are fewer than the
+  // warps), then the draft tokens' two logits: loads issued now, stored to
+  // shared memory before the decision
   const float T = __ldg(p.temps + b);
-  int xi[2] = {0, 0};
-#pragma unroll
-  for (int h = 0; h < 2; ++h)
-    if (tid + kSdT * h < g) xi[h] = __ldg(p.tokens + static_cast<size_t>(b) * g + tid + kSdT * h);
+  const int ti = kSdT - 1 - tid;  // this thread's draft token (if ti < gamma)
+  int xi = 0;
+  if (ti < g) xi = __ldg(p.tokens + static_cast<size_t>(b) * g + ti);
   const bool tvalid = (T >= 0.0f) && !isinf(T);
   const bool greedy = tvalid && T == 0.0f;
   const int nq = greedy ? g + 1 : nall;  // rows the sequence reads
@@ -154,19 +156,12 @@ __global__ void __launch_bounds__(kSdT) sd_cluster_kernel(const __grid_constant_
     else
       return reinterpret_cast<const float*>(rp)[e];
   };
-  float zp[2], zq[2];
-#pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    const int i = tid + kSdT * h;
-    zp[h] = zq[h] = __int_as_float(0x7fc00000);
-    if (i < g) {
-      if (tvalid && !greedy && xi[h] >= 0 && xi[h] < V) {
-        zp[h] = logit_at<kBf16>(grow(i), xi[h]);
-        zq[h] = logit_at<kBf16>(grow(g + 1 + i), xi[h]);
-      }
-    }
+  float zp = __int_as_float(0x7fc00000), zq = zp;
+  if (ti < g && tvalid && !greedy && xi >= 0 && xi < V) {
+    zp = logit_at<kBf16>(grow(ti), xi);
+    zq = logit_at<kBf16>(grow(g + 1 + ti), xi);
   }
-  __syncthreads();  // the scalar head and tail copies
+  if (scalar_copies) __syncthreads();  // the scalar head and tail copies
 
   // ---- 1. row statistics of the slice: a warp per row (q = warp, warp +
   // kSdW, ...; lane l takes entries l, l + 32, ...) as soon as the row has
@@ -179,7 +174,8 @@ __global__ void __launch_bounds__(kSdT) sd_cluster_kernel(const __grid_constant_
     const float c = tvalid && !greedy ? __fdiv_rn(kLog2e, T) : 0.0f;
     for (int q = warp; q < nq; q += kSdW) {
       const bool landed = mbar_wait(&sm.rbar[q], 0);
-      const char* rp = sm.rowp[q];
+      const char* rp = srows + static_cast<size_t>(q) * f.rowstride +
+                       (reinterpret_cast<uintptr_t>(grow(q) + static_cast<size_t>(v0) * es) & 15u);
       float m = -INFINITY, sum = 0.0f;
       int arg = 0x7fffffff, bad = landed ? 0 : 1;
       if (tvalid && landed) {
@@ -244,14 +240,10 @@ __global__ void __launch_bounds__(kSdT) sd_cluster_kernel(const __grid_constant_
   }
 
   // ---- 2. the decision, in every CTA (rank 0 writes the outputs)
-#pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    const int i = tid + kSdT * h;
-    if (i < g) {
-      sm.tok[i] = xi[h];
-      sm.zsel[2 * i] = zp[h];
-      sm.zsel[2 * i + 1] = zq[h];
-    }
+  if (ti < g) {
+    sm.tok[ti] = xi;
+    sm.zsel[2 * ti] = zp;
+    sm.zsel[2 * ti + 1] = zq;
   }
   __syncthreads();
   if (warp == 0) decide_single<kBf16>(p, b, T, sm.tok, sm.rows, sm.zsel, &sm.si, rank == 0);
