@@ -1,12 +1,13 @@
 // sv_multi.cu -- multi-draft verification, "SpecTr-GBV: Multi-Draft Block
 // Verification Accelerating Speculative Decoding", Methodology, Algorithm 1.
 //
-// One thread-block cluster of kMdC CTAs per sequence; CTA `rank` owns the
+// One thread-block cluster of kC CTAs per sequence (16 when the batch's
+// clusters fit in one wave, else 8); CTA `rank` owns the
 // vocabulary slice [rank * slice, (rank + 1) * slice).  Every V-wide quantity
 // of the algorithm is a sum (or a race) over the slices: each CTA reduces its
 // slice, writes its partial into every CTA's exchange buffer through
 // distributed shared memory, and after one cluster barrier every CTA adds the
-// kMdC partials in rank order -- so every CTA holds the same value and takes
+// kC partials in rank order -- so every CTA holds the same value and takes
 // the same decisions, with no further communication.  The steps:
 //   1. row statistics (maximum, softmax sum, first argmax) of the L + 1 target
 //      and L draft rows (one exchange);
@@ -42,13 +43,11 @@ namespace cg = cooperative_groups;
 
 namespace sv {
 
-constexpr int kMdC = 8;                          // CTAs per cluster (one sequence)
 constexpr int kMdT = 512;                        // threads per CTA
 constexpr int kMdW = kMdT / 32;
-constexpr int kXBatch = 64;                      // row statistics per exchange
+constexpr int kXBatch = 32;                      // row statistics per exchange
 constexpr int kXSlot = 2 * kXBatch;              // doubles per rank in an exchange buffer
 constexpr int kMaxStatRows = 256;                // row statistics per sequence (all row sets)
-constexpr int kMaxDraftTokens = SV_MAX_DRAFTS * SV_MAX_GAMMA;
 static_assert(SV_MAX_GAMMA <= kXSlot, "an exchange carries every A_i of a draft");
 
 struct MdcParams {
@@ -69,23 +68,22 @@ struct MdcParams {
 };
 
 // Fixed part of the dynamic shared memory (the local variant adds the R
-// buffers and the staged rows after it).
+// buffers and the staged rows after it), for clusters of kC CTAs.
+template <int kC>
 struct alignas(16) MdSmem {
-  double xb[2][kMdC][kXSlot];          // exchange buffers (written by every rank)
-  float4 wpart[kMdW][kXBatch];         // per-warp row statistics of a batch
+  double xb[2][kC][kXSlot];            // exchange buffers (written by every rank)
+  float4 part[kMaxStatRows];           // this slice's row statistics
   double wred[kMdW][SV_MAX_GAMMA];     // per-warp partial sums
   double res[kXSlot];                  // results of the last exchange
   float m[kMaxStatRows];               // row maxima
   float is[kMaxStatRows];              // 1 / s, s = sum_v 2^{(z_v - m) c}
   int arg[kMaxStatRows];               // first argmax (greedy target rows)
   double w[SV_MAX_GAMMA];              // the current draft's sub-block weights
-  int tok[kMaxDraftTokens];            // draft tokens [K][L]
-  float2 zg[kMaxDraftTokens];          // target / draft logit at each draft token
+  double num[SV_MAX_GAMMA], den[SV_MAX_GAMMA];  // their step ratios
   int H[SV_MAX_DRAFTS];                // rejected tokens at tau
   float4 race[kMdW];
   const char* rowp[kMaxStatRows];      // this slice's entry 0 of row q (shared or global memory)
   uint64_t rbar[kMaxStatRows];         // staging barriers, one per row
-  float eta[kMaxDraftTokens];          // sub-block acceptance uniforms [K][L]
   uint64_t xbar[2];                    // exchange barriers (one per exchange buffer)
   uint32_t xphase[2];                  // their current phase parity
   int xfail;                           // an exchange wait ran out of time
@@ -93,27 +91,37 @@ struct alignas(16) MdSmem {
   int tau, a, nH, skip, best, rcur;
 };
 
-constexpr size_t kMdFixed = (sizeof(MdSmem) + 127) / 128 * 128;
+template <int kC>
+constexpr size_t md_fixed() {
+  return (sizeof(MdSmem<kC>) + 127) / 128 * 128;
+}
 
-// The kMdC partials of an exchange, in rank order: thread t < nv contributes
-// `mine` as slot t of buffer `buf` to every CTA; after the cluster barrier
+// The draft tokens' arrays follow the fixed part: [K][L] target / draft
+// logits at the token (float2), tokens (int), sub-block acceptance uniforms
+// (float); 16 bytes per draft token, rounded up to 128.
+__host__ __device__ constexpr size_t md_token_bytes(int K, int L) {
+  return (static_cast<size_t>(K) * L * 16 + 127) / 128 * 128;
+}
+
+// The kC partials of an exchange, in rank order: thread t < nv contributes
+// `mine` as slot t of buffer `buf` to every CTA; once they have all arrived
 // thread t adds slot t over the ranks into sm.res[t]; ends with a CTA barrier.
-template <typename Cl>
-__device__ __forceinline__ void exchange(Cl& cl, MdSmem& sm, int buf, int nv, double mine) {
+template <int kC, typename Cl>
+__device__ __forceinline__ void exchange(Cl& cl, MdSmem<kC>& sm, int buf, int nv, double mine) {
   const int tid = threadIdx.x;
   const int rank = static_cast<int>(cl.block_rank());
   // every rank sends nv values to every rank: arm this CTA's barrier for them
-  if (tid == 0) mbar_arrive_expect_tx(&sm.xbar[buf], static_cast<uint32_t>(nv * kMdC * sizeof(double)));
+  if (tid == 0) mbar_arrive_expect_tx(&sm.xbar[buf], static_cast<uint32_t>(nv * kC * sizeof(double)));
   if (tid < nv) {
     // the CTA's earlier shared-memory writes (R, read remotely later) are
     // ordered before the values that announce them (callers end with a CTA barrier)
     asm volatile("fence.acq_rel.cluster;" ::: "memory");
-    for (int q = 0; q < kMdC; ++q) st_async_f64(mapa(&sm.xb[buf][rank][tid], q), mine, mapa(&sm.xbar[buf], q));
+    for (int q = 0; q < kC; ++q) st_async_f64(mapa(&sm.xb[buf][rank][tid], q), mine, mapa(&sm.xbar[buf], q));
   }
   if (!xbar_wait(&sm.xbar[buf], sm.xphase[buf])) sm.xfail = 1;
   if (tid < nv) {
     double s = 0.0;
-    for (int q = 0; q < kMdC; ++q) s += sm.xb[buf][q][tid];
+    for (int q = 0; q < kC; ++q) s += sm.xb[buf][q][tid];
     sm.res[tid] = s;
   }
   __syncthreads();
@@ -122,7 +130,8 @@ __device__ __forceinline__ void exchange(Cl& cl, MdSmem& sm, int buf, int nv, do
 }
 
 // One value slot v of a CTA-wide sum: each warp's total lands in sm.wred[warp][v].
-__device__ __forceinline__ void warp_sum_to(MdSmem& sm, int v, double x) {
+template <int kC>
+__device__ __forceinline__ void warp_sum_to(MdSmem<kC>& sm, int v, double x) {
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) x += __shfl_down_sync(0xffffffffu, x, off);
   if ((threadIdx.x & 31) == 0) sm.wred[threadIdx.x >> 5][v] = x;
@@ -136,14 +145,14 @@ __device__ __forceinline__ double step_weight(double w, double num, double den) 
   return (w > 0.0 && num > 0.0) ? 1.0 : 0.0;
 }
 
-template <bool kBf16, bool kLocal>
+template <bool kBf16, bool kLocal, int kC>
 __global__ void __launch_bounds__(kMdT) md_cluster_kernel(const __grid_constant__ MdcParams p) {
   constexpr size_t es = kBf16 ? 2 : 4;
   extern __shared__ __align__(128) char dyn[];
-  MdSmem& sm = *reinterpret_cast<MdSmem*>(dyn);
+  MdSmem<kC>& sm = *reinterpret_cast<MdSmem<kC>*>(dyn);
   cg::cluster_group cl = cg::this_cluster();
   const int rank = static_cast<int>(cl.block_rank());
-  const int b = blockIdx.x / kMdC;
+  const int b = blockIdx.x / kC;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int K = p.K, L = p.L, V = p.V, rps = 2 * L + 1;
   const int nsets = p.per_draft ? K : 1;
@@ -166,12 +175,17 @@ __global__ void __launch_bounds__(kMdT) md_cluster_kernel(const __grid_constant_
   };
   auto qt = [&](int set, int i) { return set * nrows + i; };          // target row i of a set
   auto qd = [&](int set, int i) { return set * nrows + L + 1 + i; };  // draft row i of a set
+  char* const tokreg = dyn + md_fixed<kC>();
+  float2* const s_zg = reinterpret_cast<float2*>(tokreg);
+  int* const s_tok = reinterpret_cast<int*>(tokreg + static_cast<size_t>(K) * L * sizeof(float2));
+  float* const s_eta = reinterpret_cast<float*>(tokreg + static_cast<size_t>(K) * L * (sizeof(float2) + sizeof(int)));
+  char* const dynrest = tokreg + md_token_bytes(K, L);
   float* Rb[2];
   char* srows = nullptr;
   if constexpr (kLocal) {
-    Rb[0] = reinterpret_cast<float*>(dyn + kMdFixed);
+    Rb[0] = reinterpret_cast<float*>(dynrest);
     Rb[1] = Rb[0] + p.slice;
-    srows = dyn + kMdFixed + 2 * static_cast<size_t>(p.slice) * sizeof(float);
+    srows = dynrest + 2 * static_cast<size_t>(p.slice) * sizeof(float);
   } else {
     Rb[0] = p.Rws + static_cast<size_t>(b) * 2 * V + v0;
     Rb[1] = Rb[0] + V;
@@ -249,7 +263,7 @@ __global__ void __launch_bounds__(kMdT) md_cluster_kernel(const __grid_constant_
   bool row_ok = true;
   {
     const float c = tvalid && !greedy ? __fdiv_rn(kLog2e, T) : 0.0f;
-    float4* part = &sm.wpart[0][0];  // [nq] this slice's row statistics
+    float4* part = sm.part;  // [nq] this slice's row statistics
     for (int q = warp; q < nq; q += kMdW) {
       bool landed = true;
       if constexpr (kLocal) landed = !tvalid || mbar_wait(&sm.rbar[q], 0);
@@ -303,16 +317,16 @@ __global__ void __launch_bounds__(kMdT) md_cluster_kernel(const __grid_constant_
     asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
     for (int q0 = 0; q0 < nq; q0 += kXBatch) {
       const int nb = min(kXBatch, nq - q0);
-      if (tid == 0) mbar_arrive_expect_tx(&sm.xbar[buf], static_cast<uint32_t>(nb * kMdC * sizeof(float4)));
+      if (tid == 0) mbar_arrive_expect_tx(&sm.xbar[buf], static_cast<uint32_t>(nb * kC * sizeof(float4)));
       if (tid < nb) {
         const float4 v = part[q0 + tid];
-        for (int r = 0; r < kMdC; ++r)
+        for (int r = 0; r < kC; ++r)
           st_async_f4(mapa(&sm.xb[buf][rank][2 * tid], r), v, mapa(&sm.xbar[buf], r));
       }
       if (!xbar_wait(&sm.xbar[buf], sm.xphase[buf])) sm.xfail = 1;
       if (tid < nb) {
         RowAcc a{-INFINITY, 0.0f, 0x7fffffff, 0};
-        for (int r = 0; r < kMdC; ++r) {
+        for (int r = 0; r < kC; ++r) {
           const float4 x = *reinterpret_cast<const float4*>(&sm.xb[buf][r][2 * tid]);
           const RowAcc o{x.x, x.y, __float_as_int(x.z), __float_as_int(x.w)};
           if (greedy) acc_merge<kRowArgmax>(a, o, c); else acc_merge<kRowLse>(a, o, c);
@@ -332,23 +346,23 @@ __global__ void __launch_bounds__(kMdT) md_cluster_kernel(const __grid_constant_
     }
   }
   if (tt < K * L) {
-    sm.tok[tt] = x0;
-    sm.zg[tt] = z0;
-    sm.eta[tt] = u0;
+    s_tok[tt] = x0;
+    s_zg[tt] = z0;
+    s_eta[tt] = u0;
   }
   for (int t = kMdT + tid; t < K * L; t += kMdT) {  // more than kMdT draft tokens
     int x;
     float2 z;
     float u;
     token_info(t, x, z, u);
-    sm.tok[t] = x;
-    sm.zg[t] = z;
-    sm.eta[t] = u;
+    s_tok[t] = x;
+    s_zg[t] = z;
+    s_eta[t] = u;
   }
   __syncthreads();
   // validity: temperature, rows, tokens (the same in every CTA of the cluster)
   bool ok = tvalid && row_ok && !sm.xfail;
-  for (int t = tid; t < K * L; t += kMdT) ok = ok && sm.tok[t] >= 0 && sm.tok[t] < V;
+  for (int t = tid; t < K * L; t += kMdT) ok = ok && s_tok[t] >= 0 && s_tok[t] < V;
   ok = __syncthreads_and(ok);
   int32_t* tok = p.out_tokens + static_cast<size_t>(b) * (L + 1);
   if (!ok) {
@@ -372,7 +386,7 @@ __global__ void __launch_bounds__(kMdT) md_cluster_kernel(const __grid_constant_
       for (int k = 0; k < K; ++k) {
         const int set = p.per_draft ? k : 0;
         int m = 0;
-        while (m < L && sm.tok[k * L + m] == sm.arg[qt(set, m)]) ++m;
+        while (m < L && s_tok[k * L + m] == sm.arg[qt(set, m)]) ++m;
         if (m > tau) {
           tau = m;
           a = k;
@@ -380,7 +394,7 @@ __global__ void __launch_bounds__(kMdT) md_cluster_kernel(const __grid_constant_
       }
       const int sa = p.per_draft && a >= 0 ? a : 0;
       for (int i = 0; i <= L; ++i)
-        tok[i] = i < tau ? sm.tok[a * L + i] : (i == tau ? sm.arg[qt(sa, tau)] : -1);
+        tok[i] = i < tau ? s_tok[a * L + i] : (i == tau ? sm.arg[qt(sa, tau)] : -1);
       p.accept_len[b] = tau;
       if (p.out_draft_index) p.out_draft_index[b] = a;
     }
@@ -434,45 +448,62 @@ __global__ void __launch_bounds__(kMdT) md_cluster_kernel(const __grid_constant_
   // ---- 3. the drafts in index order
   for (int k = 0; k < K; ++k) {
     const int set = p.per_draft ? k : 0;
-    if (tid == 0) {
+    if (warp == 0) {
+      // lane 0: whether the draft is considered; then lane r the ratio
+      // num / den of position tau + r (and + 32), in parallel; then lane 0
+      // the weights w_i in order
       const int tau = sm.tau;
-      int skip = tau == L ? 2 : 0;
-      const int* x = sm.tok + k * L;
-      if (!skip && tau > 0) {
-        const int* xa = sm.tok + sm.a * L;
-        for (int i = 0; i < tau; ++i)
-          if (x[i] != xa[i]) skip = 1;
+      const int* x = s_tok + k * L;
+      int skip = 0;
+      if (lane == 0) {
+        skip = tau == L ? 2 : 0;
+        if (!skip && tau > 0) {
+          const int* xa = s_tok + sm.a * L;
+          for (int i = 0; i < tau; ++i)
+            if (x[i] != xa[i]) skip = 1;
+        }
+        if (!skip)
+          for (int h = 0; h < sm.nH; ++h)
+            if (sm.H[h] == x[tau]) skip = 1;
+        sm.skip = skip;
       }
-      if (!skip)
-        for (int h = 0; h < sm.nH; ++h)
-          if (sm.H[h] == x[tau]) skip = 1;
-      sm.skip = skip;
+      skip = __shfl_sync(0xffffffffu, skip, 0);
       if (!skip) {
         const double keep = 1.0 - sm.qH;
-        sm.keep = keep;
-        const double qfirst = keep > 0.0 ? static_cast<double>(prob_x(qd(set, tau), sm.zg[k * L + tau].y)) / keep : 0.0;
-        // R at the draft's token: read from the CTA that owns that entry
-        const int xt = x[tau], owner = xt / p.slice, eo = xt - owner * p.slice;
-        float rx;
-        if constexpr (kLocal) {
-          const float* Rl = reinterpret_cast<const float*>(dyn + kMdFixed) + sm.rcur * p.slice;
-          rx = cl.map_shared_rank(Rl, owner)[eo];
-        } else {
-          rx = p.Rws[static_cast<size_t>(b) * 2 * V + static_cast<size_t>(sm.rcur) * V + xt];
-          (void)eo;
-        }
-        double w = 1.0;
-        for (int i = tau; i < L; ++i) {
-          double num, den;
-          if (i == tau) {
-            num = static_cast<double>(rx) / sm.Rn;
-            den = qfirst;
-          } else {
-            num = prob_x(qt(set, i), sm.zg[k * L + i].x);
-            den = prob_x(qd(set, i), sm.zg[k * L + i].y);
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+          const int i = tau + lane + 32 * h2;
+          if (i < L) {
+            double num, den;
+            if (i == tau) {
+              // R at the draft's token: read from the CTA that owns that entry
+              const int xt = x[tau], owner = xt / p.slice, eo = xt - owner * p.slice;
+              float rx;
+              if constexpr (kLocal) {
+                const float* Rl = reinterpret_cast<const float*>(dynrest) + sm.rcur * p.slice;
+                rx = cl.map_shared_rank(Rl, owner)[eo];
+              } else {
+                rx = p.Rws[static_cast<size_t>(b) * 2 * V + static_cast<size_t>(sm.rcur) * V + xt];
+                (void)eo;
+              }
+              num = static_cast<double>(rx) / sm.Rn;
+              den = keep > 0.0 ? static_cast<double>(prob_x(qd(set, tau), s_zg[k * L + tau].y)) / keep : 0.0;
+            } else {
+              num = prob_x(qt(set, i), s_zg[k * L + i].x);
+              den = prob_x(qd(set, i), s_zg[k * L + i].y);
+            }
+            sm.num[i] = num;
+            sm.den[i] = den;
           }
-          w = step_weight(w, num, den);
-          sm.w[i] = w;
+        }
+        __syncwarp();
+        if (lane == 0) {
+          sm.keep = keep;
+          double w = 1.0;
+          for (int i = tau; i < L; ++i) {
+            w = step_weight(w, sm.num[i], sm.den[i]);
+            sm.w[i] = w;
+          }
         }
       }
     }
@@ -480,7 +511,7 @@ __global__ void __launch_bounds__(kMdT) md_cluster_kernel(const __grid_constant_
     if (sm.skip == 2) break;
     if (sm.skip) continue;
     const int tau = sm.tau;
-    const int* x = sm.tok + k * L;
+    const int* x = s_tok + k * L;
     // all of the draft's sums A_i, i = tau .. L-2, in one pass (at least one
     // exchange, which also orders the R reads above before any R update)
     const int nA = max(L - 1 - tau, 0);
@@ -502,26 +533,40 @@ __global__ void __launch_bounds__(kMdT) md_cluster_kernel(const __grid_constant_
       exchange(cl, sm, buf, max(nA, 1), loc);
       buf ^= 1;
     }
-    if (tid == 0) {
-      int best = tau;
-      double wbest = 1.0;
-      for (int i = tau; i < L; ++i) {
-        const double w = sm.w[i];
-        double h;
-        if (i < L - 1) {
-          const double A = sm.res[i - tau];
-          const double den = A + 1.0 - w;
-          h = den == 0.0 ? 1.0 : A / den;
-        } else {
-          h = w;
+    if (warp == 0) {
+      // the coins h_i, lane r for position tau + r (and + 32); the accepted
+      // sub-block is the longest one: up to the last position whose coin
+      // came up
+      unsigned acc[2];
+#pragma unroll
+      for (int h2 = 0; h2 < 2; ++h2) {
+        const int i = tau + lane + 32 * h2;
+        bool up = false;
+        if (i < L) {
+          const double w = sm.w[i];
+          double h;
+          if (i < L - 1) {
+            const double A = sm.res[i - tau];
+            const double den = A + 1.0 - w;
+            h = den == 0.0 ? 1.0 : A / den;
+          } else {
+            h = w;
+          }
+          up = static_cast<double>(s_eta[k * L + i]) < h;
         }
-        if (static_cast<double>(sm.eta[k * L + i]) < h) {
-          best = i + 1;
-          wbest = w;
-        }
+        acc[h2] = __ballot_sync(0xffffffffu, up);
       }
-      sm.best = best;
-      sm.wbest = wbest;
+      if (lane == 0) {
+        int best = tau;
+        double wbest = 1.0;
+        const int r = acc[1] ? 63 - __clz(acc[1]) : (acc[0] ? 31 - __clz(acc[0]) : -1);
+        if (r >= 0) {
+          best = tau + r + 1;
+          wbest = sm.w[tau + r];
+        }
+        sm.best = best;
+        sm.wbest = wbest;
+      }
     }
     __syncthreads();
     const int best = sm.best;
@@ -580,7 +625,7 @@ __global__ void __launch_bounds__(kMdT) md_cluster_kernel(const __grid_constant_
           sm.rcur = rc ^ 1;
         }
         sm.H[sm.nH++] = x[tau];
-        sm.qH += static_cast<double>(prob_x(qd(set, tau), sm.zg[k * L + tau].y));
+        sm.qH += static_cast<double>(prob_x(qd(set, tau), s_zg[k * L + tau].y));
       }
     }
     __syncthreads();
@@ -620,7 +665,7 @@ __global__ void __launch_bounds__(kMdT) md_cluster_kernel(const __grid_constant_
     be = 1.0f;
     bi = INT_MAX;
     int fail = 0;
-    for (int q = 0; q < kMdC; ++q) {
+    for (int q = 0; q < kC; ++q) {
       const float4 g = *reinterpret_cast<const float4*>(&sm.xb[buf][q][0]);
       fail |= __float_as_int(g.w);
       if (race_better(g.x, g.y, __float_as_int(g.z), bw, be, bi)) {
@@ -636,7 +681,7 @@ __global__ void __launch_bounds__(kMdT) md_cluster_kernel(const __grid_constant_
       return;
     }
     const int a = sm.a;
-    for (int i = 0; i <= L; ++i) tok[i] = i < tau ? sm.tok[a * L + i] : (i == tau ? bi : -1);
+    for (int i = 0; i <= L; ++i) tok[i] = i < tau ? s_tok[a * L + i] : (i == tau ? bi : -1);
     p.accept_len[b] = tau;
     if (p.out_draft_index) p.out_draft_index[b] = a;
   }
@@ -651,59 +696,101 @@ struct MdShape {
   size_t smem_local;
 };
 
-MdShape md_shape(int rows, int V, int dtype) {
+MdShape md_shape(int rows, int V, int dtype, int C, size_t fixed) {
   const size_t es = dtype == SV_BF16 ? 2 : 4;
   MdShape s{};
-  s.slice = ((V + kMdC - 1) / kMdC + 7) / 8 * 8;
+  s.slice = ((V + C - 1) / C + 7) / 8 * 8;
   s.rowstride = static_cast<int>((static_cast<size_t>(s.slice) * es + 16 + 15) / 16 * 16);
-  s.smem_local = kMdFixed + 2 * static_cast<size_t>(s.slice) * sizeof(float) +
+  s.smem_local = fixed + 2 * static_cast<size_t>(s.slice) * sizeof(float) +
                  static_cast<size_t>(rows) * s.rowstride;
   return s;
 }
 
-// Opt a variant into its dynamic shared memory and check that one cluster
-// of it can be resident (once per device and size); false if it cannot.
-template <typename Kernel>
-bool md_ready(Kernel kernel, size_t smem) {
-  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(smem)) != cudaSuccess) {
-    (void)cudaGetLastError();
-    return false;
-  }
+template <int kC, typename Kernel>
+cudaLaunchConfig_t md_config(Kernel, int B, size_t smem, cudaStream_t stream, cudaLaunchAttribute* attr) {
   cudaLaunchConfig_t cfg{};
-  cfg.gridDim = dim3(kMdC);
-  cfg.blockDim = dim3(kMdT);
-  cfg.dynamicSmemBytes = smem;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = kMdC;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) != cudaSuccess) {
-    (void)cudaGetLastError();
-    return false;
-  }
-  return n > 0;
-}
-
-template <typename Kernel>
-cudaError_t md_launch(Kernel kernel, int B, size_t smem, cudaStream_t stream, const MdcParams& p) {
-  cudaLaunchConfig_t cfg{};
-  cfg.gridDim = dim3(static_cast<unsigned>(B) * kMdC);
+  cfg.gridDim = dim3(static_cast<unsigned>(B) * kC);
   cfg.blockDim = dim3(kMdT);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = kMdC;
+  attr[0].val.clusterDim.x = kC;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kernel, p);
+  return cfg;
+}
+
+// Clusters of a variant that can be resident at once at this shared-memory
+// size (the variant opted into the largest size and, for 16 CTAs, into a
+// non-portable cluster size); 0 if none.
+template <int kC, typename Kernel>
+int md_clusters(Kernel kernel, size_t smem) {
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(kMaxDynSmem)) != cudaSuccess ||
+      (kC > 8 && cudaFuncSetAttribute(kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)) {
+    (void)cudaGetLastError();
+    return 0;
+  }
+  cudaLaunchAttribute attr[1];
+  const cudaLaunchConfig_t cfg = md_config<kC>(kernel, 1, smem, nullptr, attr);
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return 0;
+  }
+  return n;
+}
+
+// md_clusters asked once per device, variant and size (rounded up to 8 KB).
+template <bool kBf16, bool kLocal, int kC>
+int md_capacity(size_t smem) {
+  constexpr size_t kStep = 8 * 1024;
+  constexpr int kClasses = static_cast<int>((kMaxDynSmem + kStep - 1) / kStep) + 1;
+  static std::atomic<int> cap[kClasses][64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  const int cls = static_cast<int>((smem + kStep - 1) / kStep);
+  if (cls >= kClasses) return 0;
+  int v = cap[cls][dev].load(std::memory_order_relaxed);
+  if (v == 0) {
+    const size_t probe = static_cast<size_t>(cls) * kStep < kMaxDynSmem ? static_cast<size_t>(cls) * kStep : kMaxDynSmem;
+    const int n = md_clusters<kC>(md_cluster_kernel<kBf16, kLocal, kC>, probe);
+    v = n > 0 ? n : -1;
+    cap[cls][dev].store(v, std::memory_order_relaxed);
+  }
+  return v > 0 ? v : 0;
+}
+
+// Launch with clusters of kC CTAs: the variant that stages the rows in
+// shared memory when they fit, else the one that reads them from global
+// memory.  With need_wave, only when all B clusters fit in one wave.  Sets
+// `launched`; returns a status.
+template <bool kBf16, int kC>
+int md_try(MdcParams p, int B, int rows, bool need_wave, cudaStream_t stream, bool& launched) {
+  launched = false;
+  const size_t fixed = md_fixed<kC>() + md_token_bytes(p.K, p.L);
+  const MdShape sh = md_shape(rows, p.V, kBf16 ? SV_BF16 : SV_F32, kC, fixed);
+  p.slice = sh.slice;
+  p.rowstride = sh.rowstride;
+  const bool local = sh.smem_local <= kMaxDynSmem && md_capacity<kBf16, true, kC>(sh.smem_local) > 0;
+  const size_t smem = local ? sh.smem_local : fixed;
+  const int cap = local ? md_capacity<kBf16, true, kC>(smem) : md_capacity<kBf16, false, kC>(smem);
+  if (cap <= 0 || (need_wave && B > cap)) return SV_OK;
+  cudaLaunchAttribute attr[1];
+  cudaError_t e;
+  if (local) {
+    const cudaLaunchConfig_t cfg = md_config<kC>(md_cluster_kernel<kBf16, true, kC>, B, smem, stream, attr);
+    e = cudaLaunchKernelEx(&cfg, md_cluster_kernel<kBf16, true, kC>, p);
+  } else {
+    const cudaLaunchConfig_t cfg = md_config<kC>(md_cluster_kernel<kBf16, false, kC>, B, smem, stream, attr);
+    e = cudaLaunchKernelEx(&cfg, md_cluster_kernel<kBf16, false, kC>, p);
+  }
+  if (e != cudaSuccess)
+    return set_error(SV_ERR_CUDA, "multi-draft kernel launch failed: %s", cudaGetErrorString(e));
+  launched = true;
+  return SV_OK;
 }
 }  // namespace
 
@@ -724,7 +811,6 @@ int launch_multi(const void* target, const void* draft, const int32_t* tokens,
     return set_error(SV_ERR_UNSUPPORTED,
                      "per-draft rows: K (2L + 1) = %d row statistics per sequence, more than %d",
                      nsets * (2 * L + 1), kMaxStatRows);
-  const MdShape sh = md_shape(nsets * (2 * L + 1), V, dtype);
   MdcParams p{};
   p.target = target;
   p.draft = draft;
@@ -737,48 +823,24 @@ int launch_multi(const void* target, const void* draft, const int32_t* tokens,
   p.per_draft = per_draft ? 1 : 0;
   p.seed = seed;
   p.step = static_cast<uint32_t>(step);
-  p.slice = sh.slice;
-  p.rowstride = sh.rowstride;
   p.Rws = reinterpret_cast<float*>(ws + lay.resid);
   p.accept_len = out_accept_len;
   p.out_tokens = out_tokens;
   p.out_draft_index = out_draft_index;
-  if (static_cast<long long>(B) * kMdC > INT_MAX)
+  if (static_cast<long long>(B) * 16 > INT_MAX)
     return set_error(SV_ERR_INVALID_ARG, "B too large for one launch");
+  // Clusters of 16 CTAs when all B of them fit in one wave (each CTA then
+  // stages and sweeps half as many entries), else of 8.
+  const int rows = nsets * (2 * L + 1);
   const bool bf16 = dtype == SV_BF16;
-  // Once per device: each variant opted into its largest shared memory, and
-  // one cluster of it found residentable (1), or not (2).
-  static std::atomic<int> ready[2][2][64];
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
-    return set_error(SV_ERR_CUDA, "no current CUDA device");
-  auto prepared = [&](bool local) {
-    std::atomic<int>& slot = ready[bf16 ? 1 : 0][local ? 1 : 0][dev];
-    int v = slot.load(std::memory_order_relaxed);
-    if (v == 0) {
-      const size_t smem = local ? kMaxDynSmem : kMdFixed;
-      bool ok;
-      if (local)
-        ok = bf16 ? md_ready(md_cluster_kernel<true, true>, smem) : md_ready(md_cluster_kernel<false, true>, smem);
-      else
-        ok = bf16 ? md_ready(md_cluster_kernel<true, false>, smem) : md_ready(md_cluster_kernel<false, false>, smem);
-      v = ok ? 1 : 2;
-      slot.store(v, std::memory_order_relaxed);
-    }
-    return v == 1;
-  };
-  const bool use_local = sh.smem_local <= kMaxDynSmem && prepared(true);
-  if (!use_local && !prepared(false))
-    return set_error(SV_ERR_CUDA, "multi-draft cluster kernel cannot be made resident");
-  cudaError_t e;
-  if (use_local)
-    e = bf16 ? md_launch(md_cluster_kernel<true, true>, B, sh.smem_local, stream, p)
-             : md_launch(md_cluster_kernel<false, true>, B, sh.smem_local, stream, p);
-  else
-    e = bf16 ? md_launch(md_cluster_kernel<true, false>, B, kMdFixed, stream, p)
-             : md_launch(md_cluster_kernel<false, false>, B, kMdFixed, stream, p);
-  if (e != cudaSuccess)
-    return set_error(SV_ERR_CUDA, "multi-draft kernel launch failed: %s", cudaGetErrorString(e));
+  bool launched = false;
+  int st = bf16 ? md_try<true, 16>(p, B, rows, true, stream, launched)
+                : md_try<false, 16>(p, B, rows, true, stream, launched);
+  if (st == SV_OK && !launched)
+    st = bf16 ? md_try<true, 8>(p, B, rows, false, stream, launched)
+              : md_try<false, 8>(p, B, rows, false, stream, launched);
+  if (st != SV_OK) return st;
+  if (!launched) return set_error(SV_ERR_CUDA, "multi-draft cluster kernel cannot be made resident");
   return check_launch("multidraft");
 }
 
