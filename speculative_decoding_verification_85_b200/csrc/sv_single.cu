@@ -48,7 +48,8 @@ struct SingleParams {
   int nc2;              // draw CTAs per sequence
   int gpc;              // race groups per draw CTA
   int nseg;             // row segments per row
-  int segvec;           // 16-byte vectors per row segment (multiple of kTileVec)
+  int tiles;            // kTileVec-vector tiles covering a row's body; segment s
+                        // covers tiles [s tiles / nseg, (s + 1) tiles / nseg)
   float4* pairpart;     // [B][gamma + 1][nseg] x {target, draft} partials
   float* zx;            // [B][gamma][nseg][2] draft token's target / draft logit
 };
@@ -246,8 +247,9 @@ __global__ void __launch_bounds__(kRowThreads, 3) rows_kernel(const __grid_const
   const char* rpA = target_row<kBf16>(p, b, i);
   const char* rpB = loadB ? draft_row<kBf16>(p, b, i) : rpA;
   const RowGeom<kBf16> gA(rpA, p.V), gB(rpB, p.V);
-  const int k0 = seg * f.segvec;
-  const int a1 = min(gA.nvec, k0 + f.segvec), b1 = min(gB.nvec, k0 + f.segvec);
+  const int k0 = static_cast<int>(static_cast<long long>(seg) * f.tiles / f.nseg) * kTileVec;
+  const int kseg1 = static_cast<int>(static_cast<long long>(seg + 1) * f.tiles / f.nseg) * kTileVec;
+  const int a1 = min(gA.nvec, kseg1), b1 = min(gB.nvec, kseg1);
   const uint4* vA = gA.body(rpA);
   const uint4* vB = gB.body(rpB);
   const int ownA = owned_vector<kBf16>(gA, xg, k0, a1);
@@ -766,9 +768,8 @@ int launch_single(const void* target, const void* draft, const int32_t* tokens,
     st = st < 1 ? 1 : (st > kMaxSegTiles ? kMaxSegTiles : st);
     int nseg = static_cast<int>((tiles + st - 1) / st);
     if (nseg > lay.nc) nseg = lay.nc;
-    st = (tiles + nseg - 1) / nseg;
     f.nseg = nseg;
-    f.segvec = static_cast<int>(st) * kTileVec;
+    f.tiles = tiles;
   }
   f.pairpart = reinterpret_cast<float4*>(ws + lay.part1);
   f.zx = reinterpret_cast<float*>(ws + lay.resid);
