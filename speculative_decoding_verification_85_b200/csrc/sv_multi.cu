@@ -158,12 +158,11 @@ __global__ void __launch_bounds__(kMdT) md_cluster_kernel(const __grid_constant_
   const int nsets = p.per_draft ? K : 1;
   const int v0 = rank * p.slice;
   const int n = max(0, min(V - v0, p.slice));  // entries of this slice
-  const float T = __ldg(p.temps + b);
-  const bool tvalid = (T >= 0.0f) && !isinf(T);
-  const bool greedy = tvalid && T == 0.0f;
-  // the rows a sequence needs, numbered q = set * nrows + r: per row set the
-  // target rows 0..L, then (softmax rows only) the draft rows 0..L-1 as r = L+1..2L
-  const int nrows = greedy ? L + 1 : rps;
+  // the rows, numbered q = set * rps + r: per row set the target rows 0..L,
+  // then the draft rows 0..L-1 as r = L+1..2L.  All of them are staged at
+  // once, before the temperature is known; a greedy sequence reads only its
+  // target rows.
+  const int nrows = rps;
   const int nq = nsets * nrows;
   const size_t rowb = static_cast<size_t>(V) * es;
   const char* tgt = static_cast<const char*>(p.target) + static_cast<size_t>(b) * nsets * (L + 1) * rowb;
@@ -215,7 +214,7 @@ __global__ void __launch_bounds__(kMdT) md_cluster_kernel(const __grid_constant_
   // tokens, their logits and the sub-block acceptance uniforms while the
   // rows are in flight
   if (tid == 0) {
-    if (kLocal && tvalid)
+    if (kLocal)
       for (int q = 0; q < nq; ++q) mbar_init(&sm.rbar[q], 1);
     mbar_init(&sm.xbar[0], 1);
     mbar_init(&sm.xbar[1], 1);
@@ -225,9 +224,18 @@ __global__ void __launch_bounds__(kMdT) md_cluster_kernel(const __grid_constant_
   }
   __syncthreads();  // the barriers are initialised before any thread waits on them
   bool scalar_copies = false;
-  if constexpr (kLocal) {
-    if (tvalid) scalar_copies = stage_rows_issue<es, kMdT>(grow, nq, v0, n, srows, p.rowstride, sm.rbar);
-  }
+  if constexpr (kLocal) scalar_copies = stage_rows_issue<es, kMdT>(grow, nq, v0, n, srows, p.rowstride, sm.rbar);
+  const float T = __ldg(p.temps + b);
+  const bool tvalid = (T >= 0.0f) && !isinf(T);
+  const bool greedy = tvalid && T == 0.0f;
+  auto needed = [&](int q) { return !greedy || q % rps <= L; };  // rows the sequence reads
+  // every staged row has landed before the CTA leaves (rows a greedy sequence
+  // never read included)
+  auto drain = [&]() {
+    if constexpr (kLocal)
+      if (tid == 0)
+        for (int q = 0; q < nq; ++q) (void)mbar_wait(&sm.rbar[q], 0);
+  };
   // every CTA's barriers are initialised before any remote store: arrive
   // now, wait just before the first exchange
   asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
@@ -266,7 +274,11 @@ __global__ void __launch_bounds__(kMdT) md_cluster_kernel(const __grid_constant_
     float4* part = sm.part;  // [nq] this slice's row statistics
     for (int q = warp; q < nq; q += kMdW) {
       bool landed = true;
-      if constexpr (kLocal) landed = !tvalid || mbar_wait(&sm.rbar[q], 0);
+      if constexpr (kLocal) landed = mbar_wait(&sm.rbar[q], 0);
+      if (!needed(q)) {
+        if (lane == 0) part[q] = make_float4(-INFINITY, 0.0f, __int_as_float(0x7fffffff), __int_as_float(0));
+        continue;
+      }
       const char* gq = grow(q) + static_cast<size_t>(v0) * es;
       const char* rp = kLocal ? srows + static_cast<size_t>(q) * p.rowstride + (reinterpret_cast<uintptr_t>(gq) & 15u) : gq;
       float m = -INFINITY, sum = 0.0f;
@@ -337,7 +349,7 @@ __global__ void __launch_bounds__(kMdT) md_cluster_kernel(const __grid_constant_
         sm.arg[q] = a.arg;
         bool rv = !a.bad && isfinite(a.m);
         if (!greedy) rv = rv && isfinite(__fdiv_rn(a.m, T));
-        row_ok = row_ok && rv;
+        if (needed(q)) row_ok = row_ok && rv;
       }
       __syncthreads();  // every thread has read the buffer
       if (tid == 0) sm.xphase[buf] ^= 1u;
@@ -373,6 +385,7 @@ __global__ void __launch_bounds__(kMdT) md_cluster_kernel(const __grid_constant_
         if (p.out_draft_index) p.out_draft_index[b] = -1;
       }
     }
+    drain();
     cl.sync();  // every CTA returns here, after every remote store has landed
     return;
   }
@@ -398,6 +411,7 @@ __global__ void __launch_bounds__(kMdT) md_cluster_kernel(const __grid_constant_
       p.accept_len[b] = tau;
       if (p.out_draft_index) p.out_draft_index[b] = a;
     }
+    drain();
     cl.sync();
     return;
   }
@@ -659,6 +673,7 @@ __global__ void __launch_bounds__(kMdT) md_cluster_kernel(const __grid_constant_
   if (tid == 0)
     *reinterpret_cast<float4*>(cl.map_shared_rank(&sm.xb[buf][rank][0], 0)) =
         make_float4(bw, be, __int_as_float(bi), __int_as_float(sm.xfail));
+  drain();
   cl.sync();
   if (rank == 0 && tid == 0) {
     bw = 0.0f;

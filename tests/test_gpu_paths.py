@@ -83,3 +83,25 @@ def test_the_two_paths_agree_on_the_same_sequences():
             assert np.array_equal(few["tokens"][b], big["tokens"][b])
         np.testing.assert_allclose(few["lp"], big["lp"][:small], rtol=0, atol=2e-5)
     led.check()
+
+
+@pytest.mark.parametrize("B,K,L,V,T,csize", [
+    (2, 3, 4, 32000, [0.4, 1.0], 16),
+    (24, 3, 4, 32000, [0.0, 0.4, 1.0], 8),
+])
+def test_multidraft_cluster_sizes(B, K, L, V, T, csize):
+    """Multi-draft: 16-CTA clusters when the batch's clusters fit one wave,
+    else 8; both against the oracle."""
+    st = workloads.make_custom(B, L, V, dtype="bf16", seed=B * 7 + K, T=T, K=K, device=DEV)
+    led = TieLedger(f"multi-draft {csize}-CTA clusters B={B} K={K} L={L}")
+    for step in range(2):
+        with profile(activities=[ProfilerActivity.CUDA]) as prof:
+            acc, tok, di = sv.spec_verify_multidraft(st.target, st.draft, st.tokens, st.temps,
+                                                     seed=3, step=step)
+            torch.cuda.synchronize()
+        names = [e.name for e in prof.events() if "md_cluster_kernel" in e.name]
+        assert names and all(n.split("(")[0].rstrip(">").endswith(f" {csize}") for n in names), names
+        gpu = {"accept_len": acc.cpu().numpy(), "tokens": tok.cpu().numpy(),
+               "draft_index": di.cpu().numpy()}
+        led.add(compare(gpu, run_oracle(st, 3, step), check_logprobs=False))
+    led.check()
