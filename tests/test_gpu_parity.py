@@ -34,6 +34,15 @@ def gpu_multi(st, seed=0, step=0, ws=None):
             "draft_index": idx.cpu().numpy()}
 
 
+def widen(st, min_b=80):
+    """The batch tiled to at least min_b sequences: more clusters than one wave
+    holds, so the row and draw kernels take it (small batches of narrow rows
+    take the one-cluster-per-sequence kernel)."""
+    r = -(-min_b // st.target.shape[0])
+    cat = lambda x: torch.cat([x] * r, dim=0).contiguous()  # noqa: E731
+    return workloads.Step(cat(st.target), cat(st.draft), cat(st.tokens), cat(st.temps), st.step)
+
+
 SMALL = [
     # B, gamma, V, dtype, temperatures
     (1, 4, 32000, "f32", 1.0),
@@ -50,11 +59,16 @@ SMALL = [
 ]
 
 
+@pytest.mark.parametrize("wide", [False, True])
 @pytest.mark.parametrize("B,gamma,V,dtype,T", SMALL)
-def test_small_shapes(B, gamma, V, dtype, T):
+def test_small_shapes(B, gamma, V, dtype, T, wide):
+    if wide and V > 10000:
+        pytest.skip("the wide copies of the long rows only repeat the larger tests")
     for seed in (0, 123):
         st = workloads.make_custom(B, gamma, V, dtype=dtype, seed=seed + V, T=T, device=DEV,
                                    target_scale=2.5, noise=0.8)
+        if wide:
+            st = widen(st)
         for step in (0, 7):
             g = gpu_single(st, seed=seed, step=step)
             o = run_oracle(st, seed, step)
@@ -112,7 +126,8 @@ def test_multidraft_small(B, K, L, V, dtype, T):
         compare(g, run_oracle(st, seed, 3))
 
 
-def test_invalid_sequences():
+@pytest.mark.parametrize("wide", [False, True])
+def test_invalid_sequences(wide):
     st = workloads.make_custom(8, 4, 300, dtype="bf16", seed=5, T=1.0, device=DEV)
     st.temps[0] = -1.0
     st.temps[1] = float("nan")
@@ -121,29 +136,39 @@ def test_invalid_sequences():
     st.tokens[4, 0] = -5
     st.target[5, 2, 17] = float("nan")
     st.draft[6, 1, :] = float("-inf")
+    if wide:
+        st = widen(st)
     g = gpu_single(st)
     o = run_oracle(st, 0, 0)
     compare(g, o)
-    for b in range(7):
-        assert g["accept_len"][b] == -1 and np.all(g["tokens"][b] == -1)
-    assert g["accept_len"][7] >= 0
+    for b in range(st.target.shape[0]):
+        if b % 8 < 7:
+            assert g["accept_len"][b] == -1 and np.all(g["tokens"][b] == -1)
+        else:
+            assert g["accept_len"][b] >= 0
 
 
-def test_inf_entries_and_plus_inf():
+@pytest.mark.parametrize("wide", [False, True])
+def test_inf_entries_and_plus_inf(wide):
     st = workloads.make_custom(6, 3, 500, dtype="f32", seed=9, T=[1.0, 0.0], device=DEV)
     st.target[0, :, ::3] = float("-inf")  # probability-zero entries
     st.draft[1, :, ::5] = float("-inf")
     st.target[2, 1, 10] = float("inf")     # invalid row
     st.target[3, 0, 4] = float("inf")      # invalid greedy row
+    if wide:
+        st = widen(st)
     g = gpu_single(st)
     compare(g, run_oracle(st, 0, 0))
     assert g["accept_len"][2] == -1 and g["accept_len"][3] == -1
 
 
-def test_unaligned_rows_and_offsets():
+@pytest.mark.parametrize("wide", [False, True])
+def test_unaligned_rows_and_offsets(wide):
     """Rows whose start is not 16-byte aligned (odd V, sliced base pointers)."""
     for V in (31, 1001, 8193):
         st = workloads.make_custom(5, 3, V, dtype="bf16", seed=V, T=[0.7, 1.0, 0.0], device=DEV)
+        if wide:
+            st = widen(st)
         big_t = torch.empty(st.target.numel() + 3, dtype=st.target.dtype, device=DEV)
         big_d = torch.empty(st.draft.numel() + 5, dtype=st.draft.dtype, device=DEV)
         t = big_t[3:].view(st.target.shape)
