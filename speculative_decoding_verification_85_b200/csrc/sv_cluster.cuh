@@ -49,57 +49,10 @@ __device__ __forceinline__ bool xbar_wait(uint64_t* bar, uint32_t parity) {
 // Stage the slice [v0, v0 + n) of nq rows (row q starts at grow(q) in global
 // memory) into shared memory: row q's slice goes to srows + q rowstride +
 // (its global address mod 16), so the aligned body of each row slice is one
-// bulk copy (completing on `bar`, an initialised mbarrier at phase 0) and
-// the unaligned head and tail are copied as scalars.  Called by all
-// kThreads threads; returns false if the bulk copies did not complete in
-// time (the bounded mbarrier wait).  Nothing outside the slice is read.
-template <size_t es, int kThreads, typename RowFn>
-__device__ __forceinline__ bool stage_slices(RowFn grow, int nq, int v0, int n, char* srows, int rowstride,
-                                             uint64_t* bar) {
-  const int tid = threadIdx.x;
-  auto geom = [&](int q, const char*& g, uint32_t& hb, uint32_t& body) {
-    g = grow(q) + static_cast<size_t>(v0) * es;
-    const uintptr_t ga = reinterpret_cast<uintptr_t>(g);
-    hb = min(static_cast<uint32_t>((16u - (ga & 15u)) & 15u), static_cast<uint32_t>(n * es));
-    body = (static_cast<uint32_t>(n * es) - hb) / 16u * 16u;
-  };
-  if (tid == 0) {
-    uint32_t total = 0;
-    for (int q = 0; q < nq; ++q) {
-      const char* g;
-      uint32_t hb, body;
-      geom(q, g, hb, body);
-      total += body;
-    }
-    if (total) {
-      mbar_arrive_expect_tx(bar, total);
-      for (int q = 0; q < nq; ++q) {
-        const char* g;
-        uint32_t hb, body;
-        geom(q, g, hb, body);
-        char* sdst = srows + static_cast<size_t>(q) * rowstride + (reinterpret_cast<uintptr_t>(g) & 15u);
-        if (body) bulk_g2s(sdst + hb, g + hb, body, bar);
-      }
-    } else {
-      mbar_arrive(bar);
-    }
-  }
-  for (int q = 0; q < nq; ++q) {
-    const char* g;
-    uint32_t hb, body;
-    geom(q, g, hb, body);
-    char* sdst = srows + static_cast<size_t>(q) * rowstride + (reinterpret_cast<uintptr_t>(g) & 15u);
-    const int h = static_cast<int>(hb / es), t0 = static_cast<int>((hb + body) / es);
-    for (int e = tid; e < h; e += kThreads) memcpy(sdst + e * es, g + e * es, es);
-    for (int e = t0 + tid; e < n; e += kThreads) memcpy(sdst + e * es, g + e * es, es);
-  }
-  return mbar_wait(bar, 0);
-}
-
-
-// The same staging with one barrier per row (bars[q], initialised, phase
-// 0), issued without waiting: thread 0 issues the bulk copies in row order
-// and all kThreads threads copy the unaligned heads and tails.  Returns
+// bulk copy, completing on its own barrier bars[q] (initialised, phase 0,
+// and ordered before this call by a CTA barrier); issued without waiting:
+// thread q issues row q's bulk copy and all kThreads threads copy the
+// unaligned heads and tails.  Returns
 // whether there were any (the same answer in every thread); if so, a CTA
 // barrier must order those scalar copies before use.  A thread may use row q
 // once mbar_wait(&bars[q], 0) returns true, so a row is processed while
@@ -108,23 +61,36 @@ template <size_t es, int kThreads, typename RowFn>
 __device__ __forceinline__ bool stage_rows_issue(RowFn grow, int nq, int v0, int n, char* srows,
                                                  int rowstride, uint64_t* bars) {
   const int tid = threadIdx.x;
+  auto geom = [&](int q, const char*& g, uint32_t& hb, uint32_t& body, char*& sdst) {
+    g = grow(q) + static_cast<size_t>(v0) * es;
+    const uintptr_t ga = reinterpret_cast<uintptr_t>(g);
+    hb = min(static_cast<uint32_t>((16u - (ga & 15u)) & 15u), static_cast<uint32_t>(n * es));
+    body = (static_cast<uint32_t>(n * es) - hb) / 16u * 16u;
+    sdst = srows + static_cast<size_t>(q) * rowstride + (ga & 15u);
+  };
+  // the bulk copies, thread q issuing row q's (one instruction per warp)
+  for (int q = tid; q < nq; q += kThreads) {
+    const char* g;
+    uint32_t hb, body;
+    char* sdst;
+    geom(q, g, hb, body, sdst);
+    if (body) {
+      mbar_arrive_expect_tx(&bars[q], body);
+      bulk_g2s(sdst + hb, g + hb, body, &bars[q]);
+    } else {
+      mbar_arrive(&bars[q]);
+    }
+  }
+  // the unaligned heads and tails, by all threads
   bool scalar = false;  // some row slice has an unaligned head or tail
   for (int q = 0; q < nq; ++q) {
-    const char* g = grow(q) + static_cast<size_t>(v0) * es;
-    const uintptr_t ga = reinterpret_cast<uintptr_t>(g);
-    const uint32_t hb = min(static_cast<uint32_t>((16u - (ga & 15u)) & 15u), static_cast<uint32_t>(n * es));
-    const uint32_t body = (static_cast<uint32_t>(n * es) - hb) / 16u * 16u;
-    char* sdst = srows + static_cast<size_t>(q) * rowstride + (ga & 15u);
-    if (tid == 0) {
-      if (body) {
-        mbar_arrive_expect_tx(&bars[q], body);
-        bulk_g2s(sdst + hb, g + hb, body, &bars[q]);
-      } else {
-        mbar_arrive(&bars[q]);
-      }
-    }
+    const char* g;
+    uint32_t hb, body;
+    char* sdst;
+    geom(q, g, hb, body, sdst);
     const int h = static_cast<int>(hb / es), t0 = static_cast<int>((hb + body) / es);
-    scalar = scalar || h > 0 || t0 < n;
+    if (h == 0 && t0 >= n) continue;
+    scalar = true;
     for (int e = tid; e < h; e += kThreads) memcpy(sdst + e * es, g + e * es, es);
     for (int e = t0 + tid; e < n; e += kThreads) memcpy(sdst + e * es, g + e * es, es);
   }
