@@ -22,12 +22,13 @@ __device__ __forceinline__ double accept_prob(double lp, double lq) {
 // T is sequence b's temperature, x[0..gamma) its draft tokens (in shared
 // memory), rows[] its merged row statistics (target rows 0..gamma, then the
 // draft rows), zsel[2i], zsel[2i + 1] the draft token's target / draft logit
-// (or NULL: read from the rows in global memory).  Lane 0 writes the hand-off
-// record for the draw to *dst (global or shared memory).
+// (or NULL: read from the rows in global memory), upre[i] the acceptance
+// uniform of position i if already drawn (or NULL: drawn here).  Lane 0
+// writes the hand-off record for the draw to *dst (global or shared memory).
 template <bool kBf16>
 __device__ __noinline__ void decide_single(const CallParams& p, int b, float T, const int* x,
                                            const RowAcc* rows, const float* zsel, SeqInfo* dst,
-                                           bool outputs) {
+                                           bool outputs, const float* upre) {
   const int lane = threadIdx.x & 31;
   const int g = p.gamma;
   const bool tvalid = (T >= 0.0f) && !isinf(T);
@@ -104,8 +105,8 @@ __device__ __noinline__ void decide_single(const CallParams& p, int b, float T, 
         const float dq = __fsub_rn(__fdiv_rn(zq, T), __fdiv_rn(aq.m, T));
         const double lp = static_cast<double>(dp) - log(static_cast<double>(ap.s));
         const double lq = static_cast<double>(dq) - log(static_cast<double>(aq.s));
-        const uint4 rnd = keyed_block(p.seed, p.step, kTagAccept, b, 0, i, i);
-        const double u = accept_uniform(rnd.x);
+        const double u = upre ? static_cast<double>(upre[i])
+                              : accept_uniform(keyed_block(p.seed, p.step, kTagAccept, b, 0, i, i).x);
         reject = !(u < accept_prob(lp, lq));
         if (outputs && p.out_lp) p.out_lp[static_cast<size_t>(b) * g + i] = static_cast<float>(lp);
         if (outputs && p.out_lq) p.out_lq[static_cast<size_t>(b) * g + i] = static_cast<float>(lq);

@@ -308,7 +308,7 @@ __global__ void __launch_bounds__(kRowThreads, 3) rows_kernel(const __grid_const
   if (!s_last) return;
   combine_pairs(f, b, argmaxA, c, rows, s_zsel);
   if (tid < 32) {
-    decide_single<kBf16>(p, b, T, s_tok, rows, s_zsel, p.info + b, true);
+    decide_single<kBf16>(p, b, T, s_tok, rows, s_zsel, p.info + b, true, nullptr);
     // publish the decision: every lane's writes, then the flag (release)
     __threadfence();
     __syncwarp();

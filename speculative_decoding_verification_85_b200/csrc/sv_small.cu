@@ -40,6 +40,10 @@ constexpr int kSdW = kSdT / 32;
 constexpr int kSdBatch = 32; // row statistics per exchange
 static_assert(SV_MAX_GAMMA <= kSdT, "one thread per draft token");
 constexpr int kSdMaxUnits = 64;               // level-1 work units (group parts) per slice
+// Measured on a B200 (graph-replayed steps): for slices of up to 4096
+// entries the cluster kernel is 6-11% faster than the row and draw kernels
+// at B <= 8 and level at B = 16; for wider slices (V = 65536) it is slower.
+constexpr int kSdMaxSlice = 4 * kRaceGroup;
 
 struct SdParams {
   CallParams p;
@@ -53,6 +57,8 @@ struct alignas(16) SdSmem {
   float4 part[kMaxRowsPerSeq];       // this slice's row statistics
   RowAcc rows[kMaxRowsPerSeq];       // merged row statistics (target rows, then draft rows)
   float gpart[kSdMaxUnits];          // race-group partial sums (level 1)
+  float uacc[SV_MAX_GAMMA];          // acceptance uniforms ((x >> 8) 2^-24, exact in fp32)
+  float gE[(SV_MAX_GAMMA + 1) * (kSdMaxSlice / kRaceGroup)];  // group exponentials [j][local group]
   float zsel[2 * SV_MAX_GAMMA];      // the draft tokens' target / draft logits
   int tok[SV_MAX_GAMMA];             // the draft tokens
   float4 race[kSdW];
@@ -156,6 +162,19 @@ __global__ void __launch_bounds__(kSdT) sd_cluster_kernel(const __grid_constant_
     else
       return reinterpret_cast<const float*>(rp)[e];
   };
+  // the data-independent Philox words, while the rows are in flight (threads
+  // 384..447, warps that hold a row only when there are more than 12):
+  // every position's acceptance uniform, every (position, group) exponential
+  // of this slice's race groups
+  {
+    const int t = tid - 384;
+    const int g0 = v0 / kRaceGroup, nlg = (n + kRaceGroup - 1) / kRaceGroup;
+    if (t >= 0 && t < 64) {
+      if (t < g) sm.uacc[t] = static_cast<float>(accept_uniform(sd_block(p, b, kTagAccept, t, t).x));
+      for (int u = t; u < (g + 1) * nlg; u += 64)
+        sm.gE[u] = exponential_from_bits(sd_block(p, b, kTagGroup, u / nlg, g0 + u % nlg).x);
+    }
+  }
   float zp = __int_as_float(0x7fc00000), zq = zp;
   if (ti < g && tvalid && !greedy && xi >= 0 && xi < V) {
     zp = logit_at<kBf16>(grow(ti), xi);
@@ -246,7 +265,7 @@ __global__ void __launch_bounds__(kSdT) sd_cluster_kernel(const __grid_constant_
     sm.zsel[2 * ti + 1] = zq;
   }
   __syncthreads();
-  if (warp == 0) decide_single<kBf16>(p, b, T, sm.tok, sm.rows, sm.zsel, &sm.si, rank == 0);
+  if (warp == 0) decide_single<kBf16>(p, b, T, sm.tok, sm.rows, sm.zsel, &sm.si, rank == 0, sm.uacc);
   __syncthreads();
   const SeqInfo si = sm.si;
   const bool draw = (si.mode == kModeResidual && si.j >= 0 && si.j < g) ||
@@ -295,7 +314,7 @@ __global__ void __launch_bounds__(kSdT) sd_cluster_kernel(const __grid_constant_
         float s = 0.0f;
         for (int k = 0; k < wpg; ++k) s += sm.gpart[tid * wpg + k];
         const int gid = g0 + tid;
-        const float e = exponential_from_bits(sd_block(p, b, kTagGroup, j, gid).x);
+        const float e = sm.gE[j * nlg + tid];  // drawn in the prologue
         if (race_better(s, e, gid, bw, be, bg)) {
           bw = s;
           be = e;
@@ -415,11 +434,6 @@ int sd_capacity(bool bf16, size_t smem) {
   return v > 0 ? v : 0;
 }
 }  // namespace
-
-// Measured on a B200 (graph-replayed steps): for slices of up to 4096
-// entries the cluster kernel is 6-11% faster than the row and draw kernels
-// at B <= 8 and level at B = 16; for wider slices (V = 65536) it is slower.
-constexpr int kSdMaxSlice = 4 * kRaceGroup;
 
 bool small_path(int B, int gamma, int V, int dtype) {
   const SdShape sh = sd_shape(gamma, V, dtype);
