@@ -24,12 +24,16 @@
  *   - Randomness: Philox4x32-10 (Salmon et al., SC'11) with key
  *     (lo32(seed), hi32(seed)) and counter (c0, b, lo32(step), tag<<24 | k<<12
  *     | pos).  Acceptance uniform of position i: tag 1, c0 = i, word 0,
- *     u = (x >> 8) * 2^-24.  Correction/bonus Gumbel noise for vocabulary
- *     entry v at position j: tag 2, c0 = v >> 2, word v & 3,
- *     U = (2 (x >> 9) + 1) * 2^-24, G = -ln(-ln U).  Multi-draft uses tag 3
- *     (k = draft index, pos = i) for its acceptance uniforms and tag 4 for its
- *     Gumbel noise.  Every step therefore replays bit-exactly from
- *     (inputs, seed, step).
+ *     u = (x >> 8) * 2^-24.  The single-draft correction/bonus token at
+ *     position j is drawn by a two-level exponential race over the weights
+ *     w_v (max(p_j - q_j, 0), or p_gamma): vocabulary groups of 1024 entries
+ *     race with their summed weights, group g with the exponential
+ *     E = -ln U of tag 7, c0 = g, word 0; within the winning group entry v
+ *     races with tag 2, c0 = v >> 2, word v & 3; U = (2 (x >> 9) + 1) 2^-24
+ *     in both; the largest w / E wins (lowest index on ties).  Multi-draft
+ *     uses tag 3 (k = draft index, pos = i) for its acceptance uniforms and
+ *     the per-entry race with tag 4 for its correction token.  Every step
+ *     therefore replays bit-exactly from (inputs, seed, step).
  *   - Asynchronous: every entry point enqueues work on `stream` (a
  *     cudaStream_t; NULL is the legacy default stream) and returns without
  *     synchronising.  Results are valid once the stream has reached that
@@ -51,7 +55,8 @@
  *     that live in device data (temps[b] negative, NaN or infinite; a draft
  *     token outside [0, V); a logit row whose maximum is NaN, +inf, or -inf)
  *     mark only that sequence: accept_len[b] = -1 and all its tokens -1.  The
- *     kernels never trap and never spin.
+ *     kernels never trap; every wait on another CTA is bounded in time (two
+ *     seconds), and a wait that runs out marks its sequence the same way.
  */
 #ifndef SPEC_VERIFY_H
 #define SPEC_VERIFY_H
