@@ -329,13 +329,22 @@ def run_ours(args, cfg):
         for i in range(W):
             one(i)
     stream.synchronize()
+    # which of this library's kernels one step launches (profiler records of
+    # one more eager step): counted for gpu_launches, named in the roofline
+    from torch.profiler import ProfilerActivity, profile
+    with profile(activities=[ProfilerActivity.CUDA]) as prof:
+        with torch.cuda.stream(stream):
+            one(W)
+        stream.synchronize()
+    step_kernels = [e.name.split("(")[0].split("<")[0].replace("void ", "").replace("sv::", "")
+                    for e in prof.events()
+                    if e.device_type == torch.autograd.DeviceType.CUDA and "sv::" in e.name]
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph, stream=stream):
         for i in range(W, W + K):
             one(i)
-    # kernels of this library per step: two for single-draft (the row kernel,
-    # then the draw kernel), one for multi-draft (the cluster kernel)
-    launches_per_replay = K * (1 if cfg.multidraft else 2)
+    # kernels of this library per step, as recorded above
+    launches_per_replay = K * len(step_kernels)
     with torch.cuda.stream(stream):
         graph.replay()  # warm the graph itself
     stream.synchronize()
@@ -479,9 +488,9 @@ def run_ours(args, cfg):
                        "launch": "K steps captured in one CUDA graph, replayed",
                        "parallelism": f"batch-sharded replicas x{world}"},
             "roofline": {"bound": "hbm",
-                         "kernel": ("md_cluster_kernel (one launch per step)"
-                                    if cfg.multidraft else
-                                    "rows_kernel + draw_kernel (the whole step)"),
+                         "kernel": " + ".join(dict.fromkeys(step_kernels)) + (
+                             " (the whole step)" if len(step_kernels) > 1 else
+                             " (one launch per step)"),
                          "achieved": algo_gbs, "peak": peak, "unit": "GB/s",
                          "frac": algo_gbs / peak, "traffic": traffic,
                          "peak_source": (f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)"
