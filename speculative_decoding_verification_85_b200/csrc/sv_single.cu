@@ -1,9 +1,12 @@
 // sv_single.cu -- single-draft verification: a row kernel and a draw
-// kernel per call, chained by programmatic dependent launch.
+// kernel per call, chained by programmatic dependent launch (small batches of
+// narrow rows take the one-cluster-per-sequence kernel of sv_small.cu
+// instead; launch_single chooses).
 //
 // Row kernel (FlashSpec, Methodology s.1): one CTA per (sequence, position,
 // vocabulary segment) streams the target row and the draft row of that
-// position over the segment with 16-byte loads issued up front, reduces the
+// position over the segment with 16-byte loads issued up front (and each
+// row's next tile requested into L2 by a bulk prefetch), reduces the
 // maximum and the temperature-scaled softmax sum of both rows, picks up the
 // draft token's two logits, and publishes one partial.  The CTA that
 // completes a sequence (arrival ticket) combines its partials and makes the

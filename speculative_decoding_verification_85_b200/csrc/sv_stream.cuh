@@ -1,6 +1,6 @@
-// sv_stream.cuh -- per-thread row reductions of the single-draft row items.
+// sv_stream.cuh -- per-thread row reductions of the single-draft row kernel.
 //
-// A row item covers (sequence b, position i, vocabulary segment): target row i
+// A row-kernel CTA covers (sequence b, position i, vocabulary segment): target row i
 // and draft row i over the same segment (position gamma: the target row
 // alone).  The segment arrives in tiles of kTileVec 16-byte vectors per row;
 // each thread copies its kTileRegs vectors of a tile into registers, then
