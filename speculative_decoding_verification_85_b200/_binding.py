@@ -74,6 +74,19 @@ def lib() -> C.CDLL:
             L.sv_bandit_update_accept.restype = i32
             L.sv_bandit_stats.argtypes = [vp, vp, vp]
             L.sv_bandit_stats.restype = i32
+            L.spec_verify_shard_stats_bytes.argtypes = [i32, i32]
+            L.spec_verify_shard_stats_bytes.restype = sz
+            L.spec_verify_shard_candidate_bytes.argtypes = [i32]
+            L.spec_verify_shard_candidate_bytes.restype = sz
+            L.spec_verify_shard_stats.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32,
+                                                  vp, vp, sz, vp]
+            L.spec_verify_shard_stats.restype = i32
+            L.spec_verify_shard_decide.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32,
+                                                   vp, i32, u64, u64, vp, vp, vp, vp, vp, vp, sz,
+                                                   vp]
+            L.spec_verify_shard_decide.restype = i32
+            L.spec_verify_shard_pick.argtypes = [vp, i32, i32, i32, vp, vp, vp]
+            L.spec_verify_shard_pick.restype = i32
             _lib = L
     return _lib
 
@@ -269,6 +282,140 @@ def spec_verify_noalloc(target, draft, tokens, temps, *, seed: int = 0, step: in
 def spec_verify_noalloc_max_workspace() -> int:
     """Bytes of the fixed scratch array behind spec_verify_noalloc."""
     return int(lib().spec_verify_noalloc_max_workspace())
+
+
+# ------------------------------------------------------------ vocabulary shards
+SHARD_ALIGN = 1024  # shard offsets are multiples of one race group
+
+
+def vocab_shards(V: int, n: int):
+    """[(v0, Vs)] for n ranks over a vocabulary of V: widths rounded up to
+    multiples of SHARD_ALIGN (the last shard takes the rest), so no race group
+    straddles two ranks.  Ranks past the end of the vocabulary get no shard
+    (Vs == 0) and must not call the shard entry points."""
+    if V < 1 or n < 1:
+        raise ValueError("V and n must be positive")
+    w = -(-V // n)
+    w = -(-w // SHARD_ALIGN) * SHARD_ALIGN
+    out = []
+    for r in range(n):
+        v0 = min(r * w, V)
+        out.append((v0, min(w, V - v0)))
+    return out
+
+
+def shard_stats_bytes(B: int, gamma: int) -> int:
+    return int(lib().spec_verify_shard_stats_bytes(B, gamma))
+
+
+def shard_candidate_bytes(B: int) -> int:
+    return int(lib().spec_verify_shard_candidate_bytes(B))
+
+
+def _shard_inputs(target, draft, tokens, temps):
+    for t, n in ((target, "target"), (draft, "draft"), (tokens, "tokens"), (temps, "temps")):
+        _dev(t, n)
+    B, g1, Vs = target.shape
+    g = g1 - 1
+    if draft.dtype != target.dtype or tuple(draft.shape) != (B, g, Vs):
+        raise ValueError("draft shard must match target's dtype and be [B, gamma, Vs]")
+    if tokens.dtype != torch.int32 or tuple(tokens.shape) != (B, g):
+        raise ValueError("tokens must be int32 [B, gamma]")
+    if temps.dtype != torch.float32 or tuple(temps.shape) != (B,):
+        raise ValueError("temps must be float32 [B]")
+    return B, g, Vs, _dt(target)
+
+
+def spec_verify_shard_stats(target, draft, tokens, temps, *, V: int, v0: int, workspace,
+                            out_stats=None, stream=None):
+    """Call 1 of vocabulary-sharded verification on this rank's shard
+    (target [B, g+1, Vs], draft [B, g, Vs] = columns [v0, v0 + Vs) of the
+    full rows).  Returns the rank's statistics record (uint8)."""
+    B, g, Vs, dt = _shard_inputs(target, draft, tokens, temps)
+    dev = target.device
+    if out_stats is None:
+        out_stats = torch.empty(max(shard_stats_bytes(B, g), 16), dtype=torch.uint8, device=dev)
+    with _on(dev):
+        _check(lib().spec_verify_shard_stats(
+            _ptr(target), _ptr(draft), _ptr(tokens), _ptr(temps), B, g, V, v0, Vs, dt,
+            _ptr(out_stats), _ptr(workspace), workspace.numel() * workspace.element_size(),
+            _stream(dev, stream)))
+    return out_stats
+
+
+def spec_verify_shard_decide(target, draft, tokens, temps, all_stats, *, V: int, v0: int,
+                             nshards: int, workspace, seed: int = 0, step: int = 0,
+                             out_accept_len=None, out_tokens=None, with_logprobs: bool = False,
+                             out_candidate=None, stream=None):
+    """Call 2: the decision from the gathered records of all nshards ranks,
+    and this shard's race candidate.  Returns (accept_len, tokens, lp, lq,
+    candidate); tokens[b][accept_len[b]] is filled by call 3."""
+    B, g, Vs, dt = _shard_inputs(target, draft, tokens, temps)
+    _dev(all_stats, "all_stats")
+    dev = target.device
+    if out_accept_len is None:
+        out_accept_len = torch.empty(B, dtype=torch.int32, device=dev)
+    if out_tokens is None:
+        out_tokens = torch.empty((B, g + 1), dtype=torch.int32, device=dev)
+    lp = torch.empty((B, g), dtype=torch.float32, device=dev) if with_logprobs else None
+    lq = torch.empty((B, g), dtype=torch.float32, device=dev) if with_logprobs else None
+    if out_candidate is None:
+        out_candidate = torch.empty(max(shard_candidate_bytes(B), 16), dtype=torch.uint8,
+                                    device=dev)
+    with _on(dev):
+        _check(lib().spec_verify_shard_decide(
+            _ptr(target), _ptr(draft), _ptr(tokens), _ptr(temps), B, g, V, v0, Vs, dt,
+            _ptr(all_stats), nshards, seed, step, _ptr(out_accept_len), _ptr(out_tokens),
+            _ptr(lp), _ptr(lq), _ptr(out_candidate), _ptr(workspace),
+            workspace.numel() * workspace.element_size(), _stream(dev, stream)))
+    return out_accept_len, out_tokens, lp, lq, out_candidate
+
+
+def spec_verify_shard_pick(all_candidates, *, nshards: int, out_accept_len, out_tokens,
+                           stream=None):
+    """Call 3: the drawn token from the gathered candidates of all ranks."""
+    for t, n in ((all_candidates, "all_candidates"), (out_accept_len, "out_accept_len"),
+                 (out_tokens, "out_tokens")):
+        _dev(t, n)
+    B, g1 = out_tokens.shape
+    dev = out_tokens.device
+    with _on(dev):
+        _check(lib().spec_verify_shard_pick(_ptr(all_candidates), nshards, B, g1 - 1,
+                                            _ptr(out_accept_len), _ptr(out_tokens),
+                                            _stream(dev, stream)))
+    return out_accept_len, out_tokens
+
+
+def gather_records(local: torch.Tensor, group=None) -> torch.Tensor:
+    """All-gather of one byte record per rank, concatenated in rank order
+    (the exchange between the shard calls)."""
+    import torch.distributed as dist
+    n = dist.get_world_size(group)
+    out = torch.empty(n * local.numel(), dtype=local.dtype, device=local.device)
+    dist.all_gather_into_tensor(out, local, group=group)
+    return out
+
+
+def spec_verify_vocab_sharded(target, draft, tokens, temps, *, V: int, v0: int, seed: int = 0,
+                              step: int = 0, group=None, workspace=None,
+                              with_logprobs: bool = False, exchange=gather_records):
+    """The three shard calls with the two exchanges between them, on this
+    rank of `group` (every rank of the group calls it with its own shard).
+    Returns (accept_len, tokens, lp, lq), the same on every rank."""
+    import torch.distributed as dist
+    n = dist.get_world_size(group)
+    B, g, Vs, dt = _shard_inputs(target, draft, tokens, temps)
+    if workspace is None:
+        workspace = _zeroed(workspace_size(B, g, Vs, dt), target.device)
+    stats = spec_verify_shard_stats(target, draft, tokens, temps, V=V, v0=v0,
+                                    workspace=workspace)
+    all_stats = exchange(stats, group)
+    acc, tok, lp, lq, cand = spec_verify_shard_decide(
+        target, draft, tokens, temps, all_stats, V=V, v0=v0, nshards=n, workspace=workspace,
+        seed=seed, step=step, with_logprobs=with_logprobs)
+    spec_verify_shard_pick(exchange(cand, group), nshards=n, out_accept_len=acc,
+                           out_tokens=tok)
+    return acc, tok, lp, lq
 
 
 class Verifier:

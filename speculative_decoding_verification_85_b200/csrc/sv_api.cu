@@ -7,6 +7,7 @@
 #include <mutex>
 
 #include "spec_verify.h"
+#include "spec_verify_shard.h"
 #include "sv_internal.h"
 
 namespace sv {
@@ -104,7 +105,7 @@ using namespace sv;
 
 extern "C" {
 
-int spec_verify_version(void) { return (1 << 16) | 0; }
+int spec_verify_version(void) { return (1 << 16) | 1; }
 
 const char* spec_verify_last_error(void) { return g_err; }
 
@@ -166,6 +167,93 @@ int spec_verify(const void* target_logits, const void* draft_logits, const int32
   return launch_single(target_logits, draft_logits, draft_tokens, temps, B, gamma, V, dtype, seed,
                        step, out_accept_len, out_tokens, out_target_logp, out_draft_logp, workspace,
                        lay, static_cast<cudaStream_t>(stream));
+}
+
+// ------------------------------------------------------- vocabulary shards
+size_t spec_verify_shard_stats_bytes(int B, int gamma) {
+  if (B < 0 || B > SV_MAX_BATCH || gamma < 1 || gamma > SV_MAX_GAMMA) return 0;
+  return static_cast<size_t>(B) * (gamma + 1) * 3 * sizeof(float4);
+}
+
+size_t spec_verify_shard_candidate_bytes(int B) {
+  if (B < 0 || B > SV_MAX_BATCH) return 0;
+  return static_cast<size_t>(B) * sizeof(ShardCand);
+}
+
+static int check_shard(int V, int v0, int Vs) {
+  if (v0 < 0 || Vs < 1 || static_cast<long long>(v0) + Vs > V)
+    return set_error(SV_ERR_INVALID_ARG, "shard [v0, v0 + Vs) = [%d, %lld) must lie in [0, V = %d)",
+                     v0, static_cast<long long>(v0) + Vs, V);
+  if (v0 % SV_SHARD_ALIGN)
+    return set_error(SV_ERR_INVALID_ARG, "shard offset v0 = %d must be a multiple of %d", v0,
+                     SV_SHARD_ALIGN);
+  if (v0 + Vs != V && Vs % SV_SHARD_ALIGN)
+    return set_error(SV_ERR_INVALID_ARG,
+                     "every shard but the last needs a width that is a multiple of %d (got Vs = %d)",
+                     SV_SHARD_ALIGN, Vs);
+  return SV_OK;
+}
+
+static bool aligned16(const void* q) { return reinterpret_cast<uintptr_t>(q) % 16 == 0; }
+
+int spec_verify_shard_stats(const void* target_shard, const void* draft_shard,
+                            const int32_t* draft_tokens, const float* temps, int B, int gamma,
+                            int V, int v0, int Vs, int dtype, void* out_stats, void* workspace,
+                            size_t workspace_bytes, void* stream) {
+  const bool shape_ok = B > 0 && sizes_ok(B, gamma, Vs, dtype);
+  const Layout lay = shape_ok ? layout_single(B, gamma, Vs, dtype) : Layout{};
+  int rc = check_common(target_shard, draft_shard, draft_tokens, temps, B, gamma, Vs, dtype, 0,
+                        out_stats, out_stats, workspace, workspace_bytes, lay.total);
+  if (rc != SV_OK || B == 0) return rc;
+  if ((rc = check_shard(V, v0, Vs)) != SV_OK) return rc;
+  if (!aligned16(out_stats)) return set_error(SV_ERR_INVALID_ARG, "out_stats must be 16-byte aligned");
+  if ((rc = check_device()) != SV_OK) return rc;
+  return launch_shard_stats(target_shard, draft_shard, draft_tokens, temps, B, gamma, V, v0, Vs,
+                            dtype, out_stats, workspace, lay, static_cast<cudaStream_t>(stream));
+}
+
+int spec_verify_shard_decide(const void* target_shard, const void* draft_shard,
+                             const int32_t* draft_tokens, const float* temps, int B, int gamma,
+                             int V, int v0, int Vs, int dtype, const void* all_stats, int nshards,
+                             uint64_t seed, uint64_t step, int32_t* out_accept_len,
+                             int32_t* out_tokens, float* out_target_logp, float* out_draft_logp,
+                             void* out_candidate, void* workspace, size_t workspace_bytes,
+                             void* stream) {
+  const bool shape_ok = B > 0 && sizes_ok(B, gamma, Vs, dtype);
+  const Layout lay = shape_ok ? layout_single(B, gamma, Vs, dtype) : Layout{};
+  int rc = check_common(target_shard, draft_shard, draft_tokens, temps, B, gamma, Vs, dtype, step,
+                        out_accept_len, out_tokens, workspace, workspace_bytes, lay.total);
+  if (rc != SV_OK || B == 0) return rc;
+  if ((rc = check_shard(V, v0, Vs)) != SV_OK) return rc;
+  if (nshards < 1 || nshards > SV_MAX_SHARDS)
+    return set_error(SV_ERR_INVALID_ARG, "nshards must be in [1, %d] (got %d)", SV_MAX_SHARDS, nshards);
+  if (!all_stats || !out_candidate) return set_error(SV_ERR_INVALID_ARG, "NULL shard buffer");
+  if (!aligned16(all_stats) || !aligned16(out_candidate))
+    return set_error(SV_ERR_INVALID_ARG, "shard buffers must be 16-byte aligned");
+  if ((rc = check_device()) != SV_OK) return rc;
+  return launch_shard_decide(target_shard, draft_shard, draft_tokens, temps, B, gamma, V, v0, Vs,
+                             dtype, all_stats, nshards, seed, step, out_accept_len, out_tokens,
+                             out_target_logp, out_draft_logp, out_candidate, workspace, lay,
+                             static_cast<cudaStream_t>(stream));
+}
+
+int spec_verify_shard_pick(const void* all_candidates, int nshards, int B, int gamma,
+                           int32_t* out_accept_len, int32_t* out_tokens, void* stream) {
+  if (B < 0 || B > SV_MAX_BATCH)
+    return set_error(SV_ERR_INVALID_ARG, "B must be in [0, %d] (got %d)", SV_MAX_BATCH, B);
+  if (gamma < 1 || gamma > SV_MAX_GAMMA)
+    return set_error(SV_ERR_INVALID_ARG, "draft length must be in [1, %d] (got %d)", SV_MAX_GAMMA, gamma);
+  if (nshards < 1 || nshards > SV_MAX_SHARDS)
+    return set_error(SV_ERR_INVALID_ARG, "nshards must be in [1, %d] (got %d)", SV_MAX_SHARDS, nshards);
+  if (B == 0) return SV_OK;
+  if (!all_candidates || !out_accept_len || !out_tokens)
+    return set_error(SV_ERR_INVALID_ARG, "NULL input or output pointer");
+  if (!aligned16(all_candidates))
+    return set_error(SV_ERR_INVALID_ARG, "all_candidates must be 16-byte aligned");
+  int rc;
+  if ((rc = check_device()) != SV_OK) return rc;
+  return launch_shard_pick(all_candidates, nshards, B, gamma, out_accept_len, out_tokens,
+                           static_cast<cudaStream_t>(stream));
 }
 
 static int multidraft_call(const void* target_logits, const void* draft_logits,

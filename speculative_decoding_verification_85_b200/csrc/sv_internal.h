@@ -31,6 +31,20 @@ struct alignas(16) RacePartial {
   int pad;
 };
 
+// Vocabulary shards: one rank's race candidate for sequence b (32 bytes,
+// the layout spec_verify_shard.h documents).
+enum ShardKind { kShardNoDraw = 0, kShardDrawLaw = 1, kShardTargetRace = 2 };
+struct alignas(16) ShardCand {
+  float w;      // the shard's best group weight (0: no mass in this shard)
+  float e;      // its exponential
+  int group;    // its global group index
+  int token;    // the level-2 winner inside that group (-1: none)
+  int kind;     // ShardKind
+  int j;        // draw position
+  int pad0, pad1;
+};
+static_assert(sizeof(ShardCand) == 32, "candidate record is 32 bytes");
+
 // Inputs, outputs and decision state of a single-draft call.
 struct CallParams {
   const void* target;
@@ -88,5 +102,19 @@ int launch_multi(const void* target, const void* draft, const int32_t* tokens,
                  int32_t* out_draft_index, void* workspace, const Layout& lay,
                  cudaStream_t stream);
 int multidraft_max_row_sets(int L);  // largest K with a row set per draft (sv_multi.cu)
+
+// Vocabulary-sharded single draft (sv_single.cu).  The target / draft
+// pointers are the shard's [B][gamma + 1][Vs] / [B][gamma][Vs] rows.
+int launch_shard_stats(const void* target, const void* draft, const int32_t* tokens,
+                       const float* temps, int B, int gamma, int V, int v0, int Vs, int dtype,
+                       void* out_stats, void* workspace, const Layout& lay, cudaStream_t stream);
+int launch_shard_decide(const void* target, const void* draft, const int32_t* tokens,
+                        const float* temps, int B, int gamma, int V, int v0, int Vs, int dtype,
+                        const void* all_stats, int nshards, uint64_t seed, uint64_t step,
+                        int32_t* out_accept_len, int32_t* out_tokens, float* out_lp,
+                        float* out_lq, void* out_candidate, void* workspace, const Layout& lay,
+                        cudaStream_t stream);
+int launch_shard_pick(const void* all_candidates, int nshards, int B, int gamma,
+                      int32_t* out_accept_len, int32_t* out_tokens, cudaStream_t stream);
 
 }  // namespace sv

@@ -55,6 +55,12 @@ struct SingleParams {
                         // covers tiles [s tiles / nseg, (s + 1) tiles / nseg)
   float4* pairpart;     // [B][gamma + 1][nseg] x {target, draft} partials
   float* zx;            // [B][gamma][nseg][2] draft token's target / draft logit
+  // vocabulary shards (kShard kernels only): this shard's first column, the
+  // full vocabulary, the shard's statistics record and race candidates
+  int voff;
+  int vfull;
+  float4* xstats;       // [B][gamma + 1][3]
+  ShardCand* cand;      // [B]
 };
 
 template <bool kBf16>
@@ -120,6 +126,41 @@ __device__ __forceinline__ float sum_rel_max(const RowAcc& a, float c) {
   return a.s * ex2_approx(e);
 }
 
+// Merge, by one warp, the nseg segment partials of position i of sequence b:
+// target row A, draft row B (raw {m, S, R} or {m, -, argmax, bad}), and the
+// draft token's two logits (NaN where no segment holds the token).
+__device__ __forceinline__ void merge_segments(const SingleParams& f, int b, int i, bool argmaxA,
+                                               RowAcc& A, RowAcc& B, float& zt, float& zd) {
+  const int lane = threadIdx.x & 31;
+  const int g = f.p1.gamma;
+  A = argmaxA ? empty_argmax_acc() : empty_lse_acc();
+  B = empty_lse_acc();
+  zt = __int_as_float(0x7fc00000);
+  zd = zt;
+  const float4* pp = f.pairpart + (static_cast<size_t>(b) * (g + 1) + i) * f.nseg * 2;
+  const float* zp = f.zx + (static_cast<size_t>(b) * g + i) * f.nseg * 2;
+  for (int q = lane; q < f.nseg; q += 32) {
+    const float4 a = __ldcg(pp + 2 * q), d = __ldcg(pp + 2 * q + 1);
+    merge_ref(A, RowAcc{a.x, a.y, __float_as_int(a.z), __float_as_int(a.w)}, argmaxA);
+    merge_ref(B, RowAcc{d.x, d.y, __float_as_int(d.z), __float_as_int(d.w)}, false);
+    if (i < g) {
+      // the draft token's logits: the one segment that holds it reports them
+      const float za = __ldcg(zp + 2 * q), zb = __ldcg(zp + 2 * q + 1);
+      if (za == za) zt = za;
+      if (zb == zb) zd = zb;
+    }
+  }
+  warp_merge(A, argmaxA);
+  warp_merge(B, false);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    const float a = __shfl_xor_sync(0xffffffffu, zt, off);
+    const float d = __shfl_xor_sync(0xffffffffu, zd, off);
+    if (zt != zt) zt = a;
+    if (zd != zd) zd = d;
+  }
+}
+
 // Combine the nseg segment partials of every position of sequence b into the
 // row table rows[] (target rows 0..gamma, then draft rows), and pick up the
 // draft tokens' logits (zsel[2i], zsel[2i+1]).  argmaxA and c describe the
@@ -129,30 +170,9 @@ __device__ __forceinline__ void combine_pairs(const SingleParams& f, int b, bool
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int g = f.p1.gamma;
   for (int i = warp; i <= g; i += kRowThreads / 32) {
-    RowAcc A = argmaxA ? empty_argmax_acc() : empty_lse_acc(), B = empty_lse_acc();
-    float zt = __int_as_float(0x7fc00000), zd = zt;
-    const float4* pp = f.pairpart + (static_cast<size_t>(b) * (g + 1) + i) * f.nseg * 2;
-    const float* zp = f.zx + (static_cast<size_t>(b) * g + i) * f.nseg * 2;
-    for (int q = lane; q < f.nseg; q += 32) {
-      const float4 a = __ldcg(pp + 2 * q), d = __ldcg(pp + 2 * q + 1);
-      merge_ref(A, RowAcc{a.x, a.y, __float_as_int(a.z), __float_as_int(a.w)}, argmaxA);
-      merge_ref(B, RowAcc{d.x, d.y, __float_as_int(d.z), __float_as_int(d.w)}, false);
-      if (i < g) {
-        // the draft token's logits: the one segment that holds it reports them
-        const float za = __ldcg(zp + 2 * q), zb = __ldcg(zp + 2 * q + 1);
-        if (za == za) zt = za;
-        if (zb == zb) zd = zb;
-      }
-    }
-    warp_merge(A, argmaxA);
-    warp_merge(B, false);
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-      const float a = __shfl_xor_sync(0xffffffffu, zt, off);
-      const float d = __shfl_xor_sync(0xffffffffu, zd, off);
-      if (zt != zt) zt = a;
-      if (zd != zd) zd = d;
-    }
+    RowAcc A, B;
+    float zt, zd;
+    merge_segments(f, b, i, argmaxA, A, B, zt, zd);
     if (lane == 0) {
       if (!argmaxA) A.s = sum_rel_max(A, c);
       B.s = sum_rel_max(B, c);
@@ -165,6 +185,26 @@ __device__ __forceinline__ void combine_pairs(const SingleParams& f, int b, bool
     }
   }
   block_sync<kRowThreads>();
+}
+
+// Vocabulary shards: the shard's record of sequence b, per position the
+// merged target and draft partials as they merge across shards (raw, argmax
+// as a global index) and the draft token's two logits.
+__device__ __forceinline__ void export_pairs(const SingleParams& f, int b, bool argmaxA) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int g = f.p1.gamma;
+  for (int i = warp; i <= g; i += kRowThreads / 32) {
+    RowAcc A, B;
+    float zt, zd;
+    merge_segments(f, b, i, argmaxA, A, B, zt, zd);
+    if (lane == 0) {
+      if (argmaxA && A.arg != 0x7fffffff) A.arg += f.voff;
+      float4* o = f.xstats + (static_cast<size_t>(b) * (g + 1) + i) * 3;
+      o[0] = make_float4(A.m, A.s, __int_as_float(A.arg), __int_as_float(A.bad));
+      o[1] = make_float4(B.m, B.s, __int_as_float(B.arg), __int_as_float(B.bad));
+      o[2] = make_float4(zt, zd, 0.0f, 0.0f);
+    }
+  }
 }
 
 // Head (entries before the first 16-byte boundary) and tail (after the last)
@@ -212,8 +252,10 @@ __device__ __forceinline__ void pick_logit(const uint4 (&r)[kTileRegs], int own,
 // --------------------------------------------------------------- row kernel
 // Grid: one CTA per (row pair, segment), blockIdx.x = (b (gamma + 1) + i)
 // nseg + seg: a sequence's CTAs are consecutive, so sequences complete in
-// order of b while the kernel runs.
-template <bool kBf16>
+// order of b while the kernel runs.  kShard: the rows are one vocabulary
+// shard (columns [voff, voff + V) of vfull), and the CTA that completes a
+// sequence writes the shard's record instead of deciding.
+template <bool kBf16, bool kShard = false>
 __global__ void __launch_bounds__(kRowThreads, 3) rows_kernel(const __grid_constant__ SingleParams f) {
   __shared__ RowAcc rows[kMaxRowsPerSeq];
   __shared__ RowAcc scratch[2 * (kRowThreads / 32)];
@@ -237,7 +279,12 @@ __global__ void __launch_bounds__(kRowThreads, 3) rows_kernel(const __grid_const
   int xg = -1;
   if (modeA == kRowLse && i < p.gamma) {
     const int xt = __ldg(p.tokens + static_cast<size_t>(b) * p.gamma + i);
-    if (xt >= 0 && xt < p.V) xg = xt;
+    if constexpr (kShard) {
+      const int xl = xt - f.voff;  // the token's column in this shard
+      if (xt >= 0 && xt < f.vfull && xl >= 0 && xl < p.V) xg = xl;
+    } else {
+      if (xt >= 0 && xt < p.V) xg = xt;
+    }
   }
   if (tid == 0) s_zx[0] = s_zx[1] = __int_as_float(0x7fc00000);  // NaN: "not in this segment"
   // the sequence's draft tokens, for the decision if this CTA completes it
@@ -309,6 +356,10 @@ __global__ void __launch_bounds__(kRowThreads, 3) rows_kernel(const __grid_const
   }
   block_sync<kRowThreads>();  // orders the other threads after thread 0's acquire
   if (!s_last) return;
+  if constexpr (kShard) {
+    export_pairs(f, b, argmaxA);
+    return;
+  }
   combine_pairs(f, b, argmaxA, c, rows, s_zsel);
   if (tid < 32) {
     decide_single<kBf16>(p, b, T, s_tok, rows, s_zsel, p.info + b, true, nullptr);
@@ -446,10 +497,13 @@ struct DrawRow {
 // the lanes gives every lane the same W_g.  The k-th group's W_g stays with
 // lane k % 32; every 32 groups (and at the end) those lanes draw their
 // groups' exponentials in parallel and enter the race.  Returns the warp's
-// winner in (bw, be, bi) (bi: the group index).
+// winner in (bw, be, bi) (bi: the group index).  goff: the global index of
+// the row's group 0 (a vocabulary shard's offset / 1024; 0 for whole rows):
+// the race keys and bi are global, the loads local.
 template <bool kBf16>
 __device__ __forceinline__ void race_groups(const DrawRow<kBf16>& r, const RaceKey& gkey, int g0,
-                                            int gstride, int g1, float& bw, float& be, int& bi) {
+                                            int gstride, int g1, float& bw, float& be, int& bi,
+                                            int goff) {
   constexpr int kPasses = kRaceGroup / 128;
   constexpr int kBatch = kBf16 ? 8 : 4;  // passes loaded together (32 registers of logits)
   const int lane = threadIdx.x & 31;
@@ -489,23 +543,24 @@ __device__ __forceinline__ void race_groups(const DrawRow<kBf16>& r, const RaceK
     for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
     if (lane == (k & 31)) {
       myW = s;
-      myG = gid;
+      myG = gid + goff;
     }
     if ((k & 31) == 31) enter();
   }
   enter();
 }
 
-// Level 2, by the whole CTA: the entries of group gid, one Philox block per
-// thread (block 256 gid + t), in the race of w_v / E_v with the per-entry
-// noise.  Returns the CTA's winner in every thread.
+// Level 2, by the whole CTA: the entries of global group gid, one Philox
+// block per thread (block 256 gid + t), in the race of w_v / E_v with the
+// per-entry noise; the row's group 0 is global group goff.  Returns the CTA's
+// winner (a global vocabulary index) in every thread.
 template <bool kBf16>
 __device__ __forceinline__ int race_entries(const DrawRow<kBf16>& r, const RaceKey& ekey, int gid,
-                                            float4* scratch) {
+                                            float4* scratch, int goff) {
   static_assert(kDrawThreads * 4 == kRaceGroup, "one Philox block per thread");
-  const int g = gid * (kRaceGroup / 4) + static_cast<int>(threadIdx.x);
+  const int g = gid * (kRaceGroup / 4) + static_cast<int>(threadIdx.x);  // global block
   Block4<kBf16> tb, db;
-  r.load(g, tb, db);
+  r.load(g - goff * (kRaceGroup / 4), tb, db);
   const float4 w4 = r.weights(tb, db);
   const float w[4] = {w4.x, w4.y, w4.z, w4.w};
   const uint4 rnd = ekey.block(g);
@@ -527,16 +582,23 @@ __device__ __forceinline__ int race_entries(const DrawRow<kBf16>& r, const RaceK
 
 // Both levels over the whole target row j in one CTA: the draw from p_j
 // when the residual max(p_j - q_j, 0) vanished (p_j == q_j to rounding).
+// The level-1 winner goes to *win ({w, E, global group}) when win is not
+// NULL; -1 when no entry of the row has weight (a vocabulary shard far
+// below the row's maximum).
 template <bool kBf16>
 __device__ __noinline__ int draw_from_target(const CallParams& p, const SeqInfo& si, int b,
-                                             const RaceKey& gkey, const RaceKey& ekey, float4* scratch) {
+                                             const RaceKey& gkey, const RaceKey& ekey, float4* scratch,
+                                             int goff, float4* win) {
   const DrawRow<kBf16> prow(p, si, b, false);
   const int ng = (p.V + kRaceGroup - 1) / kRaceGroup;
   float bw = 0.0f, be = 1.0f;
   int bi = INT_MAX;
-  race_groups<kBf16>(prow, gkey, static_cast<int>(threadIdx.x >> 5), kDrawThreads / 32, ng, bw, be, bi);
+  race_groups<kBf16>(prow, gkey, static_cast<int>(threadIdx.x >> 5), kDrawThreads / 32, ng, bw, be, bi,
+                     goff);
   race_reduce<kDrawThreads>(bw, be, bi, scratch);
-  return race_entries<kBf16>(prow, ekey, bi, scratch);
+  if (win) *win = make_float4(bw, be, __int_as_float(bi), 0.0f);
+  if (!(bw > 0.0f)) return -1;  // uniform: race_reduce returns the winner to every thread
+  return race_entries<kBf16>(prow, ekey, bi, scratch, goff);
 }
 
 // Draw kernel.  Grid: nc2 CTAs per sequence; CTA c of sequence b runs level
@@ -556,7 +618,12 @@ __device__ __forceinline__ bool wait_ready(const unsigned* flag) {
   }
 }
 
-template <bool kBf16>
+// kShard: the rows are one vocabulary shard; the race runs over the shard's
+// groups with global group and entry indices, and the completing CTA writes
+// the shard's candidate (its best group with that group's level-2 winner, or,
+// where the shard's residual has no weight, the same for the race over p_j)
+// instead of the token.
+template <bool kBf16, bool kShard = false>
 __global__ void __launch_bounds__(kDrawThreads, 4) draw_kernel(const __grid_constant__ SingleParams f) {
   __shared__ float4 scratch[kDrawThreads / 32];
   __shared__ int s_last, s_ready;
@@ -595,12 +662,14 @@ __global__ void __launch_bounds__(kDrawThreads, 4) draw_kernel(const __grid_cons
   const RaceKey gkey{k0, k1, static_cast<uint32_t>(b), p.step, (kTagGroup << 24) | static_cast<uint32_t>(si.j)};
   const RaceKey ekey{k0, k1, static_cast<uint32_t>(b), p.step, (kTagGumbel << 24) | static_cast<uint32_t>(si.j)};
   const int ng = (p.V + kRaceGroup - 1) / kRaceGroup;
+  const int goff = kShard ? f.voff / kRaceGroup : 0;
   float bw = 0.0f, be = 1.0f;
   int bi = INT_MAX;
   if (draw) {  // uniform
     const DrawRow<kBf16> row(p, si, b, si.mode == kModeResidual);
     const int gc0 = chunk * f.gpc;
-    race_groups<kBf16>(row, gkey, gc0 + warp, kDrawThreads / 32, min(ng, gc0 + f.gpc), bw, be, bi);
+    race_groups<kBf16>(row, gkey, gc0 + warp, kDrawThreads / 32, min(ng, gc0 + f.gpc), bw, be, bi,
+                       goff);
     race_reduce<kDrawThreads>(bw, be, bi, scratch);
   }
   // Every CTA of the sequence arrives (drawing or not), so the last one can
@@ -616,7 +685,13 @@ __global__ void __launch_bounds__(kDrawThreads, 4) draw_kernel(const __grid_cons
     }
   }
   block_sync<kDrawThreads>();  // orders the other threads after thread 0's acquire
-  if (!s_last || !draw) return;
+  if (!s_last) return;
+  if constexpr (!kShard) {
+    if (!draw) return;
+  } else if (!draw) {
+    if (threadIdx.x == 0) f.cand[b] = ShardCand{0.0f, 1.0f, INT_MAX, -1, kShardNoDraw, si.j, 0, 0};
+    return;
+  }
   bw = 0.0f;
   be = 1.0f;
   bi = INT_MAX;
@@ -629,14 +704,134 @@ __global__ void __launch_bounds__(kDrawThreads, 4) draw_kernel(const __grid_cons
     }
   }
   race_reduce<kDrawThreads>(bw, be, bi, scratch);
-  int y;
-  if (bw > 0.0f) {  // uniform: race_reduce returns the winner to every thread
-    const DrawRow<kBf16> row(p, si, b, si.mode == kModeResidual);
-    y = race_entries<kBf16>(row, ekey, bi, scratch);
+  if constexpr (kShard) {
+    ShardCand cd{bw, be, bi, -1, kShardDrawLaw, si.j, 0, 0};
+    if (bw > 0.0f) {  // uniform
+      const DrawRow<kBf16> row(p, si, b, si.mode == kModeResidual);
+      cd.token = race_entries<kBf16>(row, ekey, bi, scratch, goff);
+    } else if (si.mode == kModeResidual) {
+      // no residual weight in this shard: its candidate of the race over p_j,
+      // used only if no shard has residual weight
+      float4 w;
+      cd.token = draw_from_target<kBf16>(p, si, b, gkey, ekey, scratch, goff, &w);
+      cd = ShardCand{w.x, w.y, __float_as_int(w.z), cd.token, kShardTargetRace, si.j, 0, 0};
+    }
+    if (threadIdx.x == 0) f.cand[b] = cd;
   } else {
-    y = draw_from_target<kBf16>(p, si, b, gkey, ekey, scratch);  // the residual vanished
+    int y;
+    if (bw > 0.0f) {  // uniform: race_reduce returns the winner to every thread
+      const DrawRow<kBf16> row(p, si, b, si.mode == kModeResidual);
+      y = race_entries<kBf16>(row, ekey, bi, scratch, 0);
+    } else {
+      y = draw_from_target<kBf16>(p, si, b, gkey, ekey, scratch, 0, nullptr);  // the residual vanished
+    }
+    if (threadIdx.x == 0) p.out_tokens[static_cast<size_t>(b) * (p.gamma + 1) + si.j] = y;
   }
-  if (threadIdx.x == 0) p.out_tokens[static_cast<size_t>(b) * (p.gamma + 1) + si.j] = y;
+}
+
+// ------------------------------------------------- vocabulary shards: decide
+// Sequence inputs of the decision over all shards' records.
+struct ShardDecideParams {
+  CallParams p;          // V: the full vocabulary (draft-token validity)
+  const float4* stats;   // [nshards][B][gamma + 1][3]: the gathered records
+  int nshards;
+  unsigned* ready;       // [B] decision published (cleared by the draw kernel)
+};
+
+// One CTA per sequence: merge the shards' records of every position (a warp
+// per position, lane r merging rank r's record, then a butterfly: the same
+// order on every rank, so every rank reaches the same bits), then the
+// decision, published to the draw kernel by the sequence's flag.
+template <bool kBf16>
+__global__ void __launch_bounds__(kRowThreads) shard_decide_kernel(const __grid_constant__ ShardDecideParams f) {
+  __shared__ RowAcc rows[kMaxRowsPerSeq];
+  __shared__ float s_zsel[2 * SV_MAX_GAMMA];
+  __shared__ int s_tok[SV_MAX_GAMMA];
+  pdl_wait_and_release();
+  const CallParams& p = f.p;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int b = blockIdx.x;
+  const int g = p.gamma;
+  const float T = __ldg(p.temps + b);
+  const int modeA = row_mode(T, true);
+  const bool argmaxA = modeA == kRowArgmax;
+  const float c = modeA == kRowLse ? __fdiv_rn(kLog2e, T) : 0.0f;
+  for (int k = tid; k < g; k += kRowThreads) s_tok[k] = __ldg(p.tokens + static_cast<size_t>(b) * g + k);
+  const size_t per_rank = static_cast<size_t>(p.B) * (g + 1) * 3;  // float4s in one rank's record
+  for (int i = warp; i <= g; i += kRowThreads / 32) {
+    RowAcc A = argmaxA ? empty_argmax_acc() : empty_lse_acc(), Bq = empty_lse_acc();
+    float zt = __int_as_float(0x7fc00000), zd = zt;
+    for (int r = lane; r < f.nshards; r += 32) {
+      const float4* o = f.stats + r * per_rank + (static_cast<size_t>(b) * (g + 1) + i) * 3;
+      const float4 a = __ldcg(o), d = __ldcg(o + 1), z = __ldcg(o + 2);
+      merge_ref(A, RowAcc{a.x, a.y, __float_as_int(a.z), __float_as_int(a.w)}, argmaxA);
+      merge_ref(Bq, RowAcc{d.x, d.y, __float_as_int(d.z), __float_as_int(d.w)}, false);
+      if (z.x == z.x) zt = z.x;  // the one shard that holds the draft token reports its logits
+      if (z.y == z.y) zd = z.y;
+    }
+    warp_merge(A, argmaxA);
+    warp_merge(Bq, false);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      const float a = __shfl_xor_sync(0xffffffffu, zt, off);
+      const float d = __shfl_xor_sync(0xffffffffu, zd, off);
+      if (zt != zt) zt = a;
+      if (zd != zd) zd = d;
+    }
+    if (lane == 0) {
+      if (!argmaxA) A.s = sum_rel_max(A, c);
+      Bq.s = sum_rel_max(Bq, c);
+      rows[i] = A;
+      if (i < g) {
+        rows[g + 1 + i] = Bq;
+        s_zsel[2 * i] = zt;
+        s_zsel[2 * i + 1] = zd;
+      }
+    }
+  }
+  block_sync<kRowThreads>();
+  if (tid < 32) {
+    decide_single<kBf16>(p, b, T, s_tok, rows, s_zsel, p.info + b, true, nullptr);
+    __threadfence();
+    __syncwarp();
+    if (tid == 0) st_release(f.ready + b, 1u);
+  }
+}
+
+// --------------------------------------------------- vocabulary shards: pick
+// One thread per sequence: the winning candidate over the gathered shards'
+// candidates (the draw law's when any shard has weight in it, else the race
+// over p_j), written at the draw position.  Shards that disagree on the draw
+// (a rank whose wait ran out reports none) mark the sequence invalid.
+__global__ void __launch_bounds__(256) shard_pick_kernel(const ShardCand* all, int nshards, int B,
+                                                          int gamma, int32_t* accept_len,
+                                                          int32_t* out_tokens) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int b = static_cast<int>(blockIdx.x * blockDim.x + threadIdx.x);
+  if (b >= B) return;
+  const ShardCand c0 = all[b];
+  float bw[2] = {0.0f, 0.0f}, be[2] = {1.0f, 1.0f};
+  int bi[2] = {INT_MAX, INT_MAX}, bt[2] = {-1, -1};
+  bool agree = true;
+  for (int r = 0; r < nshards; ++r) {
+    const ShardCand c = all[static_cast<size_t>(r) * B + b];
+    agree = agree && (c.kind == kShardNoDraw) == (c0.kind == kShardNoDraw) && c.j == c0.j;
+    const int k = c.kind == kShardTargetRace ? 1 : 0;
+    if (c.kind != kShardNoDraw && race_better(c.w, c.e, c.group, bw[k], be[k], bi[k])) {
+      bw[k] = c.w;
+      be[k] = c.e;
+      bi[k] = c.group;
+      bt[k] = c.token;
+    }
+  }
+  int32_t* tok = out_tokens + static_cast<size_t>(b) * (gamma + 1);
+  if (!agree) {
+    for (int i = 0; i <= gamma; ++i) tok[i] = -1;
+    accept_len[b] = -1;
+    return;
+  }
+  if (c0.kind == kShardNoDraw || c0.j < 0 || c0.j > gamma) return;
+  tok[c0.j] = bw[0] > 0.0f ? bt[0] : bt[1];
 }
 
 // ------------------------------------------------------------------ launch
@@ -708,9 +903,8 @@ int draw_ctas_per_sm(bool bf16) {
               : per_device(slots[0], 4, [](int) { return occupancy(draw_kernel<false>, kDrawThreads); });
 }
 
-template <typename K>
-cudaError_t launch_pdl(K kernel, dim3 grid, unsigned block, cudaStream_t stream,
-                       const SingleParams& f) {
+template <typename K, typename P>
+cudaError_t launch_pdl(K kernel, dim3 grid, unsigned block, cudaStream_t stream, const P& f) {
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = grid;
   cfg.blockDim = dim3(block);
@@ -728,39 +922,16 @@ cudaError_t launch_pdl(K kernel, dim3 grid, unsigned block, cudaStream_t stream,
   }
   return e;
 }
-}  // namespace
 
-int launch_single(const void* target, const void* draft, const int32_t* tokens,
-                  const float* temps, int B, int gamma, int V, int dtype, uint64_t seed,
-                  uint64_t step, int32_t* out_accept_len, int32_t* out_tokens, float* out_lp,
-                  float* out_lq, void* workspace, const Layout& lay, cudaStream_t stream) {
-  char* ws = static_cast<char*>(workspace);
-  SingleParams f{};
-  CallParams& p1 = f.p1;
-  p1.target = target;
-  p1.draft = draft;
-  p1.tokens = tokens;
-  p1.temps = temps;
-  p1.B = B;
-  p1.gamma = gamma;
-  p1.V = V;
-  p1.rps = 2 * gamma + 1;
-  p1.seed = seed;
-  p1.step = static_cast<uint32_t>(step);
-  p1.ticket = reinterpret_cast<unsigned*>(ws + lay.ticket1);
-  p1.info = reinterpret_cast<SeqInfo*>(ws + lay.info);
-  p1.accept_len = out_accept_len;
-  p1.out_tokens = out_tokens;
-  p1.out_lp = out_lp;
-  p1.out_lq = out_lq;
-  // a batch whose sequences fit one cluster each, in one wave, with every
-  // row slice in shared memory: the latency-bound case, one cluster kernel
-  if (small_path(B, gamma, V, dtype)) return launch_small(p1, dtype, stream);
-  // Row segments: whole tiles, about kRowWaves waves of CTAs over the GPU but
-  // at most kMaxSegTiles tiles per CTA; balanced so segments differ by at
-  // most one tile.  Long segments spread each CTA's fixed cost (launch, block
-  // reduce, ticket) over more streaming; about three waves keep the last one
-  // mostly full.
+// Row segments: whole tiles, about kRowWaves waves of CTAs over the GPU but
+// at most kMaxSegTiles tiles per CTA; balanced so segments differ by at most
+// one tile.  Long segments spread each CTA's fixed cost (launch, block
+// reduce, ticket) over more streaming; about three waves keep the last one
+// mostly full.  Draw CTAs: race groups per warp chosen so that the B
+// sequences' groups fill about kDrawWaves waves of CTAs (at least one group
+// per warp, so a small batch still spreads each row over several CTAs); a
+// CTA covers 8 warps' groups.  V is the width of the rows the kernels read.
+void set_policy(SingleParams& f, int B, int gamma, int V, int dtype, char* ws, const Layout& lay) {
   const bool bf16 = dtype == SV_BF16;
   {
     constexpr int kRowWaves = 3, kMaxSegTiles = 10;
@@ -779,10 +950,6 @@ int launch_single(const void* target, const void* draft, const int32_t* tokens,
   f.part2 = reinterpret_cast<RacePartial*>(ws + lay.part2);
   f.ticket2 = reinterpret_cast<unsigned*>(ws + lay.ticket2);
   f.ready = reinterpret_cast<unsigned*>(ws + lay.ready);
-  // Draw CTAs: race groups per warp chosen so that the B sequences' groups
-  // fill about kDrawWaves waves of CTAs (at least one group per warp, so a
-  // small batch still spreads each row over several CTAs); a CTA covers
-  // 8 warps' groups.
   {
     const long long ng = (V + kRaceGroup - 1) / kRaceGroup;
     const long long warps = static_cast<long long>(sm_count()) * draw_ctas_per_sm(bf16) * (kDrawThreads / 32);
@@ -792,7 +959,47 @@ int launch_single(const void* target, const void* draft, const int32_t* tokens,
     f.gpc = static_cast<int>(gpc < ng ? gpc : ng);
     f.nc2 = static_cast<int>((ng + f.gpc - 1) / f.gpc);  // <= lay.nc2: gpc >= 8 or nc2 == 1
   }
+}
 
+// The call's inputs, outputs and the workspace's counters; V is the width of
+// the rows (a shard's width for the vocabulary-sharded kernels).
+void set_call(CallParams& p1, const void* target, const void* draft, const int32_t* tokens,
+              const float* temps, int B, int gamma, int V, uint64_t seed, uint64_t step,
+              int32_t* out_accept_len, int32_t* out_tokens, float* out_lp, float* out_lq,
+              char* ws, const Layout& lay) {
+  p1.target = target;
+  p1.draft = draft;
+  p1.tokens = tokens;
+  p1.temps = temps;
+  p1.B = B;
+  p1.gamma = gamma;
+  p1.V = V;
+  p1.rps = 2 * gamma + 1;
+  p1.seed = seed;
+  p1.step = static_cast<uint32_t>(step);
+  p1.ticket = reinterpret_cast<unsigned*>(ws + lay.ticket1);
+  p1.info = reinterpret_cast<SeqInfo*>(ws + lay.info);
+  p1.accept_len = out_accept_len;
+  p1.out_tokens = out_tokens;
+  p1.out_lp = out_lp;
+  p1.out_lq = out_lq;
+}
+}  // namespace
+
+int launch_single(const void* target, const void* draft, const int32_t* tokens,
+                  const float* temps, int B, int gamma, int V, int dtype, uint64_t seed,
+                  uint64_t step, int32_t* out_accept_len, int32_t* out_tokens, float* out_lp,
+                  float* out_lq, void* workspace, const Layout& lay, cudaStream_t stream) {
+  char* ws = static_cast<char*>(workspace);
+  SingleParams f{};
+  CallParams& p1 = f.p1;
+  set_call(p1, target, draft, tokens, temps, B, gamma, V, seed, step, out_accept_len, out_tokens,
+           out_lp, out_lq, ws, lay);
+  // a batch whose sequences fit one cluster each, in one wave, with every
+  // row slice in shared memory: the latency-bound case, one cluster kernel
+  if (small_path(B, gamma, V, dtype)) return launch_small(p1, dtype, stream);
+  const bool bf16 = dtype == SV_BF16;
+  set_policy(f, B, gamma, V, dtype, ws, lay);
   if (static_cast<long long>(B) * f.nc2 > INT_MAX)
     return set_error(SV_ERR_INVALID_ARG, "B x V too large for one launch (draw grid %lld CTAs)",
                      static_cast<long long>(B) * f.nc2);
@@ -810,6 +1017,78 @@ int launch_single(const void* target, const void* draft, const int32_t* tokens,
   if (e != cudaSuccess)
     return set_error(SV_ERR_CUDA, "draw kernel launch failed: %s", cudaGetErrorString(e));
   return check_launch("verify");
+}
+
+// ---------------------------------------------------- vocabulary shards: launch
+namespace {
+int shard_params(SingleParams& f, const void* target, const void* draft, const int32_t* tokens,
+                 const float* temps, int B, int gamma, int V, int v0, int Vs, int dtype,
+                 uint64_t seed, uint64_t step, int32_t* out_accept_len, int32_t* out_tokens,
+                 float* out_lp, float* out_lq, void* workspace, const Layout& lay) {
+  char* ws = static_cast<char*>(workspace);
+  set_call(f.p1, target, draft, tokens, temps, B, gamma, Vs, seed, step, out_accept_len, out_tokens,
+           out_lp, out_lq, ws, lay);
+  set_policy(f, B, gamma, Vs, dtype, ws, lay);
+  f.voff = v0;
+  f.vfull = V;
+  if (static_cast<long long>(B) * f.nc2 > INT_MAX ||
+      static_cast<long long>(B) * (gamma + 1) * f.nseg > INT_MAX)
+    return set_error(SV_ERR_INVALID_ARG, "B x Vs too large for one launch");
+  return SV_OK;
+}
+}  // namespace
+
+int launch_shard_stats(const void* target, const void* draft, const int32_t* tokens,
+                       const float* temps, int B, int gamma, int V, int v0, int Vs, int dtype,
+                       void* out_stats, void* workspace, const Layout& lay, cudaStream_t stream) {
+  SingleParams f{};
+  int rc = shard_params(f, target, draft, tokens, temps, B, gamma, V, v0, Vs, dtype, 0, 0, nullptr,
+                        nullptr, nullptr, nullptr, workspace, lay);
+  if (rc != SV_OK) return rc;
+  f.xstats = static_cast<float4*>(out_stats);
+  const dim3 grid(static_cast<unsigned>(static_cast<long long>(B) * (gamma + 1) * f.nseg));
+  const cudaError_t e = dtype == SV_BF16 ? launch_pdl(rows_kernel<true, true>, grid, kRowThreads, stream, f)
+                                         : launch_pdl(rows_kernel<false, true>, grid, kRowThreads, stream, f);
+  if (e != cudaSuccess)
+    return set_error(SV_ERR_CUDA, "shard row kernel launch failed: %s", cudaGetErrorString(e));
+  return check_launch("shard statistics");
+}
+
+int launch_shard_decide(const void* target, const void* draft, const int32_t* tokens,
+                        const float* temps, int B, int gamma, int V, int v0, int Vs, int dtype,
+                        const void* all_stats, int nshards, uint64_t seed, uint64_t step,
+                        int32_t* out_accept_len, int32_t* out_tokens, float* out_lp,
+                        float* out_lq, void* out_candidate, void* workspace, const Layout& lay,
+                        cudaStream_t stream) {
+  SingleParams f{};
+  int rc = shard_params(f, target, draft, tokens, temps, B, gamma, V, v0, Vs, dtype, seed, step,
+                        out_accept_len, out_tokens, out_lp, out_lq, workspace, lay);
+  if (rc != SV_OK) return rc;
+  f.cand = static_cast<ShardCand*>(out_candidate);
+  ShardDecideParams d{};
+  d.p = f.p1;
+  d.p.V = V;  // the decision checks draft tokens against the full vocabulary
+  d.stats = static_cast<const float4*>(all_stats);
+  d.nshards = nshards;
+  d.ready = f.ready;
+  const bool bf16 = dtype == SV_BF16;
+  cudaError_t e = bf16 ? launch_pdl(shard_decide_kernel<true>, dim3(B), kRowThreads, stream, d)
+                       : launch_pdl(shard_decide_kernel<false>, dim3(B), kRowThreads, stream, d);
+  if (e != cudaSuccess)
+    return set_error(SV_ERR_CUDA, "shard decide kernel launch failed: %s", cudaGetErrorString(e));
+  const dim3 grid2(static_cast<unsigned>(static_cast<long long>(B) * f.nc2));
+  e = bf16 ? launch_pdl(draw_kernel<true, true>, grid2, kDrawThreads, stream, f)
+           : launch_pdl(draw_kernel<false, true>, grid2, kDrawThreads, stream, f);
+  if (e != cudaSuccess)
+    return set_error(SV_ERR_CUDA, "shard draw kernel launch failed: %s", cudaGetErrorString(e));
+  return check_launch("shard decide");
+}
+
+int launch_shard_pick(const void* all_candidates, int nshards, int B, int gamma,
+                      int32_t* out_accept_len, int32_t* out_tokens, cudaStream_t stream) {
+  shard_pick_kernel<<<(B + 255) / 256, 256, 0, stream>>>(static_cast<const ShardCand*>(all_candidates),
+                                                        nshards, B, gamma, out_accept_len, out_tokens);
+  return check_launch("shard pick");
 }
 
 }  // namespace sv

@@ -89,3 +89,38 @@ def test_noalloc_reports_bad_shapes_before_any_device_setup():
     rc = L.spec_verify_noalloc(None, None, None, None, 1, 4, 100, 9, 0, 0, None, None, None,
                                None, None)
     assert rc == 1 and b"dtype" in L.spec_verify_last_error()
+
+
+def test_shard_sizes_and_host_side_checks():
+    """Vocabulary shards: record sizes, and the shard rules checked on the
+    host before any CUDA call (the pointers below are never dereferenced)."""
+    L = sv.lib()
+    assert sv.shard_stats_bytes(4, 3) == 4 * 4 * 48
+    assert sv.shard_candidate_bytes(5) == 5 * 32
+    assert sv.shard_stats_bytes(1, 0) == 0 and sv.shard_candidate_bytes(-1) == 0
+    fake = ctypes.c_void_p(1 << 20)
+    ws_bytes = 1 << 30
+
+    def stats(V, v0, Vs):
+        return L.spec_verify_shard_stats(fake, fake, fake, fake, 2, 3, V, v0, Vs, sv.BF16, fake,
+                                         fake, ws_bytes, None)
+
+    assert stats(5000, 100, 2048) == 1
+    assert b"multiple of 1024" in L.spec_verify_last_error()
+    assert stats(5000, 0, 1000) == 1
+    assert b"every shard but the last" in L.spec_verify_last_error()
+    assert stats(5000, 4096, 1000) == 1
+    assert b"must lie in" in L.spec_verify_last_error()
+    assert L.spec_verify_shard_pick(fake, 0, 2, 3, fake, fake, None) == 1
+    assert b"nshards" in L.spec_verify_last_error()
+    assert L.spec_verify_shard_pick(None, 1, 0, 3, None, None, None) == 0  # B = 0: nothing to do
+
+
+def test_vocab_shards_cover_the_vocabulary():
+    for V, n in ((32000, 2), (32000, 3), (151936, 8), (128256, 4), (5000, 3), (1024, 1),
+                 (1025, 2)):
+        b = sv.vocab_shards(V, n)
+        assert len(b) == n and b[0][0] == 0
+        for (v0, Vs), (v1, _) in zip(b, b[1:]):
+            assert v0 % sv.SHARD_ALIGN == 0 and Vs % sv.SHARD_ALIGN == 0 and v0 + Vs == v1
+        assert b[-1][0] + b[-1][1] == V and b[-1][0] % sv.SHARD_ALIGN == 0

@@ -72,3 +72,36 @@ def test_two_rank_reductions_and_shards(world):
     solo = oracle.verify(tg, dr, tok, tm, seed=0, step=0)
     assert out[0][2][0][1] == solo["tokens"].tolist()
     assert np.array_equal(np.array(out[1][2][0][1]), solo["tokens"])
+
+
+def _gather_main(rank, world, port, out):
+    os.environ.update(RANK=str(rank), WORLD_SIZE=str(world), LOCAL_RANK=str(rank),
+                      MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import torch
+    import torch.distributed as dist
+
+    import speculative_decoding_verification_85_b200 as sv
+
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    local = torch.arange(48, dtype=torch.uint8) + 100 * rank
+    got = sv.gather_records(local)
+    dist.destroy_process_group()
+    out[rank] = got.tolist()
+
+
+def test_vocab_shard_exchange_is_rank_ordered():
+    """The exchange between the vocabulary-shard calls: every rank receives
+    all ranks' records concatenated in rank order (two gloo ranks on CPU)."""
+    world = 2
+    ctx = mp.get_context("spawn")
+    mgr = ctx.Manager()
+    out = mgr.dict()
+    port = _free_port()
+    procs = [ctx.Process(target=_gather_main, args=(r, world, port, out)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=180)
+    assert all(p.exitcode == 0 for p in procs)
+    want = list(range(48)) + [100 + i for i in range(48)]
+    assert out[0] == want and out[1] == want
