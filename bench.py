@@ -517,6 +517,144 @@ def run_ours(args, cfg):
         dist.destroy_process_group()
 
 
+def run_vocab_shards(args, cfg):
+    """--vocab-shards n: the vocabulary-sharded path as rank 0 of n runs it,
+    on one GPU.  Rank 0's three calls (shard statistics, decision and shard
+    race, pick) on its 1/n of every row are timed; the other ranks' records
+    are computed once per input set before timing and sit in their slots of
+    the two exchange buffers, which rank 0 fills in place (so the two
+    all-gathers of an n-GPU run are not in the timed region).  Each input set
+    is verified with a fixed step value, so every timed step repeats the
+    setup's computation and its outputs are checked against the unsharded
+    path."""
+    import dataclasses
+
+    import speculative_decoding_verification_85_b200 as sv
+
+    world, rank, local = _dist_init()
+    if world != 1:
+        raise SystemExit("--vocab-shards times one emulated rank on one GPU")
+    if cfg.multidraft:
+        raise SystemExit("--vocab-shards: single-draft workloads only")
+    n = args.vocab_shards
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    K, W = args.steps, args.warmup
+    B, g, V = cfg.B, cfg.gamma, cfg.V
+    dt = sv.BF16 if cfg.dtype == "bf16" else sv.F32
+    es = 2 if cfg.dtype == "bf16" else 4
+    bounds = sv.vocab_shards(V, n)
+    v00, Vs0 = bounds[0]
+    shard_set_bytes = B * (2 * g + 1) * Vs0 * es
+    R = args.sets if args.sets else max(ring_size(cfg), -(-4 * L2_BYTES // shard_set_bytes))
+    rec, crec = sv.shard_stats_bytes(B, g), sv.shard_candidate_bytes(B)
+    wss = [torch.zeros(sv.workspace_size(B, g, Vs, dt), dtype=torch.uint8, device=dev)
+           for _, Vs in bounds]
+    stream = torch.cuda.Stream(device=dev)
+    sets, differ = [], 0
+    with torch.cuda.stream(stream):
+        for k in range(R):
+            st = workloads.make_step(cfg, k, device=dev)
+            sl = [(v0, st.target[:, :, v0:v0 + Vs].contiguous(),
+                   st.draft[:, :, v0:v0 + Vs].contiguous()) for v0, Vs in bounds]
+            all_stats = torch.empty(n * rec, dtype=torch.uint8, device=dev)
+            all_cands = torch.empty(n * crec, dtype=torch.uint8, device=dev)
+            acc = torch.empty(B, dtype=torch.int32, device=dev)
+            tok = torch.empty((B, g + 1), dtype=torch.int32, device=dev)
+            for r, (v0, t, d) in enumerate(sl):
+                sv.spec_verify_shard_stats(t, d, st.tokens, st.temps, V=V, v0=v0, workspace=wss[r],
+                                           out_stats=all_stats[r * rec:(r + 1) * rec],
+                                           stream=stream)
+            for r, (v0, t, d) in enumerate(sl):
+                a_r = acc if r == 0 else torch.empty_like(acc)
+                t_r = tok if r == 0 else torch.empty_like(tok)
+                sv.spec_verify_shard_decide(t, d, st.tokens, st.temps, all_stats, V=V, v0=v0,
+                                            nshards=n, workspace=wss[r], seed=0, step=k,
+                                            out_accept_len=a_r, out_tokens=t_r,
+                                            out_candidate=all_cands[r * crec:(r + 1) * crec],
+                                            stream=stream)
+            sv.spec_verify_shard_pick(all_cands, nshards=n, out_accept_len=acc, out_tokens=tok,
+                                      stream=stream)
+            a1, t1, _, _ = sv.spec_verify(st.target, st.draft, st.tokens, st.temps, seed=0,
+                                          step=k, stream=stream)
+            stream.synchronize()
+            differ += int(((a1 != acc) | (t1 != tok).any(dim=1)).sum())
+            sets.append((sl[0][1], sl[0][2], st.tokens, st.temps, all_stats, all_cands, acc, tok))
+            del st, sl
+    torch.cuda.empty_cache()
+
+    def one(i: int):
+        k = i % R
+        t, d, x, temps, all_stats, all_cands, acc, tok = sets[k]
+        sv.spec_verify_shard_stats(t, d, x, temps, V=V, v0=v00, workspace=wss[0],
+                                   out_stats=all_stats[:rec], stream=stream)
+        sv.spec_verify_shard_decide(t, d, x, temps, all_stats, V=V, v0=v00, nshards=n,
+                                    workspace=wss[0], seed=0, step=k, out_accept_len=acc,
+                                    out_tokens=tok, out_candidate=all_cands[:crec], stream=stream)
+        sv.spec_verify_shard_pick(all_cands, nshards=n, out_accept_len=acc, out_tokens=tok,
+                                  stream=stream)
+
+    with torch.cuda.stream(stream):
+        for i in range(W):
+            one(i)
+    stream.synchronize()
+    from torch.profiler import ProfilerActivity, profile
+    with profile(activities=[ProfilerActivity.CUDA]) as prof:
+        with torch.cuda.stream(stream):
+            one(W)
+        stream.synchronize()
+    step_kernels = [e.name.split("(")[0].split("<")[0].replace("void ", "").replace("sv::", "")
+                    for e in prof.events()
+                    if e.device_type == torch.autograd.DeviceType.CUDA and "sv::" in e.name]
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        for i in range(W, W + K):
+            one(i)
+    with torch.cuda.stream(stream):
+        graph.replay()
+    stream.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(gpu_ident(dev)) as clk:
+        t_end = time.time() + args.soak
+        while time.time() < t_end:
+            with torch.cuda.stream(stream):
+                graph.replay()
+            stream.synchronize()
+        torch.cuda.synchronize(dev)
+        with torch.cuda.stream(stream):
+            ev0.record(stream)
+            graph.replay()
+            ev1.record(stream)
+        torch.cuda.synchronize(dev)
+    ms = ev0.elapsed_time(ev1)
+    # rank 0's algorithmic bytes: its slice of every needed row and draw row
+    scfg = dataclasses.replace(cfg, V=Vs0)
+    algo = int(round(sum(step_bytes(scfg, s_[3], s_[6])["algorithmic"] for s_ in sets) / R))
+    gbs = algo / (ms / K / 1e3) / 1e9
+    peak, peak_kind = _peaks()
+    line = {
+        "metric": METRIC, "value": cfg.rows_per_step * K / (ms / 1e3), "unit": UNIT,
+        "n_gpus": 1, "steps": K, "warmup": W, "ms_per_step": ms / K, "higher_is_better": True,
+        "scaling": "strong", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": cfg.name, "vocab_shards": n, "rank": 0, "shard": [v00, Vs0],
+                   "timed": "rank 0's three calls on its 1/n of every row; the other ranks' "
+                            "records gathered before timing (the two all-gathers are not "
+                            "timed: one GPU)",
+                   "inputs": f"ring of {R} input sets ({R * shard_set_bytes / 1e9:.2f} GB of "
+                             f"rank 0's rows, {R * shard_set_bytes / L2_BYTES:.1f}x L2)",
+                   "launch": "K steps captured in one CUDA graph, replayed"},
+        "roofline": {"bound": "hbm", "kernel": " + ".join(dict.fromkeys(step_kernels)),
+                     "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
+                     "traffic": None, "peak_source": peak_kind,
+                     "algorithmic_bytes_per_launch": algo},
+        "gpu_launches": K * len(step_kernels), "clocks": clk.summary(), "e2e": None,
+        "cpu_baseline": None,
+        "check": {"sequences": R * B, "differ_from_unsharded": differ},
+    }
+    print(json.dumps(line), flush=True)
+    del graph
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -534,6 +672,9 @@ def main():
                          "(small profiling captures; not a bench line)")
     ap.add_argument("--sets", type=int, default=None,
                     help="distinct input sets in the ring (default: at least 4x L2)")
+    ap.add_argument("--vocab-shards", type=int, default=None,
+                    help="time rank 0 of this many vocabulary shards on one GPU (not the "
+                         "bench line)")
     args = ap.parse_args()
     cfg = workloads.get(args.config)
     if args.batch is not None and args.batch != cfg.B:
@@ -546,6 +687,8 @@ def main():
         args.warmup = 3
     if args.impl == "reference":
         run_reference(args, cfg)
+    elif args.vocab_shards:
+        run_vocab_shards(args, cfg)
     else:
         run_ours(args, cfg)
 

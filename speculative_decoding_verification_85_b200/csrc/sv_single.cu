@@ -61,6 +61,8 @@ struct SingleParams {
   int vfull;
   float4* xstats;       // [B][gamma + 1][3]
   ShardCand* cand;      // [B]
+  const float4* allstats;  // [nshards][B][gamma + 1][3]: the gathered records
+  int nshards;
 };
 
 template <bool kBf16>
@@ -618,29 +620,100 @@ __device__ __forceinline__ bool wait_ready(const unsigned* flag) {
   }
 }
 
-// kShard: the rows are one vocabulary shard; the race runs over the shard's
-// groups with global group and entry indices, and the completing CTA writes
-// the shard's candidate (its best group with that group's level-2 winner, or,
-// where the shard's residual has no weight, the same for the race over p_j)
-// instead of the token.
+// ------------------------------------------------- vocabulary shards: decide
+// Merge the gathered shards' records of sequence b into the row table rows[]
+// (target rows 0..gamma, then draft rows) and the draft tokens' logits
+// zsel[]: a warp per position, lane r merging rank r's record, then a
+// butterfly -- the same order on every rank, so every rank reaches the same
+// bits.  All kDrawThreads threads; ends with a barrier.
+__device__ __forceinline__ void merge_shards(const SingleParams& f, int b, bool argmaxA, float c,
+                                             RowAcc* rows, float* zsel) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int g = f.p1.gamma;
+  const size_t per_rank = static_cast<size_t>(f.p1.B) * (g + 1) * 3;  // float4s in one record
+  for (int i = warp; i <= g; i += kDrawThreads / 32) {
+    RowAcc A = argmaxA ? empty_argmax_acc() : empty_lse_acc(), Bq = empty_lse_acc();
+    float zt = __int_as_float(0x7fc00000), zd = zt;
+    for (int r = lane; r < f.nshards; r += 32) {
+      const float4* o = f.allstats + r * per_rank + (static_cast<size_t>(b) * (g + 1) + i) * 3;
+      const float4 a = __ldcg(o), d = __ldcg(o + 1), z = __ldcg(o + 2);
+      merge_ref(A, RowAcc{a.x, a.y, __float_as_int(a.z), __float_as_int(a.w)}, argmaxA);
+      merge_ref(Bq, RowAcc{d.x, d.y, __float_as_int(d.z), __float_as_int(d.w)}, false);
+      if (z.x == z.x) zt = z.x;  // the one shard that holds the draft token reports its logits
+      if (z.y == z.y) zd = z.y;
+    }
+    warp_merge(A, argmaxA);
+    warp_merge(Bq, false);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      const float a = __shfl_xor_sync(0xffffffffu, zt, off);
+      const float d = __shfl_xor_sync(0xffffffffu, zd, off);
+      if (zt != zt) zt = a;
+      if (zd != zd) zd = d;
+    }
+    if (lane == 0) {
+      if (!argmaxA) A.s = sum_rel_max(A, c);
+      Bq.s = sum_rel_max(Bq, c);
+      rows[i] = A;
+      if (i < g) {
+        rows[g + 1 + i] = Bq;
+        zsel[2 * i] = zt;
+        zsel[2 * i + 1] = zd;
+      }
+    }
+  }
+  block_sync<kDrawThreads>();
+}
+
+// kShard: the rows are one vocabulary shard; every CTA first takes its
+// sequence's decision from the gathered shards' records, the race runs over
+// the shard's groups with global group and entry indices, and the completing
+// CTA writes the shard's candidate (its best group with that group's level-2
+// winner, or, where the shard's residual has no weight, the same for the race
+// over p_j) instead of the token.
 template <bool kBf16, bool kShard = false>
 __global__ void __launch_bounds__(kDrawThreads, 4) draw_kernel(const __grid_constant__ SingleParams f) {
   __shared__ float4 scratch[kDrawThreads / 32];
   __shared__ int s_last, s_ready;
-  // No griddepcontrol.wait: this grid may start while the row kernel's last
-  // CTAs still run, and each CTA waits for its own sequence's decision flag
-  // instead.  (It starts only once every row-kernel CTA has started, so the
-  // row kernel never waits for SM room held by this grid.)
-  asm volatile("griddepcontrol.launch_dependents;");
+  // Whole rows: no griddepcontrol.wait -- this grid may start while the row
+  // kernel's last CTAs still run, and each CTA waits for its own sequence's
+  // decision flag instead.  (It starts only once every row-kernel CTA has
+  // started, so the row kernel never waits for SM room held by this grid.)
   const int b = blockIdx.x / f.nc2;
   const int chunk = blockIdx.x - b * f.nc2;
   const int warp = threadIdx.x >> 5;
   const CallParams& p = f.p1;
-  if (threadIdx.x == 0) s_ready = wait_ready(f.ready + b) ? 1 : 0;
-  block_sync<kDrawThreads>();  // orders the other threads after thread 0's acquire
   SeqInfo si{};
   si.mode = kModeNone;
-  if (s_ready) {
+  if constexpr (kShard) {
+    // Vocabulary shards: every CTA of the sequence takes the decision from
+    // the gathered records (no wait on another CTA); chunk 0 writes the
+    // outputs.  The records may come from the previous grid in the stream.
+    __shared__ RowAcc rows[kMaxRowsPerSeq];
+    __shared__ float s_zsel[2 * SV_MAX_GAMMA];
+    __shared__ int s_tok[SV_MAX_GAMMA];
+    __shared__ CallParams s_p;
+    __shared__ SeqInfo s_si;
+    pdl_wait_and_release();
+    const float T = __ldg(p.temps + b);
+    const int modeA = row_mode(T, true);
+    const float c = modeA == kRowLse ? __fdiv_rn(kLog2e, T) : 0.0f;
+    for (int k = threadIdx.x; k < p.gamma; k += kDrawThreads)
+      s_tok[k] = __ldg(p.tokens + static_cast<size_t>(b) * p.gamma + k);
+    if (threadIdx.x == 0) {
+      s_p = p;
+      s_p.V = f.vfull;  // draft tokens are checked against the full vocabulary
+    }
+    merge_shards(f, b, modeA == kRowArgmax, c, rows, s_zsel);
+    if (warp == 0) decide_single<kBf16>(s_p, b, T, s_tok, rows, s_zsel, &s_si, chunk == 0, nullptr);
+    block_sync<kDrawThreads>();
+    si = s_si;
+  } else {
+    asm volatile("griddepcontrol.launch_dependents;");
+    if (threadIdx.x == 0) s_ready = wait_ready(f.ready + b) ? 1 : 0;
+    block_sync<kDrawThreads>();  // orders the other threads after thread 0's acquire
+  }
+  if (!kShard && s_ready) {
     const float4* ip = reinterpret_cast<const float4*>(p.info + b);
     const float4 w0 = __ldcg(ip), w1 = __ldcg(ip + 1);
     si.mode = __float_as_int(w0.x);
@@ -650,7 +723,7 @@ __global__ void __launch_bounds__(kDrawThreads, 4) draw_kernel(const __grid_cons
     si.c = w1.x;
     si.lsp = w1.y;
     si.lsq = w1.z;
-  } else if (chunk == 0) {
+  } else if (!kShard && chunk == 0) {
     // the decision never came (a wait ran out of time): no result
     for (int i = threadIdx.x; i <= p.gamma; i += kDrawThreads)
       p.out_tokens[static_cast<size_t>(b) * (p.gamma + 1) + i] = -1;
@@ -729,108 +802,63 @@ __global__ void __launch_bounds__(kDrawThreads, 4) draw_kernel(const __grid_cons
   }
 }
 
-// ------------------------------------------------- vocabulary shards: decide
-// Sequence inputs of the decision over all shards' records.
-struct ShardDecideParams {
-  CallParams p;          // V: the full vocabulary (draft-token validity)
-  const float4* stats;   // [nshards][B][gamma + 1][3]: the gathered records
-  int nshards;
-  unsigned* ready;       // [B] decision published (cleared by the draw kernel)
-};
+// --------------------------------------------------- vocabulary shards: pick
+constexpr int kPickThreads = 256;
 
-// One CTA per sequence: merge the shards' records of every position (a warp
-// per position, lane r merging rank r's record, then a butterfly: the same
-// order on every rank, so every rank reaches the same bits), then the
-// decision, published to the draw kernel by the sequence's flag.
-template <bool kBf16>
-__global__ void __launch_bounds__(kRowThreads) shard_decide_kernel(const __grid_constant__ ShardDecideParams f) {
-  __shared__ RowAcc rows[kMaxRowsPerSeq];
-  __shared__ float s_zsel[2 * SV_MAX_GAMMA];
-  __shared__ int s_tok[SV_MAX_GAMMA];
-  pdl_wait_and_release();
-  const CallParams& p = f.p;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int b = blockIdx.x;
-  const int g = p.gamma;
-  const float T = __ldg(p.temps + b);
-  const int modeA = row_mode(T, true);
-  const bool argmaxA = modeA == kRowArgmax;
-  const float c = modeA == kRowLse ? __fdiv_rn(kLog2e, T) : 0.0f;
-  for (int k = tid; k < g; k += kRowThreads) s_tok[k] = __ldg(p.tokens + static_cast<size_t>(b) * g + k);
-  const size_t per_rank = static_cast<size_t>(p.B) * (g + 1) * 3;  // float4s in one rank's record
-  for (int i = warp; i <= g; i += kRowThreads / 32) {
-    RowAcc A = argmaxA ? empty_argmax_acc() : empty_lse_acc(), Bq = empty_lse_acc();
-    float zt = __int_as_float(0x7fc00000), zd = zt;
-    for (int r = lane; r < f.nshards; r += 32) {
-      const float4* o = f.stats + r * per_rank + (static_cast<size_t>(b) * (g + 1) + i) * 3;
-      const float4 a = __ldcg(o), d = __ldcg(o + 1), z = __ldcg(o + 2);
-      merge_ref(A, RowAcc{a.x, a.y, __float_as_int(a.z), __float_as_int(a.w)}, argmaxA);
-      merge_ref(Bq, RowAcc{d.x, d.y, __float_as_int(d.z), __float_as_int(d.w)}, false);
-      if (z.x == z.x) zt = z.x;  // the one shard that holds the draft token reports its logits
-      if (z.y == z.y) zd = z.y;
-    }
-    warp_merge(A, argmaxA);
-    warp_merge(Bq, false);
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-      const float a = __shfl_xor_sync(0xffffffffu, zt, off);
-      const float d = __shfl_xor_sync(0xffffffffu, zd, off);
-      if (zt != zt) zt = a;
-      if (zd != zd) zd = d;
-    }
-    if (lane == 0) {
-      if (!argmaxA) A.s = sum_rel_max(A, c);
-      Bq.s = sum_rel_max(Bq, c);
-      rows[i] = A;
-      if (i < g) {
-        rows[g + 1 + i] = Bq;
-        s_zsel[2 * i] = zt;
-        s_zsel[2 * i + 1] = zd;
-      }
-    }
-  }
-  block_sync<kRowThreads>();
-  if (tid < 32) {
-    decide_single<kBf16>(p, b, T, s_tok, rows, s_zsel, p.info + b, true, nullptr);
-    __threadfence();
-    __syncwarp();
-    if (tid == 0) st_release(f.ready + b, 1u);
+// The better of two candidates of one kind (exponential race: larger w / E,
+// lower group on ties), the token travelling with its group.
+__device__ __forceinline__ void pick_better(float& bw, float& be, int& bg, int& bt, float w, float e,
+                                            int grp, int t) {
+  if (race_better(w, e, grp, bw, be, bg)) {
+    bw = w;
+    be = e;
+    bg = grp;
+    bt = t;
   }
 }
 
-// --------------------------------------------------- vocabulary shards: pick
-// One thread per sequence: the winning candidate over the gathered shards'
-// candidates (the draw law's when any shard has weight in it, else the race
-// over p_j), written at the draw position.  Shards that disagree on the draw
-// (a rank whose wait ran out reports none) mark the sequence invalid.
-__global__ void __launch_bounds__(256) shard_pick_kernel(const ShardCand* all, int nshards, int B,
-                                                          int gamma, int32_t* accept_len,
-                                                          int32_t* out_tokens) {
+// One warp per sequence, lane r reading rank r's candidate (and r + 32, ...):
+// the winning candidate over the gathered shards' candidates (the draw law's
+// when any shard has weight in it, else the race over p_j), written at the
+// draw position.  Shards that disagree on the draw (a rank whose wait ran out
+// reports none) mark the sequence invalid.
+__global__ void __launch_bounds__(kPickThreads) shard_pick_kernel(const ShardCand* all, int nshards, int B,
+                                                                   int gamma, int32_t* accept_len,
+                                                                   int32_t* out_tokens) {
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  const int b = static_cast<int>(blockIdx.x * blockDim.x + threadIdx.x);
-  if (b >= B) return;
+  const int lane = threadIdx.x & 31;
+  const int b = static_cast<int>(blockIdx.x) * (kPickThreads / 32) + static_cast<int>(threadIdx.x >> 5);
+  if (b >= B) return;  // uniform over the warp
   const ShardCand c0 = all[b];
   float bw[2] = {0.0f, 0.0f}, be[2] = {1.0f, 1.0f};
-  int bi[2] = {INT_MAX, INT_MAX}, bt[2] = {-1, -1};
+  int bg[2] = {INT_MAX, INT_MAX}, bt[2] = {-1, -1};
   bool agree = true;
-  for (int r = 0; r < nshards; ++r) {
+  for (int r = lane; r < nshards; r += 32) {
     const ShardCand c = all[static_cast<size_t>(r) * B + b];
     agree = agree && (c.kind == kShardNoDraw) == (c0.kind == kShardNoDraw) && c.j == c0.j;
+    if (c.kind == kShardNoDraw) continue;
     const int k = c.kind == kShardTargetRace ? 1 : 0;
-    if (c.kind != kShardNoDraw && race_better(c.w, c.e, c.group, bw[k], be[k], bi[k])) {
-      bw[k] = c.w;
-      be[k] = c.e;
-      bi[k] = c.group;
-      bt[k] = c.token;
+    pick_better(bw[k], be[k], bg[k], bt[k], c.w, c.e, c.group, c.token);
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const float w = __shfl_xor_sync(0xffffffffu, bw[k], off);
+      const float e = __shfl_xor_sync(0xffffffffu, be[k], off);
+      const int grp = __shfl_xor_sync(0xffffffffu, bg[k], off);
+      const int t = __shfl_xor_sync(0xffffffffu, bt[k], off);
+      pick_better(bw[k], be[k], bg[k], bt[k], w, e, grp, t);
     }
   }
+  agree = __all_sync(0xffffffffu, agree);
   int32_t* tok = out_tokens + static_cast<size_t>(b) * (gamma + 1);
   if (!agree) {
-    for (int i = 0; i <= gamma; ++i) tok[i] = -1;
-    accept_len[b] = -1;
+    for (int i = lane; i <= gamma; i += 32) tok[i] = -1;
+    if (lane == 0) accept_len[b] = -1;
     return;
   }
-  if (c0.kind == kShardNoDraw || c0.j < 0 || c0.j > gamma) return;
+  if (lane != 0 || c0.kind == kShardNoDraw || c0.j < 0 || c0.j > gamma) return;
   tok[c0.j] = bw[0] > 0.0f ? bt[0] : bt[1];
 }
 
@@ -1029,6 +1057,10 @@ int shard_params(SingleParams& f, const void* target, const void* draft, const i
   set_call(f.p1, target, draft, tokens, temps, B, gamma, Vs, seed, step, out_accept_len, out_tokens,
            out_lp, out_lq, ws, lay);
   set_policy(f, B, gamma, Vs, dtype, ws, lay);
+  // a shard's rows are short: one segment per row when they span at most four
+  // tiles (fewer, longer CTAs; measured 56 against 66 us for rank 0 of 8 on
+  // 256 x 5 rows of 151936 bf16 entries)
+  if (f.tiles <= 4) f.nseg = 1;
   f.voff = v0;
   f.vfull = V;
   if (static_cast<long long>(B) * f.nc2 > INT_MAX ||
@@ -1065,20 +1097,11 @@ int launch_shard_decide(const void* target, const void* draft, const int32_t* to
                         out_accept_len, out_tokens, out_lp, out_lq, workspace, lay);
   if (rc != SV_OK) return rc;
   f.cand = static_cast<ShardCand*>(out_candidate);
-  ShardDecideParams d{};
-  d.p = f.p1;
-  d.p.V = V;  // the decision checks draft tokens against the full vocabulary
-  d.stats = static_cast<const float4*>(all_stats);
-  d.nshards = nshards;
-  d.ready = f.ready;
-  const bool bf16 = dtype == SV_BF16;
-  cudaError_t e = bf16 ? launch_pdl(shard_decide_kernel<true>, dim3(B), kRowThreads, stream, d)
-                       : launch_pdl(shard_decide_kernel<false>, dim3(B), kRowThreads, stream, d);
-  if (e != cudaSuccess)
-    return set_error(SV_ERR_CUDA, "shard decide kernel launch failed: %s", cudaGetErrorString(e));
+  f.allstats = static_cast<const float4*>(all_stats);
+  f.nshards = nshards;
   const dim3 grid2(static_cast<unsigned>(static_cast<long long>(B) * f.nc2));
-  e = bf16 ? launch_pdl(draw_kernel<true, true>, grid2, kDrawThreads, stream, f)
-           : launch_pdl(draw_kernel<false, true>, grid2, kDrawThreads, stream, f);
+  const cudaError_t e = dtype == SV_BF16 ? launch_pdl(draw_kernel<true, true>, grid2, kDrawThreads, stream, f)
+                                         : launch_pdl(draw_kernel<false, true>, grid2, kDrawThreads, stream, f);
   if (e != cudaSuccess)
     return set_error(SV_ERR_CUDA, "shard draw kernel launch failed: %s", cudaGetErrorString(e));
   return check_launch("shard decide");
@@ -1086,8 +1109,9 @@ int launch_shard_decide(const void* target, const void* draft, const int32_t* to
 
 int launch_shard_pick(const void* all_candidates, int nshards, int B, int gamma,
                       int32_t* out_accept_len, int32_t* out_tokens, cudaStream_t stream) {
-  shard_pick_kernel<<<(B + 255) / 256, 256, 0, stream>>>(static_cast<const ShardCand*>(all_candidates),
-                                                        nshards, B, gamma, out_accept_len, out_tokens);
+  constexpr int kPerBlock = kPickThreads / 32;  // sequences per CTA
+  shard_pick_kernel<<<(B + kPerBlock - 1) / kPerBlock, kPickThreads, 0, stream>>>(
+      static_cast<const ShardCand*>(all_candidates), nshards, B, gamma, out_accept_len, out_tokens);
   return check_launch("shard pick");
 }
 
