@@ -25,6 +25,13 @@
 // The row kernel waits on no other CTA (arrival tickets only); a draw CTA
 // waits, with a time limit, for one flag that a row-kernel CTA already
 // running sets.
+// Vocabulary shards (the kShard instantiations): the row kernel runs on one
+// shard's columns and its completing CTA exports the shard's merged row
+// statistics; after the caller's all-gather, every draw CTA merges all
+// shards' records and decides, the race runs over the shard's groups with
+// global Philox keys, and the completing CTA exports the shard's candidate;
+// after a second all-gather a pick kernel takes the winner.  No wait on
+// another CTA in that path.
 #include <atomic>
 #include <climits>
 
