@@ -265,7 +265,7 @@ __device__ __forceinline__ void pick_logit(const uint4 (&r)[kTileRegs], int own,
 // shard (columns [voff, voff + V) of vfull), and the CTA that completes a
 // sequence writes the shard's record instead of deciding.
 template <bool kBf16, bool kShard = false>
-__global__ void __launch_bounds__(kRowThreads, 3) rows_kernel(const __grid_constant__ SingleParams f) {
+__global__ void __launch_bounds__(kRowThreads, 4) rows_kernel(const __grid_constant__ SingleParams f) {
   __shared__ RowAcc rows[kMaxRowsPerSeq];
   __shared__ RowAcc scratch[2 * (kRowThreads / 32)];
   __shared__ float s_zx[2];
@@ -927,8 +927,8 @@ int occupancy(Kernel kernel, int threads) {
 // Resident row-kernel CTAs per SM.
 int row_ctas_per_sm(bool bf16) {
   static std::atomic<int> slots[2][64];
-  return bf16 ? per_device(slots[1], 3, [](int) { return occupancy(rows_kernel<true>, kRowThreads); })
-              : per_device(slots[0], 3, [](int) { return occupancy(rows_kernel<false>, kRowThreads); });
+  return bf16 ? per_device(slots[1], 4, [](int) { return occupancy(rows_kernel<true>, kRowThreads); })
+              : per_device(slots[0], 4, [](int) { return occupancy(rows_kernel<false>, kRowThreads); });
 }
 
 // Resident draw-kernel CTAs per SM.
@@ -961,15 +961,16 @@ cudaError_t launch_pdl(K kernel, dim3 grid, unsigned block, cudaStream_t stream,
 // Row segments: whole tiles, about kRowWaves waves of CTAs over the GPU but
 // at most kMaxSegTiles tiles per CTA; balanced so segments differ by at most
 // one tile.  Long segments spread each CTA's fixed cost (launch, block
-// reduce, ticket) over more streaming; about three waves keep the last one
-// mostly full.  Draw CTAs: race groups per warp chosen so that the B
+// reduce, ticket) over more streaming; about two waves of four CTAs per SM
+// (64 registers a thread) measured best (C2 76.2 us against 83.3 at four
+// waves and 77.4 at three).  Draw CTAs: race groups per warp chosen so that the B
 // sequences' groups fill about kDrawWaves waves of CTAs (at least one group
 // per warp, so a small batch still spreads each row over several CTAs); a
 // CTA covers 8 warps' groups.  V is the width of the rows the kernels read.
 void set_policy(SingleParams& f, int B, int gamma, int V, int dtype, char* ws, const Layout& lay) {
   const bool bf16 = dtype == SV_BF16;
   {
-    constexpr int kRowWaves = 3, kMaxSegTiles = 10;
+    constexpr int kRowWaves = 2, kMaxSegTiles = 10;
     const int tiles = body_tiles(V, dtype);
     const long long pairs = static_cast<long long>(B) * (gamma + 1);
     const long long slots = static_cast<long long>(sm_count()) * row_ctas_per_sm(bf16);

@@ -203,3 +203,32 @@ def test_shard_argument_errors():
         sv.spec_verify_shard_stats(t, d, st.tokens, st.temps, V=V, v0=0, workspace=ws)
     with pytest.raises(sv.SpecVerifyError, match="must lie in"):
         sv.spec_verify_shard_stats(t, d, st.tokens, st.temps, V=V, v0=4096, workspace=ws)
+
+
+def test_vocab_sharded_through_a_process_group_of_one():
+    """spec_verify_vocab_sharded with its all-gathers on a real NCCL process
+    group (one rank: the whole row is its shard)."""
+    import socket
+
+    import torch.distributed as dist
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0,
+                            world_size=1, device_id=torch.device(DEV))
+    try:
+        st = workloads.make_custom(6, 4, 7000, dtype="bf16", seed=44, T=[0.0, 0.7, 1.0],
+                                   device=DEV)
+        led = TieLedger("vocab-sharded through NCCL, one rank")
+        for step in range(2):
+            acc, tok, lp, lq = sv.spec_verify_vocab_sharded(st.target, st.draft, st.tokens,
+                                                            st.temps, V=7000, v0=0, seed=2,
+                                                            step=step, with_logprobs=True)
+            torch.cuda.synchronize()
+            got = {"accept_len": acc.cpu().numpy(), "tokens": tok.cpu().numpy(),
+                   "lp": lp.cpu().numpy(), "lq": lq.cpu().numpy()}
+            led.add(compare(got, run_oracle(st, 2, step)))
+        led.check()
+    finally:
+        dist.destroy_process_group()
