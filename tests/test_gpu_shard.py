@@ -232,3 +232,35 @@ def test_vocab_sharded_through_a_process_group_of_one():
         led.check()
     finally:
         dist.destroy_process_group()
+
+
+# ------------------------------------------------------------ seeded sweep
+from hypothesis import HealthCheck, given, settings  # noqa: E402
+from hypothesis import strategies as hs  # noqa: E402
+
+_sweep = TieLedger("vocab-sharded sweep")
+
+
+@settings(max_examples=30, deadline=None, derandomize=True, database=None,
+          suppress_health_check=list(HealthCheck))
+@given(B=hs.integers(1, 24), gamma=hs.integers(1, 10), V=hs.integers(1025, 60000),
+       n=hs.integers(1, 6), dtype=hs.sampled_from(["bf16", "f32"]),
+       T=hs.lists(hs.sampled_from([0.0, 0.05, 0.3, 0.7, 1.0, 2.5]), min_size=1, max_size=4),
+       scale=hs.sampled_from([0.5, 2.0, 6.0]), noise=hs.sampled_from([0.0, 0.05, 0.6, 2.0]),
+       seed=hs.integers(0, 2**31 - 1), step=hs.integers(0, 2**32 - 1))
+def test_sharded_sweep(B, gamma, V, n, dtype, T, scale, noise, seed, step):
+    """Shapes, shard counts (shards of whole 1024-entry groups, a ragged
+    last one), dtypes, temperature mixes, logit scales and draft noise drawn
+    by Hypothesis (derandomised): every rank identical, and equal to the
+    oracle on the whole rows."""
+    bounds = [b for b in sv.vocab_shards(V, n) if b[1] > 0]
+    s = workloads.make_custom(B, gamma, V, dtype=dtype, seed=seed, T=T, device=DEV,
+                              target_scale=scale, noise=noise)
+    res = run_sharded(s, len(bounds), seed=seed, step=step, bounds=bounds)
+    same_on_every_rank(res)
+    _sweep.add(compare(res[0], run_oracle(s, seed, step)))
+
+
+def test_sharded_sweep_tie_counts():
+    """Runs after the sweep: its excluded (tie) count stays small."""
+    _sweep.check(max_rate=5e-3, slack=3)
