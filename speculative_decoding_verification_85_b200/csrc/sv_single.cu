@@ -1069,6 +1069,18 @@ int shard_params(SingleParams& f, const void* target, const void* draft, const i
   // tiles (fewer, longer CTAs; measured 56 against 66 us for rank 0 of 8 on
   // 256 x 5 rows of 151936 bf16 entries)
   if (f.tiles <= 4) f.nseg = 1;
+  // Draw CTAs of a shard take their sequence's decision before the race, so
+  // one wave of them: chunks per sequence = draw slots / B, at least one and
+  // at most one per 8 groups (f.nc2 <= lay.nc2).
+  {
+    const long long ng = (Vs + kRaceGroup - 1) / kRaceGroup;
+    const long long slots = static_cast<long long>(sm_count()) * draw_ctas_per_sm(dtype == SV_BF16);
+    const long long maxc = (ng + kDrawThreads / 32 - 1) / (kDrawThreads / 32);
+    long long nc = slots / B;
+    nc = nc < 1 ? 1 : (nc > maxc ? maxc : nc);
+    f.gpc = static_cast<int>((ng + nc - 1) / nc);
+    f.nc2 = static_cast<int>((ng + f.gpc - 1) / f.gpc);
+  }
   f.voff = v0;
   f.vfull = V;
   if (static_cast<long long>(B) * f.nc2 > INT_MAX ||
