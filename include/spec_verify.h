@@ -14,6 +14,8 @@
  *   spec_verify_multidraft "SpecTr-GBV: Multi-Draft Block Verification
  *                          Accelerating Speculative Decoding", Methodology,
  *                          Algorithm 1.
+ *   spec_verify_shard_*    spec_verify for logits split over the vocabulary
+ *                          across ranks (spec_verify_shard.h).
  *
  * Conventions shared by every entry point
  *   - Logit tensors are dense, row-major, contiguous, in device memory, fp32

@@ -104,9 +104,9 @@ int spec_verify_shard_decide(const void* target_shard, const void* draft_shard,
 /* Call 3.  all_candidates: the n candidate arrays of call 2 gathered in
  * rank order (device, 16-byte aligned); out_accept_len [B] and out_tokens
  * [B][gamma + 1] as left by call 2.  Candidates whose ranks disagree on the
- * draw (a rank whose bounded wait ran out writes "no draw") mark the
- * sequence as spec_verify marks invalid data: accept_len -1, tokens -1, on
- * every rank.  Needs no workspace. */
+ * draw (ranks given different sequence inputs, or records gathered in
+ * different orders) mark the sequence as spec_verify marks invalid data:
+ * accept_len -1, tokens -1, on every rank.  Needs no workspace. */
 int spec_verify_shard_pick(const void* all_candidates, int nshards, int B, int gamma,
                            int32_t* out_accept_len, int32_t* out_tokens, void* stream);
 

@@ -827,8 +827,9 @@ __device__ __forceinline__ void pick_better(float& bw, float& be, int& bg, int& 
 // One warp per sequence, lane r reading rank r's candidate (and r + 32, ...):
 // the winning candidate over the gathered shards' candidates (the draw law's
 // when any shard has weight in it, else the race over p_j), written at the
-// draw position.  Shards that disagree on the draw (a rank whose wait ran out
-// reports none) mark the sequence invalid.
+// draw position.  Shards that disagree on the draw (ranks given different
+// sequence inputs, or records gathered in different orders) mark the
+// sequence invalid.
 __global__ void __launch_bounds__(kPickThreads) shard_pick_kernel(const ShardCand* all, int nshards, int B,
                                                                    int gamma, int32_t* accept_len,
                                                                    int32_t* out_tokens) {
