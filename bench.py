@@ -543,7 +543,8 @@ def run_vocab_shards(args, cfg):
     B, g, V = cfg.B, cfg.gamma, cfg.V
     dt = sv.BF16 if cfg.dtype == "bf16" else sv.F32
     es = 2 if cfg.dtype == "bf16" else 4
-    bounds = sv.vocab_shards(V, n)
+    bounds = [b_ for b_ in sv.vocab_shards(V, n) if b_[1] > 0]  # ranks past V hold nothing
+    n = len(bounds)
     v00, Vs0 = bounds[0]
     shard_set_bytes = B * (2 * g + 1) * Vs0 * es
     R = args.sets if args.sets else max(ring_size(cfg), -(-4 * L2_BYTES // shard_set_bytes))
